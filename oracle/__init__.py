@@ -1,0 +1,146 @@
+"""Float64 CPU oracle for the BRA forward pass — TEST INFRASTRUCTURE ONLY.
+
+Only `tests/`, `__graft_entry__.smoke()` and the benchmark's CPU-baseline leg may
+import this package. The CUDA library never calls it, and it imports nothing from
+the CUDA package.
+
+The arithmetic lives in `bra_oracle.c` (plain C, float64, OpenMP over regions),
+compiled with gcc into `liboracle_bra.so` next to it. This module only marshals
+numpy arrays through ctypes.
+
+Every function follows the official BRA code as walked through on
+"BiFormer ... 前向传播过程" (niftyadmin), section "BRA模块", eqs. 4-7, and
+Algorithm 1 as described on bernice.tw ("Bi-Level Routing Attention"). Parity
+pins: see tests/test_oracle_pins.py. No page prints a numeric worked example, so
+no pin compares against printed values; every function is pinned by closed forms,
+library routines on special cases, brute force and invariants instead.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bra_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_bra.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE float64: no fast-math, no reassociation)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fno-fast-math", "-ffp-contract=off", "-shared", "-fPIC",
+             "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        i = ctypes.c_int
+        lib.oracle_route.argtypes = [dp, dp, i, i, i, i, i, i, i, ip, dp, dp]
+        lib.oracle_attend.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i, i, ip, dp]
+        lib.oracle_forward.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i, i, dp, ip, dp]
+        lib.oracle_lce.argtypes = [dp, dp, dp, i, i, i, i, dp]
+        lib.oracle_region_mean.argtypes = [dp, i, i, i, i, i, dp]
+        lib.oracle_check_shape.argtypes = [i] * 7
+        lib.oracle_set_threads.argtypes = [i]
+        for name in ("oracle_route", "oracle_attend", "oracle_forward", "oracle_check_shape",
+                     "oracle_threads"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _d(x) -> np.ndarray:
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _p(x: np.ndarray, t=ctypes.c_double):
+    return x.ctypes.data_as(ctypes.POINTER(t))
+
+
+def threads() -> int:
+    return _load().oracle_threads()
+
+
+def set_threads(t: int) -> None:
+    _load().oracle_set_threads(int(t))
+
+
+def region_mean(x, S: int) -> np.ndarray:
+    """Mean of each region's tokens, all channels: (N,H,W,C) -> (N,S*S,C)."""
+    x = _d(x)
+    N, H, W, C = x.shape
+    out = np.empty((N, S * S, C), np.float64)
+    _load().oracle_region_mean(_p(x), N, H, W, C, S, _p(out))
+    return out
+
+
+def route(q, k, heads: int, S: int, topk: int, with_logits: bool = False):
+    """Region affinity, top-k region indices (descending) and their softmax weights."""
+    q, k = _d(q), _d(k)
+    N, H, W, C = q.shape
+    P = S * S
+    r_idx = np.empty((N, P, topk), np.int32)
+    r_w = np.empty((N, P, topk), np.float64)
+    logits = np.empty((N, P, P), np.float64) if with_logits else None
+    rc = _load().oracle_route(_p(q), _p(k), N, H, W, C, heads, S, topk, _p(r_idx, ctypes.c_int32),
+                              _p(r_w), _p(logits) if with_logits else None)
+    if rc:
+        raise ValueError("oracle_route: bad shape")
+    return (r_idx, r_w, logits) if with_logits else (r_idx, r_w)
+
+
+def lce(v, lce_w, lce_b) -> np.ndarray:
+    """Depthwise 5x5 cross-correlation of v (zero pad 2) plus bias."""
+    v, w, b = _d(v), _d(lce_w), _d(lce_b)
+    N, H, W, C = v.shape
+    out = np.empty_like(v)
+    _load().oracle_lce(_p(v), _p(w), _p(b), N, H, W, C, _p(out))
+    return out
+
+
+def attend(q, k, v, lce_w, lce_b, heads: int, S: int, r_idx) -> np.ndarray:
+    """Token-to-token attention over the given routing, plus LCE(V)."""
+    q, k, v, w, b = _d(q), _d(k), _d(v), _d(lce_w), _d(lce_b)
+    r_idx = np.ascontiguousarray(r_idx, dtype=np.int32)
+    N, H, W, C = q.shape
+    topk = r_idx.shape[-1]
+    out = np.empty_like(q)
+    rc = _load().oracle_attend(_p(q), _p(k), _p(v), _p(w), _p(b), N, H, W, C, heads, S, topk,
+                               _p(r_idx, ctypes.c_int32), _p(out))
+    if rc:
+        raise ValueError("oracle_attend: bad shape or region index (rc=%d)" % rc)
+    return out
+
+
+def forward(q, k, v, lce_w, lce_b, heads: int, S: int, topk: int
+            ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """The whole BRA forward: returns (out, r_idx, r_weight)."""
+    q, k, v, w, b = _d(q), _d(k), _d(v), _d(lce_w), _d(lce_b)
+    N, H, W, C = q.shape
+    P = S * S
+    out = np.empty_like(q)
+    r_idx = np.empty((N, P, topk), np.int32)
+    r_w = np.empty((N, P, topk), np.float64)
+    rc = _load().oracle_forward(_p(q), _p(k), _p(v), _p(w), _p(b), N, H, W, C, heads, S, topk,
+                                _p(out), _p(r_idx, ctypes.c_int32), _p(r_w))
+    if rc:
+        raise ValueError("oracle_forward: bad shape (rc=%d)" % rc)
+    return out, r_idx, r_w
+
+
+def check_shape(N, H, W, C, heads, S, topk) -> bool:
+    return _load().oracle_check_shape(N, H, W, C, heads, S, topk) == 0

@@ -1,0 +1,133 @@
+"""Seeded synthetic inputs for Bi-Level Routing Attention (BRA) workloads.
+
+This module only draws numbers and rounds them to the storage dtype; it holds
+none of the attention, pooling, routing or convolution arithmetic. Both the
+float64 oracle (through the tests) and the CUDA path (through the tests and the
+benchmark) receive exactly the arrays produced here.
+
+Workload shapes follow the BiFormer stage shapes of the pages:
+  * stage-1 shape comments for a 224x224 image (niftyadmin walk-through,
+    section "BRA模块": x (1,56,56,64), 49 regions of 8x8 tokens, 2 heads of 32,
+    topk 1);
+  * per-stage top-k 1, 4, 16, S^2 and S = 7 / 16 / 8 for classification /
+    detection / segmentation (bernice.tw, "Biformer" and "消融實驗" sections).
+
+Value recipe (stated once, used everywhere):
+  * q, k, v ~ N(0, 1) i.i.d.;
+  * for the detection and segmentation workloads, a per-(image, region,
+    channel) offset ~ N(0, 0.5^2) is added to each of q, k, v separately, so
+    that region means differ and routing is non-uniform;
+  * LCE depthwise 5x5 weight ~ N(0, 0.02^2); LCE bias ~ N(0, 0.01^2) for the
+    classification stage-2/3 workloads, 0 otherwise;
+  * values are drawn in float64, cast to float32, then rounded to bfloat16
+    (round-to-nearest-even) when the workload dtype is bf16.
+Seeds: workload c, tensor slot i -> seed 0xB1F0 + 16*c + i, with slots
+q=0, k=1, v=2, lce_w=3, lce_b=4, q/k/v region offsets = 5/6/7.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional
+
+import numpy as np
+
+SLOT = {"q": 0, "k": 1, "v": 2, "lce_w": 3, "lce_b": 4, "q_off": 5, "k_off": 6, "v_off": 7}
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One BRA forward problem: feature maps (N,H,W,C), `heads` heads, S x S regions."""
+
+    name: str
+    index: int          # seed namespace
+    N: int
+    H: int
+    W: int
+    C: int
+    heads: int
+    S: int
+    topk: int
+    dtype: str          # "f32" or "bf16"
+    region_bias: float = 0.0   # std of the per-(image, region, channel) offset
+    lce_b_std: float = 0.0
+    lce_w_std: float = 0.02
+
+    @property
+    def d(self) -> int:
+        return self.C // self.heads
+
+    @property
+    def regions(self) -> int:
+        return self.S * self.S
+
+    @property
+    def w2(self) -> int:
+        return (self.H // self.S) * (self.W // self.S)
+
+    @property
+    def tokens(self) -> int:
+        return self.N * self.H * self.W
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The BiFormer stage shapes used as parity cases and as the benchmark workload.
+WORKLOADS: Dict[str, Workload] = {
+    w.name: w
+    for w in [
+        Workload("stage1_tiny_224", 1, 1, 56, 56, 64, 2, 7, 1, "f32"),
+        Workload("cls_stage2_224", 2, 64, 28, 28, 128, 4, 7, 4, "bf16", lce_b_std=0.01),
+        Workload("cls_stage3_224", 3, 128, 14, 14, 256, 8, 7, 16, "bf16", lce_b_std=0.01),
+        Workload("cls_stage3_224_dense", 6, 128, 14, 14, 256, 8, 7, 49, "bf16", lce_b_std=0.01),
+        Workload("det_stage1_1024", 4, 2, 256, 256, 64, 2, 16, 1, "bf16", region_bias=0.5),
+        Workload("seg_stage2_512", 5, 8, 64, 64, 128, 4, 8, 4, "bf16", region_bias=0.5),
+    ]
+}
+
+BENCH_WORKLOAD = "cls_stage2_224"
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16 (ties to even); returns float32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    r = ((u + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)).astype(np.uint32)
+    return r.view(np.float32)
+
+
+def _rng(w: Workload, slot: str, seed_base: Optional[int]) -> np.random.Generator:
+    base = 0xB1F0 + 16 * w.index if seed_base is None else seed_base
+    return np.random.Generator(np.random.PCG64(base + SLOT[slot]))
+
+
+def _store(x: np.ndarray, dtype: str) -> np.ndarray:
+    x32 = x.astype(np.float32)
+    return round_bf16(x32) if dtype == "bf16" else x32
+
+
+def make_inputs(w: Workload, seed_base: Optional[int] = None, batch: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Return q, k, v (N,H,W,C), lce_w (C,5,5), lce_b (C) as float32 arrays.
+
+    When the workload dtype is bf16 every value is exactly representable in
+    bfloat16. `batch` overrides N (the first `batch` images of a longer draw are
+    NOT the same as a shorter draw; each call is its own sample).
+    """
+    N = w.N if batch is None else batch
+    shape = (N, w.H, w.W, w.C)
+    out = {}
+    hr, wr = w.H // w.S, w.W // w.S
+    for name in ("q", "k", "v"):
+        x = _rng(w, name, seed_base).standard_normal(shape)
+        if w.region_bias > 0:
+            off = _rng(w, name + "_off", seed_base).standard_normal((N, w.S, 1, w.S, 1, w.C)) * w.region_bias
+            x = (x.reshape(N, w.S, hr, w.S, wr, w.C) + off).reshape(shape)
+        out[name] = _store(x, w.dtype)
+    out["lce_w"] = _store(_rng(w, "lce_w", seed_base).standard_normal((w.C, 5, 5)) * w.lce_w_std, w.dtype)
+    if w.lce_b_std > 0:
+        b = _rng(w, "lce_b", seed_base).standard_normal((w.C,)) * w.lce_b_std
+    else:
+        b = np.zeros((w.C,))
+    out["lce_b"] = _store(b, w.dtype)
+    return out
