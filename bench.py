@@ -1,0 +1,448 @@
+"""Benchmark of the B200 BRA forward (Bi-Level Routing Attention, BiFormer).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one whole BRA forward (region means, routing, routed attention + LCE)
+over one batch of the workload, through the C ABI (`bra_forward`). Prints ONE JSON
+line on rank 0.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and a
+device synchronise, timed with CUDA events on the launching stream; the max over
+ranks is taken. Each step reads a different input set from a rotation whose total
+size is at least three times the L2 cache, so inputs come from HBM, not L2. The
+steps are replayed as CUDA graphs (one per input set) to take host launch cost out.
+A second, traced pass over the same K steps times each kernel with CUDA events on
+its own stream (bra_trace_*), for the roofline of the dominant kernel.
+
+Multi-GPU (torchrun): images are independent, so every rank runs its own batch of
+the workload with no collective on the data path ("scaling": "weak"); `value` is
+the tokens of all ranks over the slowest rank's time.
+
+--impl reference times the float64 CPU oracle on this host's cores (the only
+reference this method has): each step is a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from vision_transformer_sparse_b200 import synth  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "BRA fwd tokens/s and TFLOP/s at 1 B200; % of bf16 tensor/HBM roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch each step directly")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def algorithmic(w: synth.Workload):
+    """Per-forward algorithmic figures of the workload (one batch of N images)."""
+    b = 2 if w.dtype == "bf16" else 4
+    T = w.tokens
+    L = w.topk * w.w2                               # keys per query
+    flops = 4.0 * T * L * w.C                       # QK^T and PV, 2 flops per MAC
+    gathered = float(w.N * w.regions * w.topk * w.w2 * 2 * w.C * b)  # K+V tiles per query region
+    route_bytes = w.N * w.regions * w.topk * 8      # r_idx + r_weight
+    # bytes the attention kernel must move at least once: q, k, v read, out written,
+    # the routing read, the LCE parameters
+    attn_unique = 4.0 * T * w.C * b + w.N * w.regions * w.topk * 4 + w.C * 26 * b
+    pool_bytes = 2.0 * T * w.C * b + 2 * w.N * w.regions * w.C * 4
+    return {"tokens": T, "flops": flops, "gathered_bytes": gathered, "attn_bytes": attn_unique,
+            "pool_bytes": pool_bytes, "route_bytes": route_bytes, "elem_bytes": b}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("attn.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "vision_transformer_sparse_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from a committed ncu summary,
+    if it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "attn_bf16_%s.txt" % workload)
+    if not os.path.exists(path):
+        return None, None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.split(":", 1)[0].strip() in ("source_hash", "dram_bytes_per_launch",
+                                                                   "units_scale"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("source_hash") != kernel_source_hash() or "dram_bytes_per_launch" not in vals:
+        return None, path
+    return float(vals["dram_bytes_per_launch"]), path
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a background thread."""
+
+    REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+               "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+               "display_clock_setting": 0x100}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples = []
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        self._mark = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report without clocks
+            self.err = str(e)
+
+    def _read(self):
+        nv = self.nv
+        sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        return sm, r
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                sm, r = self._read()
+                self.samples.append((time.perf_counter(), sm, r, self._mark))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def mark(self, tag):
+        self._mark = tag
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, tag="timed"):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        sel = [s for s in self.samples if s[3] == tag]
+        note = "samples during the timed region"
+        if not sel:
+            sel = self.samples[-5:]
+            note = "timed region shorter than the sampling period; nearest samples"
+        mhz = [s[1] for s in sel]
+        bits = 0
+        for s in sel:
+            bits |= s[2]
+        reasons = [k for k, v in self.REASONS.items() if bits & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sel), "note": note}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def bench_reference(args, w: synth.Workload, rank: int):
+    """The float64 CPU oracle on this host's cores; each step one image of the workload."""
+    import oracle
+    if rank != 0:
+        return None
+    sample = w.with_(N=1)
+    inp = {k: v.astype(np.float64) for k, v in synth.make_inputs(sample).items()}
+
+    def step():
+        oracle.forward(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], w.heads, w.S, w.topk)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = sample.tokens * args.steps / dt
+    cores = oracle.threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), BiFormer stage shape)",
+        "config": {"workload": w.name, "N": w.N, "H": w.H, "W": w.W, "C": w.C, "heads": w.heads,
+                   "S": w.S, "topk": w.topk, "input_dtype": w.dtype, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "1 image (%d tokens) of the workload per step" % sample.tokens},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def cpu_baseline(w: synth.Workload, budget_s: float = 12.0):
+    """The oracle as it stands on a bounded sample: whole images, repeated until the
+    budget is used (at least once)."""
+    import oracle
+    sample = w.with_(N=max(1, min(w.N, 8)))
+    inp = {k: v.astype(np.float64) for k, v in synth.make_inputs(sample).items()}
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], w.heads, w.S, w.topk)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt > budget_s or reps >= 50:
+            break
+    return {"value": sample.tokens * reps / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": "%d x forward of %d images (%d tokens), %.1f s" % (reps, sample.N, sample.tokens, dt)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if world > 1:
+            # rank 0 alone runs and prints; the others exit without work
+            if rank != 0:
+                return
+        line = bench_reference(args, w, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from vision_transformer_sparse_b200 import bra
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    acc = algorithmic(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    # inputs: this rank's own batch (weak scaling); seeded per rank
+    seed = None if rank == 0 else 0xB1F0 + 16 * w.index + 1000 * rank
+    inp = synth.make_inputs(w, seed_base=seed)
+    base = {k: torch.from_numpy(v).to(dev).to(tdt).contiguous() for k, v in inp.items()}
+    set_bytes = 4 * w.tokens * w.C * acc["elem_bytes"]
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_sets = max(2, math.ceil(3 * l2 / set_bytes))
+    sets = []
+    for _ in range(n_sets):
+        s = {k: v.clone() for k, v in base.items()}
+        s["out"] = torch.empty_like(base["q"])
+        s["r_idx"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.int32, device=dev)
+        s["r_w"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.float32, device=dev)
+        sets.append(s)
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def fwd(s):
+        bra.forward(s["q"], s["k"], s["v"], s["lce_w"], s["lce_b"], w.heads, w.S, w.topk,
+                    out=s["out"], r_idx=s["r_idx"], r_weight=s["r_w"], stream=stream)
+
+    # one CUDA graph per input set
+    graphs = []
+    kernels_per_step = None
+    with torch.cuda.stream(stream):
+        fwd(sets[0])  # first call outside capture: lazy module load, pool init
+    stream.synchronize()
+    if not args.no_graph:
+        for s in sets:
+            g = torch.cuda.CUDAGraph()
+            c0 = bra.launch_count()
+            with torch.cuda.graph(g, stream=stream):
+                fwd(s)
+            kernels_per_step = bra.launch_count() - c0
+            graphs.append(g)
+
+    def run_step(i):
+        if graphs:
+            graphs[i % n_sets].replay()
+        else:
+            fwd(sets[i % n_sets])
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            run_step(i)
+    stream.synchronize()
+
+    # ---- timed region
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    c_launch0 = bra.launch_count()
+    clocks.mark("timed")
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for i in range(args.steps):
+            run_step(i)
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark(None)
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    direct_launches = bra.launch_count() - c_launch0
+    gpu_launches = direct_launches if not graphs else kernels_per_step * args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- traced pass: per-kernel device time, same steps, direct launches
+    torch.cuda.synchronize(dev)
+    bra.trace_begin()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            fwd(sets[i % n_sets])
+    torch.cuda.synchronize(dev)
+    trace = bra.trace_end()
+    clocks.stop()
+
+    # ---- end to end through the host-buffer entry point (pinned host memory)
+    host = {k: v.cpu().pin_memory() for k, v in base.items()}
+    h_out = torch.empty_like(host["q"]).pin_memory()
+    h_idx = torch.empty((w.N, w.regions, w.topk), dtype=torch.int32).pin_memory()
+    h_w = torch.empty((w.N, w.regions, w.topk), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        bra.forward_host(host["q"], host["k"], host["v"], host["lce_w"], host["lce_b"], w.heads, w.S, w.topk,
+                         out=h_out, r_idx=h_idx, r_weight=h_w, stream=stream)
+
+    for _ in range(3):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = h_out.numel() * h_out.element_size() + h_idx.numel() * 4 + h_w.numel() * 4
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    ms_step = ms / args.steps
+    tokens_all = acc["tokens"] * world
+    value = tokens_all * args.steps / (ms / 1e3)
+    tflops = acc["flops"] * world * args.steps / (ms / 1e3) / 1e12
+
+    peaks, peak_kind = load_peaks()
+    attn_name = "attn_bf16_kernel" if w.dtype == "bf16" else "attn_f32_kernel"
+    t_ms, t_n = trace[attn_name]
+    attn_s = t_ms / max(t_n, 1) / 1e3
+    step_traced_ms = sum(v[0] for v in trace.values()) / args.steps
+    share = {k: round(v[0] / max(1e-12, sum(x[0] for x in trace.values())), 4) for k, v in trace.items() if v[1]}
+    achieved = acc["attn_bytes"] / attn_s / 1e9
+    traffic, _ = profiled_traffic(w.name)
+    # the roofline the method's own accounting states: slower of the FLOP term at the
+    # tensor peak and the gathered K/V bytes at HBM bandwidth
+    t_flop = acc["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_gath = acc["gathered_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    ns_bound = "tensor" if t_flop > t_gath else "hbm"
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1), BiFormer stage shape; no dataset)",
+        "config": {"workload": w.name, "N_per_gpu": w.N, "H": w.H, "W": w.W, "C": w.C, "heads": w.heads,
+                   "S": w.S, "topk": w.topk, "global_batch": w.N * world,
+                   "l2": "inputs larger than L2: %d rotating input sets, %.0f MB each, %.0f MB total vs L2 %.0f MB"
+                         % (n_sets, set_bytes / 1e6, n_sets * set_bytes / 1e6, l2 / 1e6),
+                   "launch": "CUDA graph per step" if graphs else "direct launches",
+                   "parallelism": "dp%d (independent images, no collective)" % world},
+        "tflops": tflops,
+        "gpu_launches": gpu_launches,
+        "roofline": {"bound": "hbm", "kernel": attn_name, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes_per_launch": acc["attn_bytes"],
+                     "avg_launch_us": attn_s * 1e6, "peak_source": peak_kind},
+        "roofline_gathered": {"definition": "max(attention FLOP / bf16 peak, gathered K/V bytes / HBM)",
+                              "bound": ns_bound, "roofline_us": max(t_flop, t_gath) * 1e6,
+                              "attn_us": attn_s * 1e6, "frac": max(t_flop, t_gath) / attn_s,
+                              "step_frac": max(t_flop, t_gath) / (ms_step / 1e3),
+                              "gathered_bytes": acc["gathered_bytes"], "flops": acc["flops"]},
+        "kernels": {k: {"ms_total": round(v[0], 4), "launches": v[1], "us_per_launch": round(v[0] * 1e3 / v[1], 3),
+                        "share": share.get(k)} for k, v in trace.items() if v[1]},
+        "traced_step_ms": step_traced_ms,
+        "clocks": clocks.summary(),
+        "e2e": {"value": tokens_all * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                "entry": "bra_forward_host (pinned host buffers)"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,150 @@
+/*
+ * bra.h — C ABI of the B200 (sm_100a) Bi-Level Routing Attention forward.
+ *
+ * Bi-Level Routing Attention (BRA) is the attention of BiFormer. The operation is
+ * the one the official code computes, as walked through on the page
+ * "BiFormer ... 前向传播过程" (TRANSFORMER.niftyadmin.cn/n/347023.html), section
+ * "BRA模块", eqs. 3-7, and Algorithm 1 as described on bernice.tw
+ * ("Bi-Level Routing Attention", parts one to three):
+ *
+ *   1. patchify: the (N,H,W,C) map is cut into S x S regions of
+ *      hr x wr = (H/S) x (W/S) tokens; region p = j*S + i is region row j,
+ *      region column i; tokens inside a region are row-major;
+ *   2. region query/key = mean of the region's tokens over all C channels;
+ *      affinity A[p][p'] = (scale * q_r[p]) . k_r[p']                     (eq. 4)
+ *   3. r_idx = the topk largest affinities of each row, in descending order
+ *      (ties: lower region index first); r_weight = softmax of those topk
+ *      affinities                                                          (eq. 5)
+ *   4. every query token attends, per head, jointly over the tokens of its
+ *      region's topk routed regions: softmax((scale*q) . k) v              (eqs. 6-7)
+ *   5. plus LCE(V): depthwise 5x5 cross-correlation of the whole V image,
+ *      zero padding 2, plus a per-channel bias                             (eq. 7)
+ *
+ * scale = d^-0.5 with d = C/heads, for both the routing and the attention.
+ * r_weight is an output only: it does not weight K or V.
+ *
+ * Conventions for every entry point:
+ *   - q, k, v, out: (N,H,W,C) contiguous channels-last, element type `dtype`;
+ *     channel m*d + c is component c of head m.
+ *   - lce_w: (C,5,5) contiguous (a PyTorch (C,1,5,5) depthwise weight), element
+ *     type `dtype`; lce_b: (C), element type `dtype`.
+ *   - r_idx: int32 (N,S*S,topk); r_weight: float32 (N,S*S,topk).
+ *   - All pointers are DEVICE pointers of the current device (except in
+ *     bra_forward_host), owned by the caller; the library never frees them.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
+ *     enqueues work on `stream`: it never synchronises it and never blocks the
+ *     host, except bra_forward_host, which returns after its results are on the
+ *     host.
+ *   - Scratch memory (the pooled region queries and keys, 2*N*S*S*C floats) is
+ *     taken stream-ordered from the device's default memory pool
+ *     (cudaMallocAsync on `stream`) and released stream-ordered after its last
+ *     use.
+ *   - Errors: arguments are checked before any CUDA call; on a bad argument
+ *     nothing is launched and a BRA_ERR_* code is returned. BRA_ERR_CUDA reports
+ *     a failed allocation or launch (the CUDA error is left for the caller to
+ *     inspect with cudaGetLastError()). No C++ exception crosses this boundary.
+ *   - Supported shapes: H % S == 0, W % S == 0, 1 <= S*S <= 256,
+ *     1 <= topk <= S*S, C % heads == 0, d in {32, 64}, C <= 1024,
+ *     W/S <= 128. N may be 0 (nothing is launched; pointers may be NULL).
+ *   - Alignment: q, k, v, out 16-byte aligned; r_idx, r_weight 4-byte aligned.
+ */
+#ifndef BRA_H
+#define BRA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *bra_stream_t;
+
+typedef enum { BRA_F32 = 0, BRA_BF16 = 1 } bra_dtype_t;
+
+enum {
+    BRA_OK = 0,
+    BRA_ERR_NULL = 1,        /* a required pointer is NULL                      */
+    BRA_ERR_SHAPE = 2,       /* shape outside the supported set listed above     */
+    BRA_ERR_ALIGN = 3,       /* a pointer is not aligned as required             */
+    BRA_ERR_DTYPE = 4,       /* dtype is not BRA_F32 or BRA_BF16                 */
+    BRA_ERR_CUDA = 5,        /* a CUDA allocation, copy or launch failed         */
+    BRA_ERR_INDEX = 6        /* bra_attend: a region index outside [0, S*S)      */
+};
+
+/* Steps 1-5: the whole BRA forward.
+ * In:  q, k, v, lce_w, lce_b (device).  Out: out (N,H,W,C) in `dtype`, r_idx,
+ * r_weight (device). Routing (steps 1-3) is computed in float32 from the
+ * stored values; the attention accumulates in float32 (bf16 tensor-core
+ * products for BRA_BF16, float32 FMA for BRA_F32); the output is rounded once
+ * to `dtype` (round to nearest even). */
+int bra_forward(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b,
+                int N, int H, int W, int C, int heads, int S, int topk, int dtype, void *out,
+                int32_t *r_idx, float *r_weight, bra_stream_t stream);
+
+/* Steps 1-3 only (region pooling, affinity, top-k routing): writes r_idx and
+ * r_weight. Same conventions as bra_forward. */
+int bra_route(const void *q, const void *k, int N, int H, int W, int C, int heads, int S, int topk,
+              int dtype, int32_t *r_idx, float *r_weight, bra_stream_t stream);
+
+/* Steps 4-5 only, for a routing given by the caller: r_idx (N,S*S,topk) int32
+ * device array of region indices (any order; duplicates allowed and counted
+ * twice). Every index must lie in [0, S*S); the kernel treats an index outside
+ * that range as a zero key/value tile that takes no part in the softmax and
+ * flags it, and the call then returns BRA_ERR_INDEX — this check reads one word
+ * back, so unlike the other entry points bra_attend synchronises `stream`. */
+int bra_attend(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b,
+               int N, int H, int W, int C, int heads, int S, int topk, int dtype,
+               const int32_t *r_idx, void *out, bra_stream_t stream);
+
+/* bra_forward on HOST buffers: copies the inputs from host memory to the
+ * device (pinned host memory gives asynchronous copies), runs the forward on
+ * `stream`, copies out, r_idx and r_weight back to the host buffers and
+ * synchronises `stream` before returning. Device buffers are taken from and
+ * returned to the device's default memory pool, stream-ordered. Same shapes,
+ * dtypes and error codes as bra_forward; host pointers need no alignment. */
+int bra_forward_host(const void *q, const void *k, const void *v, const void *lce_w,
+                     const void *lce_b, int N, int H, int W, int C, int heads, int S, int topk,
+                     int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Tracing (measurement support; no part of the computation).
+ *
+ * Kernel classes the library launches, for bra_trace_end and bra_kernel_name. */
+enum {
+    BRA_KERNEL_REGION_MEAN = 0, /* step 2 prelude: region means of q and k        */
+    BRA_KERNEL_ROUTE = 1,       /* steps 2-3: affinity row, top-k, softmax        */
+    BRA_KERNEL_ATTN_BF16 = 2,   /* steps 4-5, bfloat16 tensor-core kernel         */
+    BRA_KERNEL_ATTN_F32 = 3,    /* steps 4-5, float32 SIMT kernel                 */
+    BRA_KERNEL_CLASSES = 4
+};
+
+/* Number of kernels this library has launched since it was loaded (all threads,
+ * all devices). */
+long long bra_launch_count(void);
+
+/* Start tracing: until bra_trace_end, every kernel launch is bracketed by two
+ * CUDA events recorded on its own stream. Launches inside a CUDA graph capture
+ * are not traced. Returns BRA_OK. */
+int bra_trace_begin(void);
+
+/* Stop tracing, wait for the recorded events and write, per kernel class
+ * (BRA_KERNEL_CLASSES entries each), the summed device time in milliseconds and
+ * the number of traced launches. Either array may be NULL. Returns BRA_OK or
+ * BRA_ERR_CUDA. */
+int bra_trace_end(double *ms, long long *launches);
+
+/* Name of a kernel class, or "unknown". */
+const char *bra_kernel_name(int kernel_class);
+
+/* A static, human-readable description of a status code. */
+const char *bra_status_string(int status);
+
+/* Library ABI version: (major << 16) | minor. */
+int bra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BRA_H */

@@ -1,0 +1,107 @@
+"""Parity checks of a BRA result against the float64 oracle — TEST INFRASTRUCTURE ONLY.
+
+Works on numpy arrays; knows nothing of how the result under test was produced.
+
+Rules (fixed for this operation):
+  * r_idx: per row, the SET of routed regions must equal the oracle's wherever the
+    oracle's k-th and (k+1)-th largest affinities differ by more than 1e-3. Rows
+    under that gap ("near ties") are counted separately; there the result's set must
+    still be a valid top-k of the oracle's affinities within 1e-3.
+  * r_weight: compared index by index (after matching the orders) within 1e-5.
+  * out: float32 inputs -> max |out - ref| <= 1e-4; bfloat16 inputs ->
+    |out - ref| <= 2e-2 + 1e-2 |ref| element-wise. The reference output is the
+    oracle's attention over the routing under test, so that a near-tie row is still
+    checked element by element.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+import oracle
+
+GAP = 1e-3
+TOL_F32_ABS = 1e-4
+TOL_BF16_ABS, TOL_BF16_REL = 2e-2, 1e-2
+TOL_WEIGHT = 1e-5
+
+
+@dataclasses.dataclass
+class Report:
+    rows: int = 0
+    near_tie_rows: int = 0
+    idx_mismatch_rows: int = 0
+    weight_max_err: float = 0.0
+    out_max_abs_err: float = 0.0
+    out_worst_ratio: float = 0.0   # max over elements of err / allowed
+    ok: bool = True
+    notes: str = ""
+
+    def fail(self, msg: str):
+        self.ok = False
+        self.notes += msg + "; "
+
+
+def check_routing(logits: np.ndarray, ref_idx: np.ndarray, ref_w: np.ndarray, idx: np.ndarray,
+                  w: np.ndarray, rep: Report) -> None:
+    N, P, topk = ref_idx.shape
+    srt = -np.sort(-logits, axis=-1)
+    for n in range(N):
+        for p in range(P):
+            rep.rows += 1
+            got = idx[n, p]
+            if np.any(got < 0) or np.any(got >= P) or len(set(got.tolist())) != topk:
+                rep.fail("row (%d,%d): invalid index set %s" % (n, p, got))
+                continue
+            near = topk < P and srt[n, p, topk - 1] - srt[n, p, topk] <= GAP
+            if near:
+                rep.near_tie_rows += 1
+                kth = srt[n, p, topk - 1]
+                if np.any(logits[n, p, got] < kth - GAP):
+                    rep.fail("row (%d,%d): near-tie set is not a valid top-k" % (n, p))
+                continue
+            if set(got.tolist()) != set(ref_idx[n, p].tolist()):
+                rep.idx_mismatch_rows += 1
+                rep.fail("row (%d,%d): r_idx %s != oracle %s" % (n, p, got, ref_idx[n, p]))
+                continue
+            # descending order where neighbours are separated by more than the gap
+            lg = logits[n, p, got]
+            if np.any(np.diff(lg) > GAP):
+                rep.fail("row (%d,%d): r_idx not in descending affinity order" % (n, p))
+            ref_map = dict(zip(ref_idx[n, p].tolist(), ref_w[n, p].tolist()))
+            err = max(abs(float(w[n, p, a]) - ref_map[int(got[a])]) for a in range(topk))
+            rep.weight_max_err = max(rep.weight_max_err, err)
+    if rep.weight_max_err > TOL_WEIGHT:
+        rep.fail("r_weight err %.3g > %.1g" % (rep.weight_max_err, TOL_WEIGHT))
+
+
+def check_output(out: np.ndarray, ref: np.ndarray, dtype: str, rep: Report) -> None:
+    out = out.astype(np.float64)
+    err = np.abs(out - ref)
+    rep.out_max_abs_err = float(err.max()) if err.size else 0.0
+    if dtype == "f32":
+        allowed = np.full_like(ref, TOL_F32_ABS)
+    else:
+        allowed = TOL_BF16_ABS + TOL_BF16_REL * np.abs(ref)
+    ratio = err / allowed
+    rep.out_worst_ratio = float(ratio.max()) if ratio.size else 0.0
+    if not np.all(np.isfinite(out)):
+        rep.fail("non-finite output")
+    if rep.out_worst_ratio > 1.0:
+        where = np.unravel_index(np.argmax(ratio), ratio.shape)
+        rep.fail("out err %.3g at %s (ref %.4g, got %.4g)" % (err[where], where, ref[where], out[where]))
+
+
+def check_forward(inp: dict, heads: int, S: int, topk: int, dtype: str, out: np.ndarray, r_idx: np.ndarray,
+                  r_weight: np.ndarray, ref: Optional[tuple] = None) -> Report:
+    """Full parity check of one bra_forward result; `inp` holds the exact input values."""
+    rep = Report()
+    ref_idx, ref_w, logits = ref if ref is not None else oracle.route(inp["q"], inp["k"], heads, S, topk,
+                                                                      with_logits=True)
+    check_routing(logits, ref_idx, ref_w, r_idx, r_weight, rep)
+    if rep.ok:
+        ref_out = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], heads, S, r_idx)
+        check_output(out, ref_out, dtype, rep)
+    return rep

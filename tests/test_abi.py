@@ -1,0 +1,83 @@
+"""The C-ABI library loads, exports every entry point include/bra.h declares, and
+rejects bad arguments before touching CUDA (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from vision_transformer_sparse_b200 import bra
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "bra.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bra_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert set(names) == set(bra.SYMBOLS), names
+
+
+def test_library_exports_every_declared_symbol(bra_lib):
+    for name in declared_functions():
+        assert hasattr(bra_lib, name), name
+    assert bra_lib.bra_version() >> 16 == 1
+    for code in range(7):
+        assert bra.status_string(code) != "unknown status"
+
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: checks fail first
+ODD = ctypes.c_void_p(0x10008)
+
+
+def fwd(shape, ptrs=None):
+    p = [FAKE] * 5 if ptrs is None else ptrs[:5]
+    o = [FAKE] * 3 if ptrs is None else ptrs[5:]
+    return bra.raw_call("bra_forward", *p, *shape, *o, None)
+
+
+@pytest.mark.parametrize("shape,code", [
+    ((1, 57, 56, 64, 2, 7, 1, 1), 2),    # H % S
+    ((1, 56, 50, 64, 2, 7, 1, 1), 2),    # W % S
+    ((1, 56, 56, 64, 3, 7, 1, 1), 2),    # C % heads
+    ((1, 56, 56, 96, 2, 7, 1, 1), 2),    # d = 48
+    ((1, 56, 56, 64, 2, 7, 0, 1), 2),    # topk = 0
+    ((1, 56, 56, 64, 2, 7, 50, 1), 2),   # topk > S^2
+    ((1, 68, 68, 64, 2, 17, 1, 1), 2),   # S^2 > 256
+    ((1, 56, 56, 64, 2, 0, 1, 1), 2),    # S = 0
+    ((-1, 56, 56, 64, 2, 7, 1, 1), 2),   # N < 0
+    ((1, 56, 56, 64, 2, 7, 1, 7), 4),    # dtype
+    ((1, 1032, 1032, 64, 2, 4, 1, 1), 2),  # region wider than 128
+])
+def test_bad_shapes_rejected(bra_lib, shape, code):
+    assert fwd(shape) == code
+    assert bra.raw_call("bra_route", FAKE, FAKE, *shape, FAKE, FAKE, None) == code
+    assert bra.raw_call("bra_attend", *[FAKE] * 5, *shape, FAKE, FAKE, None) == code
+    assert bra.raw_call("bra_forward_host", *[FAKE] * 5, *shape, *[FAKE] * 3, None) == code
+
+
+def test_null_and_alignment_rejected(bra_lib):
+    shape = (1, 56, 56, 64, 2, 7, 1, 1)
+    for i in range(8):
+        ptrs = [FAKE] * 8
+        ptrs[i] = None
+        assert fwd(shape, ptrs) == 1
+    for i in (0, 1, 2, 5):   # q, k, v, out need 16 bytes
+        ptrs = [FAKE] * 8
+        ptrs[i] = ODD
+        assert fwd(shape, ptrs) == 3
+    ptrs = [FAKE] * 8
+    ptrs[6] = ctypes.c_void_p(0x10002)   # r_idx needs 4 bytes
+    assert fwd(shape, ptrs) == 3
+    assert bra.raw_call("bra_route", None, FAKE, *shape, FAKE, FAKE, None) == 1
+    assert bra.raw_call("bra_attend", *[FAKE] * 5, *shape, None, FAKE, None) == 1
+
+
+def test_empty_batch_is_a_no_op(bra_lib):
+    shape = (0, 56, 56, 64, 2, 7, 1, 1)
+    assert fwd(shape, [None] * 8) == 0
+    assert bra.raw_call("bra_route", None, None, *shape, None, None, None) == 0

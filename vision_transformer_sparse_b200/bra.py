@@ -1,0 +1,170 @@
+"""ctypes binding of the C-ABI library `libbra.so` (declared in include/bra.h).
+
+Argument marshalling only: shapes are read from the tensors, outputs are
+allocated with torch when not given, and the call goes straight to the C entry
+point of the same name on the current torch CUDA stream. Every step of the
+computation runs in the library's CUDA kernels; there is no fallback. If the
+library is missing this module raises at first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbra.so")
+_lib = None
+
+BRA_F32, BRA_BF16 = 0, 1
+STATUS = {0: "BRA_OK", 1: "BRA_ERR_NULL", 2: "BRA_ERR_SHAPE", 3: "BRA_ERR_ALIGN", 4: "BRA_ERR_DTYPE",
+          5: "BRA_ERR_CUDA", 6: "BRA_ERR_INDEX"}
+# entry points declared in include/bra.h
+SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_status_string",
+           "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name")
+KERNEL_CLASSES = 4
+
+
+class BraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (where, STATUS.get(status, status), status_string(status)))
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError("libbra.so is not built (%s); run "
+                               "`python -m vision_transformer_sparse_b200.build`" % _LIB_PATH)
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        shape = [i] * 8  # N, H, W, C, heads, S, topk, dtype
+        L.bra_forward.argtypes = [vp] * 5 + shape + [vp, vp, vp, vp]
+        L.bra_route.argtypes = [vp] * 2 + shape + [vp, vp, vp]
+        L.bra_attend.argtypes = [vp] * 5 + shape + [vp, vp, vp]
+        L.bra_forward_host.argtypes = [vp] * 5 + shape + [vp, vp, vp, vp]
+        for f in ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_version"):
+            getattr(L, f).restype = i
+        L.bra_status_string.argtypes = [i]
+        L.bra_status_string.restype = ctypes.c_char_p
+        L.bra_launch_count.restype = ctypes.c_longlong
+        L.bra_trace_begin.restype = i
+        L.bra_trace_end.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+        L.bra_trace_end.restype = i
+        L.bra_kernel_name.argtypes = [i]
+        L.bra_kernel_name.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().bra_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BRA_BF16
+    if t.dtype == torch.float32:
+        return BRA_F32
+    raise TypeError("BRA takes bfloat16 or float32 tensors, got %s" % t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_dev(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("BRA tensors must be contiguous CUDA tensors")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _raise(rc: int, where: str):
+    if rc != 0:
+        raise BraError(rc, where)
+
+
+def forward(q, k, v, lce_w, lce_b, heads: int, S: int, topk: int, out=None, r_idx=None, r_weight=None,
+            stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """bra_forward: (N,H,W,C) q, k, v; lce_w (C,5,5); lce_b (C) -> out, r_idx, r_weight."""
+    N, H, W, C = q.shape
+    P = S * S
+    out = torch.empty_like(q) if out is None else out
+    r_idx = torch.empty((N, P, topk), dtype=torch.int32, device=q.device) if r_idx is None else r_idx
+    r_weight = torch.empty((N, P, topk), dtype=torch.float32, device=q.device) if r_weight is None else r_weight
+    _check_dev(q, k, v, lce_w, lce_b, out, r_idx, r_weight)
+    rc = lib().bra_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(lce_b), N, H, W, C, heads, S, topk,
+                           _dtype_code(q), _ptr(out), _ptr(r_idx), _ptr(r_weight), _stream(stream))
+    _raise(rc, "bra_forward")
+    return out, r_idx, r_weight
+
+
+def route(q, k, heads: int, S: int, topk: int, r_idx=None, r_weight=None, stream=None):
+    """bra_route: region pooling, affinity and top-k -> r_idx (int32), r_weight (float32)."""
+    N, H, W, C = q.shape
+    P = S * S
+    r_idx = torch.empty((N, P, topk), dtype=torch.int32, device=q.device) if r_idx is None else r_idx
+    r_weight = torch.empty((N, P, topk), dtype=torch.float32, device=q.device) if r_weight is None else r_weight
+    _check_dev(q, k, r_idx, r_weight)
+    rc = lib().bra_route(_ptr(q), _ptr(k), N, H, W, C, heads, S, topk, _dtype_code(q), _ptr(r_idx),
+                         _ptr(r_weight), _stream(stream))
+    _raise(rc, "bra_route")
+    return r_idx, r_weight
+
+
+def attend(q, k, v, lce_w, lce_b, heads: int, S: int, r_idx, out=None, stream=None) -> torch.Tensor:
+    """bra_attend: attention over a given routing r_idx (N,S*S,topk) int32, plus LCE(V)."""
+    N, H, W, C = q.shape
+    topk = r_idx.shape[-1]
+    out = torch.empty_like(q) if out is None else out
+    _check_dev(q, k, v, lce_w, lce_b, r_idx, out)
+    rc = lib().bra_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(lce_b), N, H, W, C, heads, S, topk,
+                          _dtype_code(q), _ptr(r_idx), _ptr(out), _stream(stream))
+    _raise(rc, "bra_attend")
+    return out
+
+
+def forward_host(q, k, v, lce_w, lce_b, heads: int, S: int, topk: int, out=None, r_idx=None,
+                 r_weight=None, stream=None):
+    """bra_forward_host: host (CPU, ideally pinned) tensors in and out; the library copies."""
+    N, H, W, C = q.shape
+    P = S * S
+    for t in (q, k, v, lce_w, lce_b):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("bra_forward_host takes contiguous host tensors")
+    out = torch.empty_like(q) if out is None else out
+    r_idx = torch.empty((N, P, topk), dtype=torch.int32) if r_idx is None else r_idx
+    r_weight = torch.empty((N, P, topk), dtype=torch.float32) if r_weight is None else r_weight
+    rc = lib().bra_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(lce_b), N, H, W, C, heads, S,
+                                topk, _dtype_code(q), _ptr(out), _ptr(r_idx), _ptr(r_weight), _stream(stream))
+    _raise(rc, "bra_forward_host")
+    return out, r_idx, r_weight
+
+
+def launch_count() -> int:
+    """Kernels the library has launched since it was loaded."""
+    return int(lib().bra_launch_count())
+
+
+def trace_begin() -> None:
+    _raise(lib().bra_trace_begin(), "bra_trace_begin")
+
+
+def trace_end() -> dict:
+    """{kernel name: (milliseconds, launches)} over the traced launches."""
+    ms = (ctypes.c_double * KERNEL_CLASSES)()
+    n = (ctypes.c_longlong * KERNEL_CLASSES)()
+    _raise(lib().bra_trace_end(ms, n), "bra_trace_end")
+    return {lib().bra_kernel_name(i).decode(): (ms[i], n[i]) for i in range(KERNEL_CLASSES)}
+
+
+def raw_call(name: str, *args) -> int:
+    """Call an entry point with raw ctypes arguments (argument-check tests)."""
+    return getattr(lib(), name)(*args)

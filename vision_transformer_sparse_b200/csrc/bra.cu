@@ -1,0 +1,445 @@
+// bra.cu — the C ABI of the BRA forward (declared in include/bra.h): argument
+// checking, launch-shape selection and the kernel launches.
+//
+// Call path of bra_forward on one stream, no host synchronisation:
+//   region_mean_kernel  (q, k -> pooled region means, float32 scratch)
+//   route_kernel        (pooled means -> affinity row, bitonic top-k, r_idx, r_weight)
+//   attn_*_kernel       (q, gathered k/v, r_idx -> attention + LCE epilogue -> out)
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/bra.h"
+#include "attn.cuh"
+#include "route.cuh"
+
+namespace bra {
+
+constexpr int kMaxSmem = 227 * 1024;
+
+// ----------------------------------------------------------------------------- tracing
+
+static std::atomic<long long> g_launches{0};
+static std::mutex g_trace_mu;
+static bool g_tracing = false;
+struct TraceRec {
+    int kid;
+    cudaEvent_t a, b;
+};
+static std::vector<TraceRec> g_trace;
+
+// Brackets one kernel launch: counts it and, while tracing (and not capturing),
+// records an event pair on its stream.
+class LaunchScope {
+  public:
+    LaunchScope(int kid, cudaStream_t st) : kid_(kid), st_(st) {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        std::lock_guard<std::mutex> g(g_trace_mu);
+        if (!g_tracing) return;
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+        if (cudaEventCreate(&a_) != cudaSuccess) return;
+        if (cudaEventCreate(&b_) != cudaSuccess) {
+            cudaEventDestroy(a_);
+            return;
+        }
+        if (cudaEventRecord(a_, st) != cudaSuccess) {
+            cudaEventDestroy(a_);
+            cudaEventDestroy(b_);
+            return;
+        }
+        on_ = true;
+    }
+    ~LaunchScope() {
+        if (!on_) return;
+        cudaEventRecord(b_, st_);
+        std::lock_guard<std::mutex> g(g_trace_mu);
+        g_trace.push_back({kid_, a_, b_});
+    }
+
+  private:
+    int kid_;
+    cudaStream_t st_;
+    cudaEvent_t a_{}, b_{};
+    bool on_ = false;
+};
+
+struct Shape {
+    int N, H, W, C, heads, S, topk, dtype;
+    int P, hr, wr, w2, d;
+};
+
+static bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape rules of include/bra.h; nothing here touches CUDA.
+static int check_shape(const Shape &s) {
+    if (s.dtype != BRA_F32 && s.dtype != BRA_BF16) return BRA_ERR_DTYPE;
+    if (s.N < 0 || s.H <= 0 || s.W <= 0 || s.C <= 0 || s.heads <= 0 || s.S <= 0) return BRA_ERR_SHAPE;
+    if (s.S > 16 || s.H % s.S != 0 || s.W % s.S != 0) return BRA_ERR_SHAPE;
+    if (s.topk < 1 || s.topk > s.S * s.S) return BRA_ERR_SHAPE;
+    if (s.C % s.heads != 0 || s.C > 1024) return BRA_ERR_SHAPE;
+    const int d = s.C / s.heads;
+    if (d != 32 && d != 64) return BRA_ERR_SHAPE;
+    if (s.W / s.S > 128) return BRA_ERR_SHAPE;
+    // element offsets are formed in 64-bit; grid sizes must fit in int
+    if ((long long)s.N * s.S * s.S * s.H > INT_MAX) return BRA_ERR_SHAPE;
+    if ((long long)s.H * s.W > INT_MAX / 4) return BRA_ERR_SHAPE;
+    return BRA_OK;
+}
+
+static Shape make_shape(int N, int H, int W, int C, int heads, int S, int topk, int dtype) {
+    Shape s{N, H, W, C, heads, S, topk, dtype, 0, 0, 0, 0, 0};
+    if (S > 0 && heads > 0) {
+        s.P = S * S;
+        s.hr = H / S;
+        s.wr = W / S;
+        s.w2 = s.hr * s.wr;
+        s.d = C / heads;
+    }
+    return s;
+}
+
+static int largest_divisor_at_most(int n, int cap) {
+    for (int x = cap < n ? cap : n; x >= 1; --x)
+        if (n % x == 0) return x;
+    return 1;
+}
+
+// ----------------------------------------------------------------------------- routing
+
+static int launch_route(const Shape &s, const void *q, const void *k, int32_t *r_idx, float *r_weight,
+                        cudaStream_t st) {
+    float *ws = nullptr;
+    const size_t pooled = (size_t)s.N * s.P * s.C;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * pooled * sizeof(float), st) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    const dim3 pgrid(s.N * s.P, 2);
+    {
+    LaunchScope ls(BRA_KERNEL_REGION_MEAN, st);
+    if (s.dtype == BRA_BF16)
+        region_mean_kernel<__nv_bfloat16><<<pgrid, kPoolThreads, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled,
+            s.H, s.W, s.C, s.S);
+    else
+        region_mean_kernel<float><<<pgrid, kPoolThreads, 0, st>>>(
+            static_cast<const float *>(q), static_cast<const float *>(k), ws, ws + pooled, s.H, s.W, s.C, s.S);
+    }
+
+    const float scale = 1.0f / sqrtf((float)s.d);
+    const int smem = s.P * (kRouteChunk + 1) * (int)sizeof(float);
+    const dim3 rgrid((s.P + kRouteWarps - 1) / kRouteWarps, 1, 1);
+    int rc = BRA_OK;
+    auto go = [&](auto kern) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+            rc = BRA_ERR_CUDA;
+            return;
+        }
+        for (int n0 = 0; n0 < s.N; n0 += 65535) {
+            const int nb = s.N - n0 < 65535 ? s.N - n0 : 65535;
+            dim3 g = rgrid;
+            g.y = nb;
+            LaunchScope ls(BRA_KERNEL_ROUTE, st);
+            kern<<<g, kRouteWarps * 32, smem, st>>>(ws + (size_t)n0 * s.P * s.C,
+                                                    ws + pooled + (size_t)n0 * s.P * s.C, s.C, s.P, s.topk,
+                                                    scale, r_idx + (size_t)n0 * s.P * s.topk,
+                                                    r_weight + (size_t)n0 * s.P * s.topk);
+        }
+    };
+    if (s.P <= 32)
+        go(route_kernel<1>);
+    else if (s.P <= 64)
+        go(route_kernel<2>);
+    else if (s.P <= 128)
+        go(route_kernel<4>);
+    else
+        go(route_kernel<8>);
+    if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
+    if (cudaFreeAsync(ws, st) != cudaSuccess) rc = BRA_ERR_CUDA;
+    return rc;
+}
+
+// ----------------------------------------------------------------------------- attention
+
+static AttnParams base_params(const Shape &s, const void *q, const void *k, const void *v, const void *w,
+                              const void *b, void *out, const int32_t *r_idx, int *err) {
+    AttnParams p{};
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.lce_w = w;
+    p.lce_b = b;
+    p.out = out;
+    p.r_idx = r_idx;
+    p.err_flag = err;
+    p.N = s.N;
+    p.H = s.H;
+    p.W = s.W;
+    p.C = s.C;
+    p.heads = s.heads;
+    p.S = s.S;
+    p.topk = s.topk;
+    p.hr = s.hr;
+    p.wr = s.wr;
+    p.w2 = s.w2;
+    p.P = s.P;
+    p.scale_log2 = (float)(1.0 / std::sqrt((double)s.d) * 1.4426950408889634);
+    return p;
+}
+
+// Tensor-core kernel shape: HG heads (HG*d <= 128 channels) and RB region rows per
+// CTA, with at most 8 warps of (head, 16-query tile) and 128 queries per CTA.
+static bool plan_bf16(const Shape &s, AttnParams &p, int &threads, int &smem) {
+    const int Lk = s.topk * s.w2;
+    p.stages = Lk > kKC ? 2 : 1;
+    for (int hg = largest_divisor_at_most(s.heads, 128 / s.d); hg >= 1; --hg) {
+        if (s.heads % hg) continue;
+        for (int rb = s.hr; rb >= 1; --rb) {
+            if (s.hr % rb) continue;
+            const int nq = rb * s.wr;
+            const int qt = (nq + 15) / 16;
+            if (nq > 128 || qt * hg > 8) continue;
+            const Bf16Smem L = bf16_smem_layout(s.topk, qt, rb, s.wr, hg * s.d, p.stages);
+            if (L.total > kMaxSmem) continue;
+            p.HG = hg;
+            p.RB = rb;
+            p.QT = qt;
+            p.n_hg = s.heads / hg;
+            p.n_rb = s.hr / rb;
+            threads = qt * hg * 32;
+            smem = L.total;
+            return true;
+        }
+    }
+    return false;
+}
+
+// SIMT float32 kernel shape: one thread per (query, head), at most 256 per CTA.
+static bool plan_f32(const Shape &s, AttnParams &p, int &threads, int &smem) {
+    for (int hg = largest_divisor_at_most(s.heads, 128 / s.d); hg >= 1; --hg) {
+        if (s.heads % hg) continue;
+        for (int rb = s.hr; rb >= 1; --rb) {
+            if (s.hr % rb) continue;
+            const int nq = rb * s.wr;
+            if (nq * hg > 256) continue;
+            const F32Smem L = f32_smem_layout(s.topk, nq, rb, s.wr, hg * s.d);
+            if (L.total > kMaxSmem) continue;
+            p.HG = hg;
+            p.RB = rb;
+            p.QT = 0;
+            p.stages = 1;
+            p.n_hg = s.heads / hg;
+            p.n_rb = s.hr / rb;
+            threads = ((nq * hg + 31) / 32) * 32;
+            smem = L.total;
+            return true;
+        }
+    }
+    return false;
+}
+
+template <typename K>
+static int launch_kernel(K kern, int kid, int blocks, int threads, int smem, cudaStream_t st,
+                         const AttnParams &p) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    LaunchScope ls(kid, st);
+    kern<<<blocks, threads, smem, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
+static int launch_attend(const Shape &s, const void *q, const void *k, const void *v, const void *w,
+                         const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st) {
+    AttnParams p = base_params(s, q, k, v, w, b, out, r_idx, err);
+    int threads = 0, smem = 0;
+    if (s.dtype == BRA_BF16) {
+        if (!plan_bf16(s, p, threads, smem)) return BRA_ERR_SHAPE;
+        const int blocks = s.N * s.P * p.n_rb * p.n_hg;
+        return s.d == 32 ? launch_kernel(attn_bf16_kernel<32>, BRA_KERNEL_ATTN_BF16, blocks, threads, smem, st, p)
+                         : launch_kernel(attn_bf16_kernel<64>, BRA_KERNEL_ATTN_BF16, blocks, threads, smem, st, p);
+    }
+    if (!plan_f32(s, p, threads, smem)) return BRA_ERR_SHAPE;
+    const int blocks = s.N * s.P * p.n_rb * p.n_hg;
+    return s.d == 32 ? launch_kernel(attn_f32_kernel<32>, BRA_KERNEL_ATTN_F32, blocks, threads, smem, st, p)
+                     : launch_kernel(attn_f32_kernel<64>, BRA_KERNEL_ATTN_F32, blocks, threads, smem, st, p);
+}
+
+// Everything a shape must pass before any CUDA call is made.
+static int check_plan(const Shape &s) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    AttnParams p{};
+    int t, m;
+    if (s.dtype == BRA_BF16 ? !plan_bf16(s, p, t, m) : !plan_f32(s, p, t, m)) return BRA_ERR_SHAPE;
+    return BRA_OK;
+}
+
+}  // namespace bra
+
+using namespace bra;
+
+extern "C" {
+
+int bra_version(void) { return (1 << 16) | 0; }
+
+long long bra_launch_count(void) { return g_launches.load(); }
+
+int bra_trace_begin(void) {
+    std::lock_guard<std::mutex> g(g_trace_mu);
+    g_tracing = true;
+    return BRA_OK;
+}
+
+int bra_trace_end(double *ms, long long *launches) {
+    std::vector<TraceRec> recs;
+    {
+        std::lock_guard<std::mutex> g(g_trace_mu);
+        g_tracing = false;
+        recs.swap(g_trace);
+    }
+    double tot[BRA_KERNEL_CLASSES] = {0};
+    long long cnt[BRA_KERNEL_CLASSES] = {0};
+    int rc = BRA_OK;
+    for (auto &r : recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            rc = BRA_ERR_CUDA;
+        tot[r.kid] += t;
+        cnt[r.kid] += 1;
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    for (int i = 0; i < BRA_KERNEL_CLASSES; ++i) {
+        if (ms) ms[i] = tot[i];
+        if (launches) launches[i] = cnt[i];
+    }
+    return rc;
+}
+
+const char *bra_kernel_name(int kernel_class) {
+    switch (kernel_class) {
+        case BRA_KERNEL_REGION_MEAN: return "region_mean_kernel";
+        case BRA_KERNEL_ROUTE: return "route_kernel";
+        case BRA_KERNEL_ATTN_BF16: return "attn_bf16_kernel";
+        case BRA_KERNEL_ATTN_F32: return "attn_f32_kernel";
+        default: return "unknown";
+    }
+}
+
+const char *bra_status_string(int status) {
+    switch (status) {
+        case BRA_OK: return "ok";
+        case BRA_ERR_NULL: return "a required pointer is NULL";
+        case BRA_ERR_SHAPE: return "unsupported shape (H%S, W%S, C%heads, topk, S*S<=256, d in {32,64}, C<=1024, W/S<=128)";
+        case BRA_ERR_ALIGN: return "pointer misaligned (q, k, v, out need 16 bytes; r_idx, r_weight 4)";
+        case BRA_ERR_DTYPE: return "dtype must be BRA_F32 or BRA_BF16";
+        case BRA_ERR_CUDA: return "a CUDA allocation, copy or kernel launch failed";
+        case BRA_ERR_INDEX: return "a region index in r_idx lies outside [0, S*S)";
+        default: return "unknown status";
+    }
+}
+
+int bra_route(const void *q, const void *k, int N, int H, int W, int C, int heads, int S, int topk,
+              int dtype, int32_t *r_idx, float *r_weight, bra_stream_t stream) {
+    const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
+    int rc = check_plan(s);
+    if (rc) return rc;
+    if (N == 0) return BRA_OK;
+    if (!q || !k || !r_idx || !r_weight) return BRA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(r_idx, 4) || !aligned(r_weight, 4)) return BRA_ERR_ALIGN;
+    return launch_route(s, q, k, r_idx, r_weight, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static int forward_device(const Shape &s, const void *q, const void *k, const void *v, const void *lce_w,
+                          const void *lce_b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st) {
+    int rc = launch_route(s, q, k, r_idx, r_weight, st);
+    if (rc) return rc;
+    return launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, nullptr, st);
+}
+
+int bra_forward(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b, int N,
+                int H, int W, int C, int heads, int S, int topk, int dtype, void *out, int32_t *r_idx,
+                float *r_weight, bra_stream_t stream) {
+    const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
+    int rc = check_plan(s);
+    if (rc) return rc;
+    if (N == 0) return BRA_OK;
+    if (!q || !k || !v || !lce_w || !lce_b || !out || !r_idx || !r_weight) return BRA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(r_idx, 4) ||
+        !aligned(r_weight, 4))
+        return BRA_ERR_ALIGN;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    if (!aligned(lce_w, es) || !aligned(lce_b, es)) return BRA_ERR_ALIGN;
+    return forward_device(s, q, k, v, lce_w, lce_b, out, r_idx, r_weight, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bra_attend(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b, int N,
+               int H, int W, int C, int heads, int S, int topk, int dtype, const int32_t *r_idx, void *out,
+               bra_stream_t stream) {
+    const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
+    int rc = check_plan(s);
+    if (rc) return rc;
+    if (N == 0) return BRA_OK;
+    if (!q || !k || !v || !lce_w || !lce_b || !out || !r_idx) return BRA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(r_idx, 4))
+        return BRA_ERR_ALIGN;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    if (!aligned(lce_w, es) || !aligned(lce_b, es)) return BRA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int *flag = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&flag), sizeof(int), st) != cudaSuccess) return BRA_ERR_CUDA;
+    int host_flag = 0;
+    rc = cudaMemsetAsync(flag, 0, sizeof(int), st) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+    if (rc == BRA_OK) rc = launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, flag, st);
+    if (rc == BRA_OK &&
+        cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        rc = BRA_ERR_CUDA;
+    if (cudaFreeAsync(flag, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    if (rc == BRA_OK && host_flag) rc = BRA_ERR_INDEX;
+    return rc;
+}
+
+int bra_forward_host(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b, int N,
+                     int H, int W, int C, int heads, int S, int topk, int dtype, void *out, int32_t *r_idx,
+                     float *r_weight, bra_stream_t stream) {
+    const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
+    int rc = check_plan(s);
+    if (rc) return rc;
+    if (N == 0) return BRA_OK;
+    if (!q || !k || !v || !lce_w || !lce_b || !out || !r_idx || !r_weight) return BRA_ERR_NULL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    const size_t map = (size_t)N * H * W * C * es, wb = (size_t)C * 25 * es, bb = (size_t)C * es;
+    const size_t route = (size_t)N * s.P * topk * 4;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t total = 4 * up(map) + up(wb) + up(bb) + 2 * up(route);
+    char *base = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&base), total, st) != cudaSuccess) return BRA_ERR_CUDA;
+    char *dq = base, *dk = dq + up(map), *dv = dk + up(map), *dout = dv + up(map), *dw = dout + up(map);
+    char *db = dw + up(wb), *di = db + up(bb), *dr = di + up(route);
+    rc = BRA_OK;
+    const struct {
+        void *dst;
+        const void *src;
+        size_t n;
+    } h2d[] = {{dq, q, map}, {dk, k, map}, {dv, v, map}, {dw, lce_w, wb}, {db, lce_b, bb}};
+    for (const auto &c : h2d)
+        if (rc == BRA_OK && cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            rc = BRA_ERR_CUDA;
+    if (rc == BRA_OK)
+        rc = forward_device(s, dq, dk, dv, dw, db, dout, reinterpret_cast<int32_t *>(di),
+                            reinterpret_cast<float *>(dr), st);
+    if (rc == BRA_OK && cudaMemcpyAsync(out, dout, map, cudaMemcpyDeviceToHost, st) != cudaSuccess) rc = BRA_ERR_CUDA;
+    if (rc == BRA_OK && cudaMemcpyAsync(r_idx, di, route, cudaMemcpyDeviceToHost, st) != cudaSuccess) rc = BRA_ERR_CUDA;
+    if (rc == BRA_OK && cudaMemcpyAsync(r_weight, dr, route, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        rc = BRA_ERR_CUDA;
+    if (cudaFreeAsync(base, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    return rc;
+}
+
+}  // extern "C"
