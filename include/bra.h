@@ -69,7 +69,9 @@ enum {
     BRA_ERR_ALIGN = 3,       /* a pointer is not aligned as required             */
     BRA_ERR_DTYPE = 4,       /* dtype is not BRA_F32 or BRA_BF16                 */
     BRA_ERR_CUDA = 5,        /* a CUDA allocation, copy or launch failed         */
-    BRA_ERR_INDEX = 6        /* bra_attend: a region index outside [0, S*S)      */
+    BRA_ERR_INDEX = 6,       /* bra_attend: a region index outside [0, S*S)      */
+    BRA_ERR_SCRATCH = 7      /* bra_forward_noalloc: problem needs more scratch
+                                than the library's static array holds          */
 };
 
 /* Steps 1-5: the whole BRA forward.
@@ -106,6 +108,36 @@ int bra_attend(const void *q, const void *k, const void *v, const void *lce_w, c
 int bra_forward_host(const void *q, const void *k, const void *v, const void *lce_w,
                      const void *lce_b, int N, int H, int W, int C, int heads, int S, int topk,
                      int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream);
+
+/* bra_forward without any device allocation. (No counterpart on the pages: this
+ * is a deployment variant of bra_forward, not a step of the method.)
+ *
+ * Some callers cannot allocate device memory at the moment they call in: a
+ * framework whose caching allocator has already reserved the device's memory, a
+ * real-time loop that forbids allocation after start-up, or a process whose
+ * default memory pool is disabled or capped. bra_forward takes its scratch (the
+ * pooled region means, 2*N*S*S*C floats) from the memory pool on every call;
+ * this entry point instead uses one fixed scratch array compiled into the
+ * library: BRA_STATIC_SCRATCH_FLOATS floats (16 MiB), present on every GPU that
+ * loads the library and held until the process exits. It calls no allocator.
+ *
+ *   - Same arguments, layouts, results and error codes as bra_forward; the
+ *     caller still passes (and owns) every input and output buffer.
+ *   - Limit: 2*N*S*S*C must not exceed BRA_STATIC_SCRATCH_FLOATS; a larger
+ *     problem returns BRA_ERR_SCRATCH before anything is launched.
+ *   - The first call on each device looks up the array's device address on that
+ *     device (it must be the current device, as for every call); make that first
+ *     call before any CUDA graph capture starts on the device.
+ *   - All calls share the one array, which keeps the last call's contents. No
+ *     part of it needs to start at zero: a call writes every element it reads.
+ *     Two calls whose kernels overlap on the GPU (different streams, or
+ *     different host threads without ordering) race on the array and give wrong
+ *     results: order them on one stream or with events. */
+#define BRA_STATIC_SCRATCH_FLOATS (4u * 1024u * 1024u)
+int bra_forward_noalloc(const void *q, const void *k, const void *v, const void *lce_w,
+                        const void *lce_b, int N, int H, int W, int C, int heads, int S,
+                        int topk, int dtype, void *out, int32_t *r_idx, float *r_weight,
+                        bra_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Tracing (measurement support; no part of the computation).

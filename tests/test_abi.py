@@ -26,7 +26,7 @@ def test_library_exports_every_declared_symbol(bra_lib):
     for name in declared_functions():
         assert hasattr(bra_lib, name), name
     assert bra_lib.bra_version() >> 16 == 1
-    for code in range(7):
+    for code in range(8):
         assert bra.status_string(code) != "unknown status"
 
 
@@ -58,6 +58,7 @@ def test_bad_shapes_rejected(bra_lib, shape, code):
     assert bra.raw_call("bra_route", FAKE, FAKE, *shape, FAKE, FAKE, None) == code
     assert bra.raw_call("bra_attend", *[FAKE] * 5, *shape, FAKE, FAKE, None) == code
     assert bra.raw_call("bra_forward_host", *[FAKE] * 5, *shape, *[FAKE] * 3, None) == code
+    assert bra.raw_call("bra_forward_noalloc", *[FAKE] * 5, *shape, *[FAKE] * 3, None) == code
 
 
 def test_null_and_alignment_rejected(bra_lib):

@@ -19,9 +19,11 @@ _lib = None
 
 BRA_F32, BRA_BF16 = 0, 1
 STATUS = {0: "BRA_OK", 1: "BRA_ERR_NULL", 2: "BRA_ERR_SHAPE", 3: "BRA_ERR_ALIGN", 4: "BRA_ERR_DTYPE",
-          5: "BRA_ERR_CUDA", 6: "BRA_ERR_INDEX"}
+          5: "BRA_ERR_CUDA", 6: "BRA_ERR_INDEX", 7: "BRA_ERR_SCRATCH"}
+STATIC_SCRATCH_FLOATS = 4 * 1024 * 1024
 # entry points declared in include/bra.h
-SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_status_string",
+SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
+           "bra_status_string",
            "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name")
 KERNEL_CLASSES = 4
 
@@ -45,7 +47,9 @@ def lib() -> ctypes.CDLL:
         L.bra_route.argtypes = [vp] * 2 + shape + [vp, vp, vp]
         L.bra_attend.argtypes = [vp] * 5 + shape + [vp, vp, vp]
         L.bra_forward_host.argtypes = [vp] * 5 + shape + [vp, vp, vp, vp]
-        for f in ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_version"):
+        L.bra_forward_noalloc.argtypes = [vp] * 5 + shape + [vp, vp, vp, vp]
+        for f in ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
+                  "bra_version"):
             getattr(L, f).restype = i
         L.bra_status_string.argtypes = [i]
         L.bra_status_string.restype = ctypes.c_char_p
@@ -103,6 +107,24 @@ def forward(q, k, v, lce_w, lce_b, heads: int, S: int, topk: int, out=None, r_id
     rc = lib().bra_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(lce_b), N, H, W, C, heads, S, topk,
                            _dtype_code(q), _ptr(out), _ptr(r_idx), _ptr(r_weight), _stream(stream))
     _raise(rc, "bra_forward")
+    return out, r_idx, r_weight
+
+
+def forward_noalloc(q, k, v, lce_w, lce_b, heads: int, S: int, topk: int, out=None, r_idx=None,
+                    r_weight=None, stream=None):
+    """bra_forward_noalloc: bra_forward with its scratch in the library's static device
+    array (no allocation inside the call). Outputs are allocated here with torch when not
+    given; pass them in to keep the whole call allocation-free."""
+    N, H, W, C = q.shape
+    P = S * S
+    out = torch.empty_like(q) if out is None else out
+    r_idx = torch.empty((N, P, topk), dtype=torch.int32, device=q.device) if r_idx is None else r_idx
+    r_weight = torch.empty((N, P, topk), dtype=torch.float32, device=q.device) if r_weight is None else r_weight
+    _check_dev(q, k, v, lce_w, lce_b, out, r_idx, r_weight)
+    rc = lib().bra_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(lce_b), N, H, W, C, heads, S,
+                                   topk, _dtype_code(q), _ptr(out), _ptr(r_idx), _ptr(r_weight),
+                                   _stream(stream))
+    _raise(rc, "bra_forward_noalloc")
     return out, r_idx, r_weight
 
 

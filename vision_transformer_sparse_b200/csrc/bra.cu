@@ -338,6 +338,7 @@ const char *bra_status_string(int status) {
         case BRA_ERR_DTYPE: return "dtype must be BRA_F32 or BRA_BF16";
         case BRA_ERR_CUDA: return "a CUDA allocation, copy or kernel launch failed";
         case BRA_ERR_INDEX: return "a region index in r_idx lies outside [0, S*S)";
+        case BRA_ERR_SCRATCH: return "problem needs more scratch than the static array holds (2*N*S*S*C > BRA_STATIC_SCRATCH_FLOATS)";
         default: return "unknown status";
     }
 }
@@ -440,6 +441,101 @@ int bra_forward_host(const void *q, const void *k, const void *v, const void *lc
     if (cudaFreeAsync(base, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     return rc;
+}
+
+// ----------------------------------------------------------------------------- no-allocation variant
+//
+// bra_forward_noalloc keeps its scratch (the pooled region means of q and k) in
+// this file-scope device array instead of the memory pool. Host code must not
+// pass the symbol itself to a kernel: on the host it names a host-side shadow,
+// so the device address is looked up once per device with cudaGetSymbolAddress.
+
+static __device__ __align__(256) float g_static_scratch[BRA_STATIC_SCRATCH_FLOATS];
+
+static constexpr int kMaxDevices = 64;
+static std::mutex g_static_mu;
+static float *g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device (looked up on first use).
+static int static_scratch(float **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BRA_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return BRA_ERR_CUDA;
+        g_static_ptr[dev] = static_cast<float *>(p);
+    }
+    *out = g_static_ptr[dev];
+    return BRA_OK;
+}
+
+// Steps 1-3 into caller-provided scratch ws (2*N*S*S*C floats); allocates nothing.
+static int launch_route_into(const Shape &s, const void *q, const void *k, int32_t *r_idx, float *r_weight,
+                             float *ws, cudaStream_t st) {
+    const size_t pooled = (size_t)s.N * s.P * s.C;
+    const dim3 pgrid(s.N * s.P, 2);
+    {
+        LaunchScope ls(BRA_KERNEL_REGION_MEAN, st);
+        if (s.dtype == BRA_BF16)
+            region_mean_kernel<__nv_bfloat16><<<pgrid, kPoolThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled,
+                s.H, s.W, s.C, s.S);
+        else
+            region_mean_kernel<float><<<pgrid, kPoolThreads, 0, st>>>(
+                static_cast<const float *>(q), static_cast<const float *>(k), ws, ws + pooled, s.H, s.W, s.C, s.S);
+    }
+    const float scale = 1.0f / sqrtf((float)s.d);
+    const int smem = s.P * (kRouteChunk + 1) * (int)sizeof(float);
+    int rc = BRA_OK;
+    auto go = [&](auto kern) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+            rc = BRA_ERR_CUDA;
+            return;
+        }
+        for (int n0 = 0; n0 < s.N; n0 += 65535) {
+            const int nb = s.N - n0 < 65535 ? s.N - n0 : 65535;
+            const dim3 g((s.P + kRouteWarps - 1) / kRouteWarps, nb, 1);
+            LaunchScope ls(BRA_KERNEL_ROUTE, st);
+            kern<<<g, kRouteWarps * 32, smem, st>>>(ws + (size_t)n0 * s.P * s.C,
+                                                    ws + pooled + (size_t)n0 * s.P * s.C, s.C, s.P, s.topk,
+                                                    scale, r_idx + (size_t)n0 * s.P * s.topk,
+                                                    r_weight + (size_t)n0 * s.P * s.topk);
+        }
+    };
+    if (s.P <= 32)
+        go(route_kernel<1>);
+    else if (s.P <= 64)
+        go(route_kernel<2>);
+    else if (s.P <= 128)
+        go(route_kernel<4>);
+    else
+        go(route_kernel<8>);
+    if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
+    return rc;
+}
+
+int bra_forward_noalloc(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b,
+                        int N, int H, int W, int C, int heads, int S, int topk, int dtype, void *out,
+                        int32_t *r_idx, float *r_weight, bra_stream_t stream) {
+    const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
+    int rc = check_plan(s);
+    if (rc) return rc;
+    if (N == 0) return BRA_OK;
+    if (!q || !k || !v || !lce_w || !lce_b || !out || !r_idx || !r_weight) return BRA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(r_idx, 4) ||
+        !aligned(r_weight, 4))
+        return BRA_ERR_ALIGN;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    if (!aligned(lce_w, es) || !aligned(lce_b, es)) return BRA_ERR_ALIGN;
+    if (2 * (size_t)N * s.P * C > (size_t)BRA_STATIC_SCRATCH_FLOATS) return BRA_ERR_SCRATCH;
+    float *ws = nullptr;
+    rc = static_scratch(&ws);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    rc = launch_route_into(s, q, k, r_idx, r_weight, ws, st);
+    if (rc) return rc;
+    return launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, nullptr, st);
 }
 
 }  // extern "C"
