@@ -70,8 +70,10 @@ enum {
     BRA_ERR_DTYPE = 4,       /* dtype is not BRA_F32 or BRA_BF16                 */
     BRA_ERR_CUDA = 5,        /* a CUDA allocation, copy or launch failed         */
     BRA_ERR_INDEX = 6,       /* bra_attend: a region index outside [0, S*S)      */
-    BRA_ERR_SCRATCH = 7      /* bra_forward_noalloc: problem needs more scratch
+    BRA_ERR_SCRATCH = 7,     /* bra_forward_noalloc: problem needs more scratch
                                 than the library's static array holds          */
+    BRA_ERR_TIMEOUT = 8      /* bra_device_status: a kernel's bounded wait for its
+                                tile copies ran out (its outputs are invalid)  */
 };
 
 /* Steps 1-5: the whole BRA forward.
@@ -168,6 +170,33 @@ int bra_trace_end(double *ms, long long *launches);
 
 /* Name of a kernel class, or "unknown". */
 const char *bra_kernel_name(int kernel_class);
+
+/* ---------------------------------------------------------------------------
+ * Kernel selection and device status.
+ *
+ * bfloat16 attention runs in one of two kernels that compute the same function:
+ * the TMA kernel (tile boxes fetched by the tensor memory accelerator) where the
+ * shape allows it (64 or 128 channels per CTA, every tile within the shared-memory
+ * budget, 4-byte aligned lce_w and lce_b), else the generic kernel (16-byte cp.async
+ * pieces). */
+enum { BRA_VARIANT_AUTO = 0, BRA_VARIANT_GENERIC = 1 };
+
+/* Select the attention kernel for all later calls in this process (for testing and
+ * comparison): BRA_VARIANT_AUTO (default) or BRA_VARIANT_GENERIC. Returns the
+ * previous setting, or -1 for an unknown variant. */
+int bra_set_kernel_variant(int variant);
+
+/* Synchronise `stream`, then report whether any kernel of this library gave up a
+ * bounded wait since the last call (BRA_ERR_TIMEOUT; the flag is cleared) or not
+ * (BRA_OK). BRA_ERR_CUDA if the synchronisation or the read fails. Kernels never
+ * spin without a limit: a wait that runs out raises this flag and the kernel
+ * returns. */
+int bra_device_status(bra_stream_t stream);
+
+/* Launch a one-CTA kernel that waits, `polls` times at most, on a barrier that
+ * never completes, so that its bounded wait runs out and raises the flag that
+ * bra_device_status reports. It moves no data. For testing the timeout path. */
+int bra_selftest_wait_timeout(unsigned polls, bra_stream_t stream);
 
 /* A static, human-readable description of a status code. */
 const char *bra_status_string(int status);

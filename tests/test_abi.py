@@ -26,7 +26,7 @@ def test_library_exports_every_declared_symbol(bra_lib):
     for name in declared_functions():
         assert hasattr(bra_lib, name), name
     assert bra_lib.bra_version() >> 16 == 1
-    for code in range(8):
+    for code in range(9):
         assert bra.status_string(code) != "unknown status"
 
 

@@ -44,10 +44,20 @@ def _lib(bra_lib):
     return bra_lib
 
 
+@pytest.fixture(params=["auto", "generic"])
+def variant(request):
+    """Run a test under the automatic kernel choice (TMA kernel where the shape
+    allows) and again with the generic cp.async kernel forced."""
+    prev = bra.set_kernel_variant(bra.VARIANT_AUTO if request.param == "auto" else bra.VARIANT_GENERIC)
+    yield request.param
+    bra.set_kernel_variant(prev)
+
+
 @pytest.mark.parametrize("name", list(synth.WORKLOADS))
-def test_stage_workloads_full_size(name):
+def test_stage_workloads_full_size(name, variant):
     w = synth.WORKLOADS[name]
     assert_parity(w, synth.make_inputs(w))
+    assert bra.device_status() == 0
 
 
 SMALL = [
@@ -67,7 +77,7 @@ SMALL = [
 
 
 @pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
-def test_small_shapes(shape):
+def test_small_shapes(shape, variant):
     N, H, W, C, heads, S, topk, dtype = shape
     w = synth.Workload("small", 40 + sum(shape[:7]), N, H, W, C, heads, S, topk, dtype,
                        region_bias=0.5, lce_b_std=0.05, lce_w_std=0.1)
@@ -94,7 +104,7 @@ def test_route_entry_point_matches_forward():
     assert rep.ok, rep.notes
 
 
-def test_attend_given_routing_with_duplicates_and_any_order():
+def test_attend_given_routing_with_duplicates_and_any_order(variant):
     w = synth.WORKLOADS["cls_stage2_224"].with_(N=4)
     inp = synth.make_inputs(w)
     d = to_dev(inp, w.dtype)
@@ -109,7 +119,18 @@ def test_attend_given_routing_with_duplicates_and_any_order():
     assert rep.ok, rep.notes
 
 
-def test_attend_rejects_out_of_range_region_index():
+def test_bounded_wait_reports_timeout_and_recovers():
+    """A wait that can never complete gives up after its poll limit, raises the device
+    flag (reported once by bra_device_status) and leaves the context usable."""
+    assert bra.device_status() == 0
+    bra.selftest_wait_timeout(64)
+    assert bra.device_status() == 8
+    assert bra.device_status() == 0
+    w = synth.WORKLOADS["cls_stage2_224"].with_(N=2)
+    assert_parity(w, synth.make_inputs(w))
+
+
+def test_attend_rejects_out_of_range_region_index(variant):
     """The kernel checks every index it reads; a bad one is reported, never dereferenced."""
     w = synth.WORKLOADS["cls_stage2_224"].with_(N=1)
     d = to_dev(synth.make_inputs(w), w.dtype)

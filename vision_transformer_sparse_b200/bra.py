@@ -19,12 +19,14 @@ _lib = None
 
 BRA_F32, BRA_BF16 = 0, 1
 STATUS = {0: "BRA_OK", 1: "BRA_ERR_NULL", 2: "BRA_ERR_SHAPE", 3: "BRA_ERR_ALIGN", 4: "BRA_ERR_DTYPE",
-          5: "BRA_ERR_CUDA", 6: "BRA_ERR_INDEX", 7: "BRA_ERR_SCRATCH"}
+          5: "BRA_ERR_CUDA", 6: "BRA_ERR_INDEX", 7: "BRA_ERR_SCRATCH", 8: "BRA_ERR_TIMEOUT"}
+VARIANT_AUTO, VARIANT_GENERIC = 0, 1
 STATIC_SCRATCH_FLOATS = 4 * 1024 * 1024
 # entry points declared in include/bra.h
 SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
            "bra_status_string",
-           "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name")
+           "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name",
+           "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout")
 KERNEL_CLASSES = 4
 
 
@@ -59,6 +61,12 @@ def lib() -> ctypes.CDLL:
         L.bra_trace_end.restype = i
         L.bra_kernel_name.argtypes = [i]
         L.bra_kernel_name.restype = ctypes.c_char_p
+        L.bra_set_kernel_variant.argtypes = [i]
+        L.bra_set_kernel_variant.restype = i
+        L.bra_device_status.argtypes = [vp]
+        L.bra_device_status.restype = i
+        L.bra_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+        L.bra_selftest_wait_timeout.restype = i
         _lib = L
     return _lib
 
@@ -185,6 +193,23 @@ def trace_end() -> dict:
     n = (ctypes.c_longlong * KERNEL_CLASSES)()
     _raise(lib().bra_trace_end(ms, n), "bra_trace_end")
     return {lib().bra_kernel_name(i).decode(): (ms[i], n[i]) for i in range(KERNEL_CLASSES)}
+
+
+def set_kernel_variant(variant: int) -> int:
+    """bra_set_kernel_variant: VARIANT_AUTO or VARIANT_GENERIC; returns the previous one."""
+    prev = lib().bra_set_kernel_variant(int(variant))
+    if prev < 0:
+        raise ValueError("unknown kernel variant %r" % variant)
+    return prev
+
+
+def device_status(stream=None) -> int:
+    """bra_device_status: 0, or 8 (BRA_ERR_TIMEOUT) if a kernel's bounded wait ran out."""
+    return int(lib().bra_device_status(_stream(stream)))
+
+
+def selftest_wait_timeout(polls: int, stream=None) -> None:
+    _raise(lib().bra_selftest_wait_timeout(int(polls), _stream(stream)), "bra_selftest_wait_timeout")
 
 
 def raw_call(name: str, *args) -> int:

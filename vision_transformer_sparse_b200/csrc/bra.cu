@@ -4,17 +4,26 @@
 // Call path of bra_forward on one stream, no host synchronisation:
 //   region_mean_kernel  (q, k -> pooled region means, float32 scratch)
 //   route_kernel        (pooled means -> affinity row, bitonic top-k, r_idx, r_weight)
-//   attn_*_kernel       (q, gathered k/v, r_idx -> attention + LCE epilogue -> out)
+//   attn_tma_kernel     (bf16: TMA tiles of q, routed k/v and the v halo -> attention
+//                        + LCE epilogue -> out), or attn_bf16_kernel / attn_f32_kernel
+//                        (cp.async tiles) for shapes the TMA kernel does not cover
+// The route and attention kernels are launched with programmatic dependent launch,
+// so each may start (and the attention kernel may fetch its q tile and v halo)
+// while the previous kernel drains.
 #include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
+
+#include <cudaTypedefs.h>
 
 #include "../../include/bra.h"
 #include "attn.cuh"
+#include "attn_tma.cuh"
 #include "route.cuh"
 
 namespace bra {
@@ -111,42 +120,72 @@ static int largest_divisor_at_most(int n, int cap) {
 
 // ----------------------------------------------------------------------------- routing
 
-static int launch_route(const Shape &s, const void *q, const void *k, int32_t *r_idx, float *r_weight,
-                        cudaStream_t st) {
-    float *ws = nullptr;
-    const size_t pooled = (size_t)s.N * s.P * s.C;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * pooled * sizeof(float), st) != cudaSuccess)
-        return BRA_ERR_CUDA;
-    const dim3 pgrid(s.N * s.P, 2);
-    {
-    LaunchScope ls(BRA_KERNEL_REGION_MEAN, st);
-    if (s.dtype == BRA_BF16)
-        region_mean_kernel<__nv_bfloat16><<<pgrid, kPoolThreads, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled,
-            s.H, s.W, s.C, s.S);
-    else
-        region_mean_kernel<float><<<pgrid, kPoolThreads, 0, st>>>(
-            static_cast<const float *>(q), static_cast<const float *>(k), ws, ws + pooled, s.H, s.W, s.C, s.S);
-    }
+// PDL launch: the kernel may begin before the preceding kernel on the stream has
+// finished; it calls griddepcontrol.wait before reading that kernel's results.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
+// Token slots per (region, channel group) for the region-mean kernel: ns divides wr,
+// G*ns divides 32, and each thread keeps at least 4 tokens.
+static int pool_ns_log2(const Shape &s) {
+    const int V = s.dtype == BRA_BF16 ? 8 : 4;
+    const int G = s.C / V;
+    int l = 0;
+    if (32 % G != 0) return 0;
+    while ((G << (l + 1)) <= 32 && s.wr % (1 << (l + 1)) == 0 && s.w2 / (1 << (l + 1)) >= 4) ++l;
+    return l;
+}
+
+// Steps 1-3 into scratch ws (2*N*S*S*C floats): region means, then the routing.
+static int launch_route_into(const Shape &s, const void *q, const void *k, int32_t *r_idx, float *r_weight,
+                             float *ws, cudaStream_t st) {
+    const size_t pooled = (size_t)s.N * s.P * s.C;
+    {
+        const int V = s.dtype == BRA_BF16 ? 8 : 4;
+        const int l = pool_ns_log2(s);
+        const long long total = 2LL * s.N * s.P * (s.C / V) << l;
+        const unsigned blocks = (unsigned)((total + kPoolThreads - 1) / kPoolThreads);
+        LaunchScope ls(BRA_KERNEL_REGION_MEAN, st);
+        if (s.dtype == BRA_BF16)
+            region_mean_kernel<__nv_bfloat16><<<blocks, kPoolThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled, s.N,
+                s.H, s.W, s.C, s.S, l, total);
+        else
+            region_mean_kernel<float><<<blocks, kPoolThreads, 0, st>>>(static_cast<const float *>(q),
+                                                                      static_cast<const float *>(k), ws,
+                                                                      ws + pooled, s.N, s.H, s.W, s.C, s.S, l, total);
+        if (cudaGetLastError() != cudaSuccess) return BRA_ERR_CUDA;
+    }
     const float scale = 1.0f / sqrtf((float)s.d);
-    const int smem = s.P * (kRouteChunk + 1) * (int)sizeof(float);
-    const dim3 rgrid((s.P + kRouteWarps - 1) / kRouteWarps, 1, 1);
+    const int cc = route_chunk(s.P, s.C);
+    const int smem = route_smem_bytes(s.P, cc);
     int rc = BRA_OK;
     auto go = [&](auto kern) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
             rc = BRA_ERR_CUDA;
             return;
         }
-        for (int n0 = 0; n0 < s.N; n0 += 65535) {
+        for (int n0 = 0; n0 < s.N && rc == BRA_OK; n0 += 65535) {
             const int nb = s.N - n0 < 65535 ? s.N - n0 : 65535;
-            dim3 g = rgrid;
-            g.y = nb;
+            const dim3 g((s.P + kRouteWarps - 1) / kRouteWarps, nb, 1);
             LaunchScope ls(BRA_KERNEL_ROUTE, st);
-            kern<<<g, kRouteWarps * 32, smem, st>>>(ws + (size_t)n0 * s.P * s.C,
-                                                    ws + pooled + (size_t)n0 * s.P * s.C, s.C, s.P, s.topk,
-                                                    scale, r_idx + (size_t)n0 * s.P * s.topk,
-                                                    r_weight + (size_t)n0 * s.P * s.topk);
+            if (launch_pdl(kern, g, dim3(kRouteWarps * 32), smem, st, (const float *)(ws + (size_t)n0 * s.P * s.C),
+                           (const float *)(ws + pooled + (size_t)n0 * s.P * s.C), s.C, s.P, s.topk, cc, scale,
+                           r_idx + (size_t)n0 * s.P * s.topk, r_weight + (size_t)n0 * s.P * s.topk) != cudaSuccess)
+                rc = BRA_ERR_CUDA;
         }
     };
     if (s.P <= 32)
@@ -157,8 +196,6 @@ static int launch_route(const Shape &s, const void *q, const void *k, int32_t *r
         go(route_kernel<4>);
     else
         go(route_kernel<8>);
-    if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
-    if (cudaFreeAsync(ws, st) != cudaSuccess) rc = BRA_ERR_CUDA;
     return rc;
 }
 
@@ -251,8 +288,113 @@ static int launch_kernel(K kern, int kid, int blocks, int threads, int smem, cud
     return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
 }
 
+// ----------------------------------------------------------------------------- TMA attention
+
+static std::atomic<int> g_variant{BRA_VARIANT_AUTO};
+constexpr unsigned kWaitLimit = 1u << 22;  // mbarrier polls before a kernel gives up
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// (N,H,W,C) bf16 map, boxes of (64 channels, bw columns, bh rows, 1 image), 128-byte
+// swizzle, zero fill outside the map.
+static bool encode_map(CUtensorMap *m, const void *base, const Shape &s, int bw, int bh) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)s.C, (cuuint64_t)s.W, (cuuint64_t)s.H, (cuuint64_t)s.N};
+    cuuint64_t strides[3] = {(cuuint64_t)s.C * 2, (cuuint64_t)s.W * s.C * 2, (cuuint64_t)s.H * s.W * s.C * 2};
+    cuuint32_t box[4] = {64u, (cuuint32_t)bw, (cuuint32_t)bh, 1u};
+    cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// TMA kernel shape: 64 or 128 channels (HG heads) and RB region rows per CTA, at most
+// 8 warps of (head, 16-query tile) and 128 queries; prefer two CTAs per SM.
+static bool plan_tma(const Shape &s, TmaAttnParams &p, int &threads, int &smem) {
+    if (s.dtype != BRA_BF16 || s.hr > 256 || s.wr + 4 > 256) return false;
+    for (int limit : {112 * 1024, kMaxSmem}) {
+        for (int hg = s.heads; hg >= 1; --hg) {
+            if (s.heads % hg) continue;
+            const int CH = hg * s.d;
+            if (CH != 64 && CH != 128) continue;
+            for (int rb = s.hr; rb >= 1; --rb) {
+                if (s.hr % rb) continue;
+                const int nq = rb * s.wr, qt = (nq + 15) / 16;
+                if (nq > 128 || qt * hg > 8) continue;
+                const TmaSmem L = tma_smem_layout(s.topk, s.w2, qt, rb, s.wr, CH);
+                if (L.total > limit) continue;
+                p.HG = hg;
+                p.RB = rb;
+                p.QT = qt;
+                p.n_hg = s.heads / hg;
+                p.n_rb = s.hr / rb;
+                p.slot = (s.w2 + 7) & ~7;
+                threads = qt * hg * 32;
+                smem = L.total;
+                return true;
+            }
+        }
+    }
+    return false;
+}
+
+static int launch_attend_tma(const Shape &s, const void *q, const void *k, const void *v, const void *w,
+                             const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st,
+                             bool *used) {
+    *used = false;
+    if (g_variant.load() != BRA_VARIANT_AUTO) return BRA_OK;
+    if (!aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
+    TmaAttnParams p;
+    memset(&p, 0, sizeof(p));
+    int threads = 0, smem = 0;
+    if (!plan_tma(s, p, threads, smem)) return BRA_OK;
+    if (!encode_map(&p.tmQ, q, s, s.wr, p.RB) || !encode_map(&p.tmK, k, s, s.wr, s.hr) ||
+        !encode_map(&p.tmV, v, s, s.wr, s.hr) || !encode_map(&p.tmH, v, s, s.wr + 4, p.RB + 4))
+        return BRA_OK;  // no tensor-map support: the generic kernel runs instead
+    p.lce_w = static_cast<const __nv_bfloat16 *>(w);
+    p.lce_b = static_cast<const __nv_bfloat16 *>(b);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.r_idx = r_idx;
+    p.err_flag = err;
+    p.N = s.N;
+    p.H = s.H;
+    p.W = s.W;
+    p.C = s.C;
+    p.heads = s.heads;
+    p.S = s.S;
+    p.topk = s.topk;
+    p.hr = s.hr;
+    p.wr = s.wr;
+    p.w2 = s.w2;
+    p.P = s.P;
+    p.scale_log2 = (float)(1.0 / std::sqrt((double)s.d) * 1.4426950408889634);
+    p.wait_limit = kWaitLimit;
+    const int blocks = s.N * s.P * p.n_rb * p.n_hg;
+    auto kern = s.d == 32 ? attn_tma_kernel<32> : attn_tma_kernel<64>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    *used = true;
+    LaunchScope ls(BRA_KERNEL_ATTN_BF16, st);
+    return launch_pdl(kern, dim3(blocks), dim3(threads), smem, st, p) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
 static int launch_attend(const Shape &s, const void *q, const void *k, const void *v, const void *w,
                          const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st) {
+    bool used = false;
+    int rc = launch_attend_tma(s, q, k, v, w, b, out, r_idx, err, st, &used);
+    if (rc || used) return rc;
     AttnParams p = base_params(s, q, k, v, w, b, out, r_idx, err);
     int threads = 0, smem = 0;
     if (s.dtype == BRA_BF16) {
@@ -283,7 +425,28 @@ using namespace bra;
 
 extern "C" {
 
-int bra_version(void) { return (1 << 16) | 0; }
+int bra_version(void) { return (1 << 16) | 1; }
+
+int bra_set_kernel_variant(int variant) {
+    if (variant != BRA_VARIANT_AUTO && variant != BRA_VARIANT_GENERIC) return -1;
+    return g_variant.exchange(variant);
+}
+
+int bra_device_status(bra_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BRA_ERR_CUDA;
+    int flag = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&flag, g_bra_timeout_flag, sizeof(int)) != cudaSuccess) return BRA_ERR_CUDA;
+    if (flag && cudaMemcpyToSymbol(g_bra_timeout_flag, &zero, sizeof(int)) != cudaSuccess) return BRA_ERR_CUDA;
+    return flag ? BRA_ERR_TIMEOUT : BRA_OK;
+}
+
+int bra_selftest_wait_timeout(unsigned polls, bra_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(polls);
+    return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
 
 long long bra_launch_count(void) { return g_launches.load(); }
 
@@ -339,6 +502,7 @@ const char *bra_status_string(int status) {
         case BRA_ERR_CUDA: return "a CUDA allocation, copy or kernel launch failed";
         case BRA_ERR_INDEX: return "a region index in r_idx lies outside [0, S*S)";
         case BRA_ERR_SCRATCH: return "problem needs more scratch than the static array holds (2*N*S*S*C > BRA_STATIC_SCRATCH_FLOATS)";
+        case BRA_ERR_TIMEOUT: return "a kernel's bounded wait for its tile copies ran out";
         default: return "unknown status";
     }
 }
@@ -351,14 +515,28 @@ int bra_route(const void *q, const void *k, int N, int H, int W, int C, int head
     if (N == 0) return BRA_OK;
     if (!q || !k || !r_idx || !r_weight) return BRA_ERR_NULL;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(r_idx, 4) || !aligned(r_weight, 4)) return BRA_ERR_ALIGN;
-    return launch_route(s, q, k, r_idx, r_weight, reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float *ws = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * (size_t)N * s.P * C * sizeof(float), st) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    rc = launch_route_into(s, q, k, r_idx, r_weight, ws, st);
+    if (cudaFreeAsync(ws, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    return rc;
 }
 
+// The forward with its scratch taken from (and returned to) the stream-ordered pool;
+// the scratch is released after the attention launch so that nothing separates the
+// route and attention kernels on the stream.
 static int forward_device(const Shape &s, const void *q, const void *k, const void *v, const void *lce_w,
                           const void *lce_b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st) {
-    int rc = launch_route(s, q, k, r_idx, r_weight, st);
-    if (rc) return rc;
-    return launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, nullptr, st);
+    float *ws = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * (size_t)s.N * s.P * s.C * sizeof(float), st) !=
+        cudaSuccess)
+        return BRA_ERR_CUDA;
+    int rc = launch_route_into(s, q, k, r_idx, r_weight, ws, st);
+    if (rc == BRA_OK) rc = launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, nullptr, st);
+    if (cudaFreeAsync(ws, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    return rc;
 }
 
 int bra_forward(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b, int N,
@@ -468,51 +646,6 @@ static int static_scratch(float **out) {
     }
     *out = g_static_ptr[dev];
     return BRA_OK;
-}
-
-// Steps 1-3 into caller-provided scratch ws (2*N*S*S*C floats); allocates nothing.
-static int launch_route_into(const Shape &s, const void *q, const void *k, int32_t *r_idx, float *r_weight,
-                             float *ws, cudaStream_t st) {
-    const size_t pooled = (size_t)s.N * s.P * s.C;
-    const dim3 pgrid(s.N * s.P, 2);
-    {
-        LaunchScope ls(BRA_KERNEL_REGION_MEAN, st);
-        if (s.dtype == BRA_BF16)
-            region_mean_kernel<__nv_bfloat16><<<pgrid, kPoolThreads, 0, st>>>(
-                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled,
-                s.H, s.W, s.C, s.S);
-        else
-            region_mean_kernel<float><<<pgrid, kPoolThreads, 0, st>>>(
-                static_cast<const float *>(q), static_cast<const float *>(k), ws, ws + pooled, s.H, s.W, s.C, s.S);
-    }
-    const float scale = 1.0f / sqrtf((float)s.d);
-    const int smem = s.P * (kRouteChunk + 1) * (int)sizeof(float);
-    int rc = BRA_OK;
-    auto go = [&](auto kern) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
-            rc = BRA_ERR_CUDA;
-            return;
-        }
-        for (int n0 = 0; n0 < s.N; n0 += 65535) {
-            const int nb = s.N - n0 < 65535 ? s.N - n0 : 65535;
-            const dim3 g((s.P + kRouteWarps - 1) / kRouteWarps, nb, 1);
-            LaunchScope ls(BRA_KERNEL_ROUTE, st);
-            kern<<<g, kRouteWarps * 32, smem, st>>>(ws + (size_t)n0 * s.P * s.C,
-                                                    ws + pooled + (size_t)n0 * s.P * s.C, s.C, s.P, s.topk,
-                                                    scale, r_idx + (size_t)n0 * s.P * s.topk,
-                                                    r_weight + (size_t)n0 * s.P * s.topk);
-        }
-    };
-    if (s.P <= 32)
-        go(route_kernel<1>);
-    else if (s.P <= 64)
-        go(route_kernel<2>);
-    else if (s.P <= 128)
-        go(route_kernel<4>);
-    else
-        go(route_kernel<8>);
-    if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
-    return rc;
 }
 
 int bra_forward_noalloc(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b,

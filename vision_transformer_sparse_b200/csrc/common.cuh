@@ -96,6 +96,68 @@ __device__ inline uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// ----------------------------------------------------------------------------- packed fp32
+
+// d = a * b + c on two float lanes at once (sm_100 packed FMA).
+__device__ inline float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long ai = *reinterpret_cast<unsigned long long *>(&a);
+    unsigned long long bi = *reinterpret_cast<unsigned long long *>(&b);
+    unsigned long long ci = *reinterpret_cast<unsigned long long *>(&c);
+    unsigned long long di;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(di) : "l"(ai), "l"(bi), "l"(ci));
+    return *reinterpret_cast<float2 *>(&di);
+}
+
+__device__ inline float2 bf16x2_to_float2(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+
+// ----------------------------------------------------------------------------- mbarrier / TMA / PDL
+
+__device__ inline void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ inline void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ inline void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+// One arrival that also adds `bytes` to the transaction count of the current phase.
+__device__ inline void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ inline bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// Bounded wait for phase `parity` of the barrier: gives up after `limit` polls
+// (each poll may suspend the thread for a short hardware-defined time).
+__device__ inline bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// 4-D tiled tensor load (no multicast) into shared memory, completing on `bar`.
+__device__ inline void tma_load_4d(uint32_t dst, const void *tmap, int c0, int c1, int c2, int c3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];\n" ::"r"(dst),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        : "memory");
+}
+
+// Programmatic dependent launch: wait for the preceding grid's results / let the
+// next grid start its independent prologue.
+__device__ inline void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ inline void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 __device__ inline float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));

@@ -12,50 +12,70 @@ namespace bra {
 
 constexpr int kPoolThreads = 256;
 
-// One CTA per (image, region, tensor): blockIdx.x = n*P + p, blockIdx.y = 0 (q) / 1 (k).
-// Threads own a 16-byte channel group and stride over the region's tokens; partial
-// sums meet in shared memory. Output: float32 means, (N, P, C) each.
+// One thread per (tensor, image, region, 16-byte channel group, token slot): it sums
+// the region's tokens whose column is congruent to its slot modulo `ns`, issuing its
+// 16-byte loads eight at a time so that many are in flight; the ns slots of a unit
+// are adjacent lanes G apart and meet by shuffles. ns divides wr and G*ns divides 32
+// (or ns = 1). Output: float32 means, (N, P, C) for q and for k.
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 region_mean_kernel(const T *__restrict__ q, const T *__restrict__ k, float *__restrict__ q_r,
-                   float *__restrict__ k_r, int H, int W, int C, int S) {
+                   float *__restrict__ k_r, int N, int H, int W, int C, int S, int ns_log2,
+                   long long total) {
     constexpr int V = Elem<T>::kVec;
-    __shared__ float red[kPoolThreads * V];  // [slots][C] with slots*C == threads*V
-    const int P = S * S;
-    const int np = blockIdx.x;
-    const int n = np / P, p = np - n * P;
+    const long long t = (long long)blockIdx.x * kPoolThreads + threadIdx.x;
+    const bool valid = t < total;
+    const int G = C / V, ns = 1 << ns_log2, P = S * S;
+    const long long tt = valid ? t : 0;
+    const int g = (int)(tt % G);
+    const long long rest = tt / G;
+    const int s = (int)(rest & (ns - 1));
+    const long long u = rest >> ns_log2;
+    const long long NP = (long long)N * P;
+    const int tensor = (int)(u / NP);
+    const long long np = u - tensor * NP;
+    const int n = (int)(np / P), p = (int)(np - (long long)n * P);
     const int j = p / S, i = p - j * S;
-    const int hr = H / S, wr = W / S, w2 = hr * wr;
-    const T *x = blockIdx.y ? k : q;
-    float *dst = blockIdx.y ? k_r : q_r;
+    const int hr = H / S, wr = W / S;
+    const T *x = tensor ? k : q;
+    const T *origin = x + (((size_t)n * H + j * hr) * W + i * wr) * C + g * V;
+    const int count = valid ? hr * (wr >> ns_log2) : 0;
 
-    const int G = C / V;                   // channel groups
-    const int slots = kPoolThreads / G;    // token slots
-    const int g = threadIdx.x % G, s = threadIdx.x / G;
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
-    if (s < slots) {
-        const size_t img = (size_t)n * H * W;
-#pragma unroll 4
-        for (int t = s; t < w2; t += slots) {
-            const int th = t / wr, tw = t - th * wr;
-            const size_t pix = img + (size_t)(j * hr + th) * W + (i * wr + tw);
-            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + pix * C + g * V));
+    int th = 0, tw = s;
+    for (int it = 0; it < count; it += 8) {
+        uint4 buf[8];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            buf[b] = make_uint4(0u, 0u, 0u, 0u);
+            if (it + b < count) {
+                buf[b] = __ldg(reinterpret_cast<const uint4 *>(origin + ((size_t)th * W + tw) * C));
+                tw += ns;
+                if (tw >= wr) {
+                    tw = s;
+                    ++th;
+                }
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
             float f[V];
-            unpack16(u, f, x);
+            unpack16(buf[b], f, x);
 #pragma unroll
             for (int e = 0; e < V; ++e) acc[e] += f[e];
         }
-#pragma unroll
-        for (int e = 0; e < V; ++e) red[s * C + g * V + e] = acc[e];
     }
-    __syncthreads();
-    const float inv_count = 1.0f / (float)w2;
-    for (int c = threadIdx.x; c < C; c += kPoolThreads) {
-        float sum = 0.f;
-        for (int t = 0; t < slots; ++t) sum += red[t * C + c];
-        dst[(size_t)np * C + c] = sum * inv_count;
+    for (int off = G; off < (G << ns_log2); off <<= 1)
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    if (valid && s == 0) {
+        float *dst = (tensor ? k_r : q_r) + (size_t)np * C + g * V;
+        const float w2 = (float)(hr * wr);
+#pragma unroll
+        for (int e = 0; e < V; e += 4)
+            *reinterpret_cast<float4 *>(dst + e) = make_float4(acc[e] / w2, acc[e + 1] / w2, acc[e + 2] / w2, acc[e + 3] / w2);
     }
 }
 
@@ -68,43 +88,69 @@ __device__ inline bool route_before(float av, int ai, float bv, int bi) {
 }
 
 constexpr int kRouteWarps = 8;
-constexpr int kRouteChunk = 64;  // channels of k_r staged in shared memory at a time
+
+// Channels of k_r staged in shared memory per pass, for P regions: the largest
+// multiple of 32 (at most C) whose [P][cc+1] tile plus 8 query rows fit in 96 KB.
+inline int route_chunk(int P, int C) {
+    int cc = C;
+    while (cc > 32 && (P * (cc + 1) + 4 + kRouteWarps * cc) * 4 > 96 * 1024) cc -= 32;
+    return cc;
+}
+inline int route_qoff(int P, int cc) { return (P * (cc + 1) + 3) & ~3; }  // 16-byte aligned query rows
+inline int route_smem_bytes(int P, int cc) { return (route_qoff(P, cc) + kRouteWarps * cc) * 4; }
 
 // One warp per affinity row (image n, query region p). Lane l holds columns
 // l + 32e (e < E), E*32 >= P. The row is sorted with a bitonic network over
 // 32*E (value, index) pairs — in registers across e, with shuffles across lanes —
-// and the first topk entries are the routing. Shared memory: k_r chunk [P][65].
+// and the first topk entries are the routing. Shared memory: k_r chunk [P][cc+1]
+// (odd pitch: conflict-free column reads) and the CTA's 8 query rows [8][cc].
 template <int E>
 __global__ void __launch_bounds__(kRouteWarps * 32)
-route_kernel(const float *__restrict__ q_r, const float *__restrict__ k_r, int C, int P, int topk,
+route_kernel(const float *__restrict__ q_r, const float *__restrict__ k_r, int C, int P, int topk, int cc,
              float scale, int32_t *__restrict__ r_idx, float *__restrict__ r_weight) {
-    extern __shared__ float kr_s[];  // [P][kRouteChunk + 1]
+    extern __shared__ float kr_s[];
+    float *q_s = kr_s + ((P * (cc + 1) + 3) & ~3);
     constexpr int PP = 32 * E;
+    griddep_wait();               // pooled means come from the preceding kernel
+    griddep_launch_dependents();  // the attention kernel may start its prologue
     const int n = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int p = blockIdx.x * kRouteWarps + warp;
+    const int p0 = blockIdx.x * kRouteWarps;
+    const int p = p0 + warp;
     const bool row_ok = p < P;
-    const float *qrow = q_r + ((size_t)n * P + (row_ok ? p : 0)) * C;
     const float *kimg = k_r + (size_t)n * P * C;
+    const float *qimg = q_r + (size_t)n * P * C;
 
     float dot[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) dot[e] = 0.f;
 
-    for (int c0 = 0; c0 < C; c0 += kRouteChunk) {
-        const int cw = min(kRouteChunk, C - c0);
+    for (int c0 = 0; c0 < C; c0 += cc) {
+        const int cw = min(cc, C - c0);  // multiple of 4
+        const int q4 = cw >> 2;
         __syncthreads();
-        for (int idx = threadIdx.x; idx < P * cw; idx += blockDim.x) {
-            const int r = idx / cw, c = idx - r * cw;
-            kr_s[r * (kRouteChunk + 1) + c] = kimg[(size_t)r * C + c0 + c];
+        for (int idx = threadIdx.x; idx < P * q4; idx += blockDim.x) {
+            const int r = idx / q4, c = (idx - r * q4) * 4;
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(kimg + (size_t)r * C + c0 + c));
+            float *d = kr_s + r * (cc + 1) + c;
+            d[0] = v.x;
+            d[1] = v.y;
+            d[2] = v.z;
+            d[3] = v.w;
+        }
+        for (int idx = threadIdx.x; idx < kRouteWarps * q4; idx += blockDim.x) {
+            const int r = idx / q4, c = (idx - r * q4) * 4;
+            const int pr = min(p0 + r, P - 1);
+            *reinterpret_cast<float4 *>(q_s + r * cc + c) =
+                __ldg(reinterpret_cast<const float4 *>(qimg + (size_t)pr * C + c0 + c));
         }
         __syncthreads();
         for (int c = 0; c < cw; ++c) {
-            const float qv = scale * __ldg(qrow + c0 + c);
+            const float qv = scale * q_s[warp * cc + c];
 #pragma unroll
             for (int e = 0; e < E; ++e) {
                 const int col = lane + 32 * e;
-                if (col < P) dot[e] = fmaf(qv, kr_s[col * (kRouteChunk + 1) + c], dot[e]);
+                if (col < P) dot[e] = fmaf(qv, kr_s[col * (cc + 1) + c], dot[e]);
             }
         }
     }
