@@ -158,9 +158,16 @@ enum {
 long long bra_launch_count(void);
 
 /* Start tracing: until bra_trace_end, every kernel launch is bracketed by two
- * CUDA events recorded on its own stream. Launches inside a CUDA graph capture
- * are not traced. Returns BRA_OK. */
+ * CUDA events recorded on its own stream; inside a CUDA graph capture the events
+ * become event-record nodes of the graph (see bra_trace_read). Returns BRA_OK. */
 int bra_trace_begin(void);
+
+/* Without stopping the trace: wait for the recorded events and write, per kernel
+ * class, the device time between each recorded pair summed over all pairs, and the
+ * number of pairs. A pair recorded inside a CUDA graph capture is re-recorded by
+ * every replay of that graph, so reading after a replay gives that replay's times.
+ * Returns BRA_OK or BRA_ERR_CUDA. */
+int bra_trace_read(double *ms, long long *launches);
 
 /* Stop tracing, wait for the recorded events and write, per kernel class
  * (BRA_KERNEL_CLASSES entries each), the summed device time in milliseconds and
@@ -174,16 +181,19 @@ const char *bra_kernel_name(int kernel_class);
 /* ---------------------------------------------------------------------------
  * Kernel selection and device status.
  *
- * bfloat16 attention runs in one of two kernels that compute the same function:
- * the TMA kernel (tile boxes fetched by the tensor memory accelerator) where the
- * shape allows it (64 or 128 channels per CTA, every tile within the shared-memory
- * budget, 4-byte aligned lce_w and lce_b), else the generic kernel (16-byte cp.async
- * pieces). */
-enum { BRA_VARIANT_AUTO = 0, BRA_VARIANT_GENERIC = 1 };
+ * bfloat16 attention runs in one of three kernels that compute the same function.
+ * By default (BRA_VARIANT_AUTO) it is the persistent pipeline kernel (tile boxes
+ * fetched by the tensor memory accelerator into multi-stage shared memory by a
+ * producer warp, consumed by attention warps) where the shape allows it (64 or 128
+ * channels per CTA, every stage within the shared-memory budget, 4-byte aligned
+ * lce_w and lce_b), else the generic kernel (16-byte cp.async pieces, one CTA per
+ * work unit). BRA_VARIANT_TMA selects the one-unit-per-CTA TMA kernel (same shape
+ * rules as the pipeline), BRA_VARIANT_GENERIC the generic kernel. */
+enum { BRA_VARIANT_AUTO = 0, BRA_VARIANT_GENERIC = 1, BRA_VARIANT_TMA = 2 };
 
 /* Select the attention kernel for all later calls in this process (for testing and
- * comparison): BRA_VARIANT_AUTO (default) or BRA_VARIANT_GENERIC. Returns the
- * previous setting, or -1 for an unknown variant. */
+ * comparison): BRA_VARIANT_AUTO (default), BRA_VARIANT_GENERIC or BRA_VARIANT_TMA.
+ * Returns the previous setting, or -1 for an unknown variant. */
 int bra_set_kernel_variant(int variant);
 
 /* Synchronise `stream`, then report whether any kernel of this library gave up a

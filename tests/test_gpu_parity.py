@@ -44,11 +44,22 @@ def _lib(bra_lib):
     return bra_lib
 
 
+VARIANTS = {"auto": 0, "generic": 1, "tma": 2}
+
+
 @pytest.fixture(params=["auto", "generic"])
 def variant(request):
-    """Run a test under the automatic kernel choice (TMA kernel where the shape
-    allows) and again with the generic cp.async kernel forced."""
-    prev = bra.set_kernel_variant(bra.VARIANT_AUTO if request.param == "auto" else bra.VARIANT_GENERIC)
+    """Run a test under the automatic kernel choice (persistent TMA pipeline where the
+    shape allows) and again with the generic cp.async kernel forced."""
+    prev = bra.set_kernel_variant(VARIANTS[request.param])
+    yield request.param
+    bra.set_kernel_variant(prev)
+
+
+@pytest.fixture(params=["auto", "generic", "tma"])
+def any_variant(request):
+    """All three attention kernels, including the one-unit-per-CTA TMA kernel."""
+    prev = bra.set_kernel_variant(VARIANTS[request.param])
     yield request.param
     bra.set_kernel_variant(prev)
 
@@ -77,7 +88,7 @@ SMALL = [
 
 
 @pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
-def test_small_shapes(shape, variant):
+def test_small_shapes(shape, any_variant):
     N, H, W, C, heads, S, topk, dtype = shape
     w = synth.Workload("small", 40 + sum(shape[:7]), N, H, W, C, heads, S, topk, dtype,
                        region_bias=0.5, lce_b_std=0.05, lce_w_std=0.1)
@@ -104,7 +115,7 @@ def test_route_entry_point_matches_forward():
     assert rep.ok, rep.notes
 
 
-def test_attend_given_routing_with_duplicates_and_any_order(variant):
+def test_attend_given_routing_with_duplicates_and_any_order(any_variant):
     w = synth.WORKLOADS["cls_stage2_224"].with_(N=4)
     inp = synth.make_inputs(w)
     d = to_dev(inp, w.dtype)
@@ -130,7 +141,7 @@ def test_bounded_wait_reports_timeout_and_recovers():
     assert_parity(w, synth.make_inputs(w))
 
 
-def test_attend_rejects_out_of_range_region_index(variant):
+def test_attend_rejects_out_of_range_region_index(any_variant):
     """The kernel checks every index it reads; a bad one is reported, never dereferenced."""
     w = synth.WORKLOADS["cls_stage2_224"].with_(N=1)
     d = to_dev(synth.make_inputs(w), w.dtype)

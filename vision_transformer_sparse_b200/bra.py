@@ -20,13 +20,13 @@ _lib = None
 BRA_F32, BRA_BF16 = 0, 1
 STATUS = {0: "BRA_OK", 1: "BRA_ERR_NULL", 2: "BRA_ERR_SHAPE", 3: "BRA_ERR_ALIGN", 4: "BRA_ERR_DTYPE",
           5: "BRA_ERR_CUDA", 6: "BRA_ERR_INDEX", 7: "BRA_ERR_SCRATCH", 8: "BRA_ERR_TIMEOUT"}
-VARIANT_AUTO, VARIANT_GENERIC = 0, 1
+VARIANT_AUTO, VARIANT_GENERIC, VARIANT_TMA = 0, 1, 2
 STATIC_SCRATCH_FLOATS = 4 * 1024 * 1024
 # entry points declared in include/bra.h
 SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
            "bra_status_string",
            "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name",
-           "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout")
+           "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout", "bra_trace_read")
 KERNEL_CLASSES = 4
 
 
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.bra_trace_begin.restype = i
         L.bra_trace_end.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
         L.bra_trace_end.restype = i
+        L.bra_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+        L.bra_trace_read.restype = i
         L.bra_kernel_name.argtypes = [i]
         L.bra_kernel_name.restype = ctypes.c_char_p
         L.bra_set_kernel_variant.argtypes = [i]
@@ -185,6 +187,14 @@ def launch_count() -> int:
 
 def trace_begin() -> None:
     _raise(lib().bra_trace_begin(), "bra_trace_begin")
+
+
+def trace_read() -> dict:
+    """{kernel name: (milliseconds, pairs)} summed over the recorded pairs, trace kept."""
+    ms = (ctypes.c_double * KERNEL_CLASSES)()
+    n = (ctypes.c_longlong * KERNEL_CLASSES)()
+    _raise(lib().bra_trace_read(ms, n), "bra_trace_read")
+    return {lib().bra_kernel_name(i).decode(): (ms[i], n[i]) for i in range(KERNEL_CLASSES)}
 
 
 def trace_end() -> dict:

@@ -36,7 +36,7 @@ struct TmaAttnParams {
     CUtensorMap tmQ;  // q, box (64, wr, RB, 1)
     CUtensorMap tmK;  // k, box (64, wr, hr, 1)
     CUtensorMap tmV;  // v, box (64, wr, hr, 1)
-    CUtensorMap tmH;  // v, box (64, wr + 4, RB + 4, 1): the LCE halo
+    CUtensorMap tmH;  // v, box (64, wr + 4, RB + 4, 1), unswizzled: the LCE halo
     const __nv_bfloat16 *lce_w, *lce_b;
     __nv_bfloat16 *out;
     const int32_t *r_idx;
@@ -99,6 +99,73 @@ __device__ inline uint32_t swz(uint32_t tile, int row, int col) {
 }
 
 constexpr int kRowInvalid = 0x40000000;  // rowmap flag: key masked out of the softmax
+
+// LCE epilogue rows for one (channel pair, pixel column, group of RT output rows).
+// The halo tile is unswizzled: pixel (hy, hx) is the 128-byte row hy*(wr+4)+hx of its
+// 64-channel half, so the five taps of a row sit at immediate offsets of one address.
+// acc[r] collects bias + sum_{a,b} w[a][b] * V[r0+r+a][xx+b]; every loaded halo row
+// feeds each output row it touches, with RT fixed at compile time (no register moves).
+template <int RT>
+__device__ __forceinline__ void lce_rows(uint32_t tH, int hw, int xx, int r0, int chl, const float2 *wt,
+                                         float2 bias, const float *sO, int o_ld, int wr, int cl,
+                                         __nv_bfloat16 *orow, size_t row_stride) {
+    float2 acc[RT];
+#pragma unroll
+    for (int r = 0; r < RT; ++r) acc[r] = bias;
+#pragma unroll
+    for (int hy = 0; hy < RT + 4; ++hy) {
+        const uint32_t ra = tH + ((r0 + hy) * hw + xx) * 128 + chl * 2;
+        float2 v[5];
+#pragma unroll
+        for (int b = 0; b < 5; ++b) v[b] = bf16x2_to_float2(ld_shared_u32(ra + b * 128));
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const int a = hy - r;
+            if (a >= 0 && a < 5) {
+#pragma unroll
+                for (int b = 0; b < 5; ++b) acc[r] = ffma2(wt[a * 5 + b], v[b], acc[r]);
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        const float2 o = *reinterpret_cast<const float2 *>(sO + ((r0 + r) * wr + xx) * o_ld + cl);
+        *reinterpret_cast<__nv_bfloat162 *>(orow + (size_t)(r0 + r) * row_stride) =
+            __floats2bfloat162_rn(o.x + acc[r].x, o.y + acc[r].y);
+    }
+}
+
+// Rows per epilogue item: 4 when RB allows, else 2, else 1.
+__host__ __device__ inline int lce_row_span(int RB) { return RB % 4 == 0 ? 4 : (RB % 2 == 0 ? 2 : 1); }
+
+// The whole LCE epilogue of a unit: items = (channel pair, column, row group), spread
+// over `nthreads` threads starting at `t0`. `load_weights(cp)` refreshes the thread's
+// weight registers when its channel pair changes.
+// out_px0 points at out[n][y0][x0][c0]; C is the pixel pitch, row_stride = W*C.
+template <typename LoadW>
+__device__ __forceinline__ void lce_epilogue_tma(uint32_t halo_tile, int halo_half, int CH, int wr, int RB,
+                                                 const float *sO, int o_ld, __nv_bfloat16 *out_px0, int C,
+                                                 size_t row_stride, int t0, int nthreads, int &w_pair,
+                                                 const float2 *wt, const float2 &bias, LoadW &&load_weights) {
+    const int npairs = CH / 2, hw = wr + 4, RT = lce_row_span(RB);
+    const int items = npairs * wr * (RB / RT);
+    for (int item = t0; item < items; item += nthreads) {
+        const int cp = item & (npairs - 1);
+        const int rest = item / npairs;
+        const int xx = rest % wr, rg = rest / wr;
+        if (cp != w_pair) load_weights(cp);
+        const int cl = 2 * cp;
+        const uint32_t tH = halo_tile + (cl >> 6) * halo_half;
+        const int chl = cl & 63;
+        __nv_bfloat16 *orow = out_px0 + (size_t)xx * C + cl;
+        if (RT == 4)
+            lce_rows<4>(tH, hw, xx, rg * 4, chl, wt, bias, sO, o_ld, wr, cl, orow, row_stride);
+        else if (RT == 2)
+            lce_rows<2>(tH, hw, xx, rg * 2, chl, wt, bias, sO, o_ld, wr, cl, orow, row_stride);
+        else
+            lce_rows<1>(tH, hw, xx, rg, chl, wt, bias, sO, o_ld, wr, cl, orow, row_stride);
+    }
+}
 
 template <int D>
 __global__ void __launch_bounds__(256) attn_tma_kernel(const __grid_constant__ TmaAttnParams prm) {
@@ -347,37 +414,9 @@ __global__ void __launch_bounds__(256) attn_tma_kernel(const __grid_constant__ T
     __syncthreads();
 
     // ---------------------------------------------------------------- LCE epilogue
-    // thread = (channel pair, pixel column); slides a 5x5 window of V down the RB rows
-    const int wr = prm.wr, hw = wr + 4;
-    for (int item = tid; item < npairs * wr; item += blockDim.x) {
-        const int cp = item % npairs, xx = item / npairs;
-        if (cp != w_pair) load_weights(cp);
-        const int cl = 2 * cp;
-        const uint32_t tH = base + L.halo + (cl >> 6) * L.halo_half;
-        const int chl = cl & 63;
-        float2 win[5][5];
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 5; ++b) win[a + 1][b] = bf16x2_to_float2(ld_shared_u32(swz(tH, a * hw + xx + b, chl)));
-        __nv_bfloat16 *orow = prm.out + (((size_t)n * prm.H + y0) * prm.W + x0 + xx) * prm.C + c0 + cl;
-        for (int r = 0; r < prm.RB; ++r) {
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int b = 0; b < 5; ++b) win[a][b] = win[a + 1][b];
-#pragma unroll
-            for (int b = 0; b < 5; ++b) win[4][b] = bf16x2_to_float2(ld_shared_u32(swz(tH, (r + 4) * hw + xx + b, chl)));
-            float2 acc2 = bias;
-#pragma unroll
-            for (int a = 0; a < 5; ++a)
-#pragma unroll
-                for (int b = 0; b < 5; ++b) acc2 = ffma2(wt[a * 5 + b], win[a][b], acc2);
-            const float2 o = *reinterpret_cast<const float2 *>(sO + (r * wr + xx) * o_ld + cl);
-            *reinterpret_cast<__nv_bfloat162 *>(orow + (size_t)r * prm.W * prm.C) =
-                __floats2bfloat162_rn(o.x + acc2.x, o.y + acc2.y);
-        }
-    }
+    lce_epilogue_tma(base + L.halo, L.halo_half, CH, prm.wr, prm.RB, sO, o_ld,
+                     prm.out + (((size_t)n * prm.H + y0) * prm.W + x0) * prm.C + c0, prm.C,
+                     (size_t)prm.W * prm.C, tid, blockDim.x, w_pair, wt, bias, load_weights);
 }
 
 }  // namespace bra

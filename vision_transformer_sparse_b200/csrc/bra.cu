@@ -10,12 +10,16 @@
 // The route and attention kernels are launched with programmatic dependent launch,
 // so each may start (and the attention kernel may fetch its q tile and v halo)
 // while the previous kernel drains.
+#include <algorithm>
 #include <atomic>
 #include <climits>
+#include <cstdio>
+#include <cstdlib>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -23,6 +27,7 @@
 
 #include "../../include/bra.h"
 #include "attn.cuh"
+#include "attn_pipe.cuh"
 #include "attn_tma.cuh"
 #include "route.cuh"
 
@@ -50,13 +55,15 @@ class LaunchScope {
         std::lock_guard<std::mutex> g(g_trace_mu);
         if (!g_tracing) return;
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return;
+        // inside a stream capture the pair becomes event-record nodes of the graph
+        flags_ = cs == cudaStreamCaptureStatusNone ? cudaEventRecordDefault : cudaEventRecordExternal;
         if (cudaEventCreate(&a_) != cudaSuccess) return;
         if (cudaEventCreate(&b_) != cudaSuccess) {
             cudaEventDestroy(a_);
             return;
         }
-        if (cudaEventRecord(a_, st) != cudaSuccess) {
+        if (cudaEventRecordWithFlags(a_, st, flags_) != cudaSuccess) {
             cudaEventDestroy(a_);
             cudaEventDestroy(b_);
             return;
@@ -65,7 +72,7 @@ class LaunchScope {
     }
     ~LaunchScope() {
         if (!on_) return;
-        cudaEventRecord(b_, st_);
+        cudaEventRecordWithFlags(b_, st_, flags_);
         std::lock_guard<std::mutex> g(g_trace_mu);
         g_trace.push_back({kid_, a_, b_});
     }
@@ -74,6 +81,7 @@ class LaunchScope {
     int kid_;
     cudaStream_t st_;
     cudaEvent_t a_{}, b_{};
+    unsigned flags_ = cudaEventRecordDefault;
     bool on_ = false;
 };
 
@@ -156,22 +164,33 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
     {
         const int V = s.dtype == BRA_BF16 ? 8 : 4;
         const int l = pool_ns_log2(s);
-        const long long total = 2LL * s.N * s.P * (s.C / V) << l;
+        const long long total = (long long)s.N * s.P * (s.C / V) << l;
+        if (total >= INT_MAX - kPoolThreads) return BRA_ERR_SHAPE;
         const unsigned blocks = (unsigned)((total + kPoolThreads - 1) / kPoolThreads);
         LaunchScope ls(BRA_KERNEL_REGION_MEAN, st);
         if (s.dtype == BRA_BF16)
             region_mean_kernel<__nv_bfloat16><<<blocks, kPoolThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled, s.N,
-                s.H, s.W, s.C, s.S, l, total);
+                s.H, s.W, s.C, s.S, l, (int)total);
         else
             region_mean_kernel<float><<<blocks, kPoolThreads, 0, st>>>(static_cast<const float *>(q),
                                                                       static_cast<const float *>(k), ws,
-                                                                      ws + pooled, s.N, s.H, s.W, s.C, s.S, l, total);
+                                                                      ws + pooled, s.N, s.H, s.W, s.C, s.S, l, (int)total);
         if (cudaGetLastError() != cudaSuccess) return BRA_ERR_CUDA;
     }
     const float scale = 1.0f / sqrtf((float)s.d);
-    const int cc = route_chunk(s.P, s.C);
-    const int smem = route_smem_bytes(s.P, cc);
+    const int E = s.P <= 32 ? 1 : s.P <= 64 ? 2 : s.P <= 128 ? 4 : 8;
+    // rows per CTA: as many as still leave about one CTA per SM
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    int rpw = 4;
+    while (rpw > 1 && (long long)s.N * ((s.P + kRouteWarps * rpw - 1) / (kRouteWarps * rpw)) < sms) rpw >>= 1;
+    const int rows = kRouteWarps * rpw;
+    int cc = route_chunk(32 * E, rows, s.C);
+    while (s.C % cc) cc -= 32;  // equal passes: one divisor for the staging index
+    const int smem = route_smem_bytes(32 * E, rows, cc);
+    const FastDiv div_q4((uint32_t)(cc / 4));
     int rc = BRA_OK;
     auto go = [&](auto kern) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
@@ -180,22 +199,31 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
         }
         for (int n0 = 0; n0 < s.N && rc == BRA_OK; n0 += 65535) {
             const int nb = s.N - n0 < 65535 ? s.N - n0 : 65535;
-            const dim3 g((s.P + kRouteWarps - 1) / kRouteWarps, nb, 1);
+            const dim3 g((s.P + rows - 1) / rows, nb, 1);
             LaunchScope ls(BRA_KERNEL_ROUTE, st);
             if (launch_pdl(kern, g, dim3(kRouteWarps * 32), smem, st, (const float *)(ws + (size_t)n0 * s.P * s.C),
                            (const float *)(ws + pooled + (size_t)n0 * s.P * s.C), s.C, s.P, s.topk, cc, scale,
-                           r_idx + (size_t)n0 * s.P * s.topk, r_weight + (size_t)n0 * s.P * s.topk) != cudaSuccess)
+                           r_idx + (size_t)n0 * s.P * s.topk, r_weight + (size_t)n0 * s.P * s.topk, div_q4) != cudaSuccess)
                 rc = BRA_ERR_CUDA;
         }
     };
-    if (s.P <= 32)
-        go(route_kernel<1>);
-    else if (s.P <= 64)
-        go(route_kernel<2>);
-    else if (s.P <= 128)
-        go(route_kernel<4>);
+    auto by_rpw = [&](auto e_tag) {
+        constexpr int EE = decltype(e_tag)::value;
+        if (rpw == 4)
+            go(route_kernel<EE, 4>);
+        else if (rpw == 2)
+            go(route_kernel<EE, 2>);
+        else
+            go(route_kernel<EE, 1>);
+    };
+    if (E == 1)
+        by_rpw(std::integral_constant<int, 1>{});
+    else if (E == 2)
+        by_rpw(std::integral_constant<int, 2>{});
+    else if (E == 4)
+        by_rpw(std::integral_constant<int, 4>{});
     else
-        go(route_kernel<8>);
+        by_rpw(std::integral_constant<int, 8>{});
     return rc;
 }
 
@@ -308,7 +336,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // (N,H,W,C) bf16 map, boxes of (64 channels, bw columns, bh rows, 1 image), 128-byte
 // swizzle, zero fill outside the map.
-static bool encode_map(CUtensorMap *m, const void *base, const Shape &s, int bw, int bh) {
+static bool encode_map(CUtensorMap *m, const void *base, const Shape &s, int bw, int bh, bool swizzle = true) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)s.C, (cuuint64_t)s.W, (cuuint64_t)s.H, (cuuint64_t)s.N};
@@ -316,7 +344,8 @@ static bool encode_map(CUtensorMap *m, const void *base, const Shape &s, int bw,
     cuuint32_t box[4] = {64u, (cuuint32_t)bw, (cuuint32_t)bh, 1u};
     cuuint32_t es[4] = {1u, 1u, 1u, 1u};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -354,14 +383,14 @@ static int launch_attend_tma(const Shape &s, const void *q, const void *k, const
                              const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st,
                              bool *used) {
     *used = false;
-    if (g_variant.load() != BRA_VARIANT_AUTO) return BRA_OK;
+    if (g_variant.load() != BRA_VARIANT_TMA) return BRA_OK;
     if (!aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
     TmaAttnParams p;
     memset(&p, 0, sizeof(p));
     int threads = 0, smem = 0;
     if (!plan_tma(s, p, threads, smem)) return BRA_OK;
     if (!encode_map(&p.tmQ, q, s, s.wr, p.RB) || !encode_map(&p.tmK, k, s, s.wr, s.hr) ||
-        !encode_map(&p.tmV, v, s, s.wr, s.hr) || !encode_map(&p.tmH, v, s, s.wr + 4, p.RB + 4))
+        !encode_map(&p.tmV, v, s, s.wr, s.hr) || !encode_map(&p.tmH, v, s, s.wr + 4, p.RB + 4, false))
         return BRA_OK;  // no tensor-map support: the generic kernel runs instead
     p.lce_w = static_cast<const __nv_bfloat16 *>(w);
     p.lce_b = static_cast<const __nv_bfloat16 *>(b);
@@ -390,10 +419,144 @@ static int launch_attend_tma(const Shape &s, const void *q, const void *k, const
     return launch_pdl(kern, dim3(blocks), dim3(threads), smem, st, p) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
 }
 
+// ----------------------------------------------------------------------------- persistent pipeline
+
+struct PipePlan {
+    int HG, RB, QT, NS, NE, threads, smem, ctas_per_sm;
+};
+
+// Choose (head group, row block, stages, epilogue warps): whole regions per unit where
+// possible (a region's routed K/V is then fetched once), then the most resident
+// attention warps per SM, then the most CTAs per SM, then the most stages. The
+// epilogue gets about one warp per 64 LCE items (an item is one channel pair, pixel
+// column and group of up to four rows). BRA_PIPE_PLAN="HG,RB,NS[,NE]" in the
+// environment forces a plan (for tuning sweeps) when that plan is valid.
+static bool plan_pipe(const Shape &s, PipePlan &best) {
+    if (s.dtype != BRA_BF16 || s.hr > 256 || s.wr + 4 > 256) return false;
+    // register cap per thread: 96 for CTAs of up to 160 threads (4 per SM), else 128
+    int force_hg = 0, force_rb = 0, force_ns = 0, force_ne = 0;
+    if (const char *env = getenv("BRA_PIPE_PLAN"))
+        sscanf(env, "%d,%d,%d,%d", &force_hg, &force_rb, &force_ns, &force_ne);
+    bool found = false;
+    long best_score = -1;
+    for (int hg = s.heads; hg >= 1; --hg) {
+        if (s.heads % hg) continue;
+        const int CH = hg * s.d;
+        if (CH != 64 && CH != 128) continue;
+        for (int rb = s.hr; rb >= 1; --rb) {
+            if (s.hr % rb) continue;
+            const int nq = rb * s.wr, qt = (nq + 15) / 16;
+            if (nq > 128 || qt * hg > 8) continue;
+            const int items = (CH / 2) * (s.wr / (s.wr % 2 == 0 ? 2 : 1)) * (rb / lce_row_span(rb));
+            int ne = std::max(1, std::min(7, (items + 31) / 32));
+            if (force_ne > 0) ne = std::min(7, force_ne);
+            for (int ns = 3; ns >= 2; --ns) {
+                if (force_hg && (hg != force_hg || rb != force_rb || ns != force_ns)) continue;
+                const PipeSmem L = pipe_smem_layout(ns, s.topk, s.w2, qt, rb, s.wr, CH);
+                if (L.total > kMaxSmem) continue;
+                const int threads = (qt * hg + ne + 1) * 32;
+                const int regs = threads <= 160 ? 96 : 128;
+                int occ = (228 * 1024) / (L.total + 1024);
+                occ = std::min(occ, 65536 / (threads * regs));
+                occ = std::min(occ, 2048 / threads);
+                if (occ < 1) continue;
+                const long score = (rb == s.hr ? 1L << 40 : 0) + ((long)occ * qt * hg << 16) + (occ << 4) + ns;
+                if (score > best_score) {
+                    best_score = score;
+                    best = {hg, rb, qt, ns, ne, threads, L.total, occ};
+                    found = true;
+                }
+            }
+        }
+    }
+    return found;
+}
+
+static int fill_tma_params(const Shape &s, TmaAttnParams &p, int HG, int RB, int QT, const void *q, const void *k,
+                           const void *v, const void *w, const void *b, void *out, const int32_t *r_idx, int *err,
+                           bool maps = true) {
+    p.HG = HG;
+    p.RB = RB;
+    p.QT = QT;
+    p.n_hg = s.heads / HG;
+    p.n_rb = s.hr / RB;
+    p.slot = (s.w2 + 7) & ~7;
+    if (maps && (!encode_map(&p.tmQ, q, s, s.wr, RB) || !encode_map(&p.tmK, k, s, s.wr, s.hr) ||
+        !encode_map(&p.tmV, v, s, s.wr, s.hr) || !encode_map(&p.tmH, v, s, s.wr + 4, RB + 4, false)))
+        return 0;
+    p.lce_w = static_cast<const __nv_bfloat16 *>(w);
+    p.lce_b = static_cast<const __nv_bfloat16 *>(b);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.r_idx = r_idx;
+    p.err_flag = err;
+    p.N = s.N;
+    p.H = s.H;
+    p.W = s.W;
+    p.C = s.C;
+    p.heads = s.heads;
+    p.S = s.S;
+    p.topk = s.topk;
+    p.hr = s.hr;
+    p.wr = s.wr;
+    p.w2 = s.w2;
+    p.P = s.P;
+    p.scale_log2 = (float)(1.0 / std::sqrt((double)s.d) * 1.4426950408889634);
+    p.wait_limit = kWaitLimit;
+    return 1;
+}
+
+static int launch_attend_pipe(const Shape &s, const void *q, const void *k, const void *v, const void *w,
+                              const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st,
+                              bool *used) {
+    *used = false;
+    if (g_variant.load() != BRA_VARIANT_AUTO) return BRA_OK;
+    if (!aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
+    PipePlan pl;
+    if (!plan_pipe(s, pl)) return BRA_OK;
+    PipeParams pp;
+    memset(&pp, 0, sizeof(pp));
+    if (!fill_tma_params(s, pp.t, pl.HG, pl.RB, pl.QT, q, k, v, w, b, out, r_idx, err)) return BRA_OK;
+    pp.q = static_cast<const __nv_bfloat16 *>(q);
+    pp.k = static_cast<const __nv_bfloat16 *>(k);
+    pp.v = static_cast<const __nv_bfloat16 *>(v);
+    pp.div_wr = FastDiv((uint32_t)s.wr);
+    pp.div_hw = FastDiv((uint32_t)(s.wr + 4));
+    pp.div_nq = FastDiv((uint32_t)(pl.RB * s.wr));
+    pp.div_nh = FastDiv((uint32_t)((pl.RB + 4) * (s.wr + 4)));
+    pp.NS = pl.NS;
+    pp.NE = pl.NE;
+    pp.units = s.N * s.P * pp.t.n_rb * pp.t.n_hg;
+    pp.XT = s.wr % 2 == 0 ? 2 : 1;
+    pp.fast_keys = (s.w2 % 8 == 0 && (s.topk * s.w2) % kKC == 0) ? 1 : 0;
+    pp.div_hg = FastDiv((uint32_t)pp.t.n_hg);
+    pp.div_rb = FastDiv((uint32_t)pp.t.n_rb);
+    pp.div_P = FastDiv((uint32_t)s.P);
+    pp.div_S = FastDiv((uint32_t)s.S);
+    pp.div_wx = FastDiv((uint32_t)(s.wr / pp.XT));
+    auto kern = pl.threads <= 160 ? (s.d == 32 ? attn_pipe_kernel<32, 160, 4> : attn_pipe_kernel<64, 160, 4>)
+                                  : (s.d == 32 ? attn_pipe_kernel<32, 512, 1> : attn_pipe_kernel<64, 512, 1>);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    int dev = 0, sms = 0, occ = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pl.threads, pl.smem) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    if (occ < 1) return BRA_OK;
+    int ctas = std::min(pp.units, sms * occ);
+    ctas -= ctas % pp.t.n_hg;  // a CTA keeps one head group (and its LCE weights)
+    if (ctas < pp.t.n_hg) ctas = pp.t.n_hg;
+    *used = true;
+    LaunchScope ls(BRA_KERNEL_ATTN_BF16, st);
+    return launch_pdl(kern, dim3(ctas), dim3(pl.threads), pl.smem, st, pp) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
 static int launch_attend(const Shape &s, const void *q, const void *k, const void *v, const void *w,
                          const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st) {
     bool used = false;
-    int rc = launch_attend_tma(s, q, k, v, w, b, out, r_idx, err, st, &used);
+    int rc = launch_attend_pipe(s, q, k, v, w, b, out, r_idx, err, st, &used);
+    if (rc || used) return rc;
+    rc = launch_attend_tma(s, q, k, v, w, b, out, r_idx, err, st, &used);
     if (rc || used) return rc;
     AttnParams p = base_params(s, q, k, v, w, b, out, r_idx, err);
     int threads = 0, smem = 0;
@@ -428,7 +591,7 @@ extern "C" {
 int bra_version(void) { return (1 << 16) | 1; }
 
 int bra_set_kernel_variant(int variant) {
-    if (variant != BRA_VARIANT_AUTO && variant != BRA_VARIANT_GENERIC) return -1;
+    if (variant != BRA_VARIANT_AUTO && variant != BRA_VARIANT_GENERIC && variant != BRA_VARIANT_TMA) return -1;
     return g_variant.exchange(variant);
 }
 
@@ -454,6 +617,25 @@ int bra_trace_begin(void) {
     std::lock_guard<std::mutex> g(g_trace_mu);
     g_tracing = true;
     return BRA_OK;
+}
+
+int bra_trace_read(double *ms, long long *launches) {
+    std::lock_guard<std::mutex> g(g_trace_mu);
+    double tot[BRA_KERNEL_CLASSES] = {0};
+    long long cnt[BRA_KERNEL_CLASSES] = {0};
+    int rc = BRA_OK;
+    for (auto &r : g_trace) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            rc = BRA_ERR_CUDA;
+        tot[r.kid] += t;
+        cnt[r.kid] += 1;
+    }
+    for (int i = 0; i < BRA_KERNEL_CLASSES; ++i) {
+        if (ms) ms[i] = tot[i];
+        if (launches) launches[i] = cnt[i];
+    }
+    return rc;
 }
 
 int bra_trace_end(double *ms, long long *launches) {

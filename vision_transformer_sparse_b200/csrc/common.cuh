@@ -50,6 +50,36 @@ __device__ inline void unpack16(const uint4 &u, float *f, const __nv_bfloat16 *)
     }
 }
 
+// ----------------------------------------------------------------------------- invariant division
+
+// Unsigned 32-bit division by a divisor fixed at launch, as a multiply-high and
+// shifts (Granlund & Montgomery, "Division by invariant integers using
+// multiplication", 1994): l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1,
+// q = (t + ((n - t) >> 1)) >> (l - 1) with t = mulhi(m, n). Exact for every n < 2^32.
+struct FastDiv {
+    uint32_t d, m, s1;
+    FastDiv() : d(1), m(0), s1(0) {}
+    explicit FastDiv(uint32_t div) : d(div), m(0), s1(0) {
+        if (d > 1) {
+            uint32_t l = 0;
+            while ((1ull << l) < d) ++l;
+            m = (uint32_t)(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+            s1 = l - 1;
+        }
+    }
+    __device__ __forceinline__ uint32_t div(uint32_t n) const {
+        if (d == 1) return n;
+        const uint32_t t = __umulhi(m, n);
+        return (t + ((n - t) >> 1)) >> s1;
+    }
+    // n / d and n % d
+    __device__ __forceinline__ uint32_t divmod(uint32_t n, uint32_t &r) const {
+        const uint32_t q = div(n);
+        r = n - q * d;
+        return q;
+    }
+};
+
 // ----------------------------------------------------------------------------- async copies
 
 __device__ inline uint32_t smem_u32(const void *p) {
@@ -63,6 +93,17 @@ __device__ inline void cp_async16(void *smem_dst, const void *gmem_src, bool val
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem_dst)),
                  "l"(gmem_src), "r"(src_bytes)
                  : "memory");
+}
+// 16-byte copy to a shared address given as a 32-bit shared-window offset.
+__device__ inline void cp_async16_s(uint32_t smem_dst, const void *gmem_src, bool valid) {
+    const int src_bytes = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_dst), "l"(gmem_src), "r"(src_bytes)
+                 : "memory");
+}
+// Arrive on `bar` once all prior cp.async of this thread have completed (the arrival
+// is not pre-counted: the barrier's expected count includes it).
+__device__ inline void cp_async_mbar_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
 }
 __device__ inline void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N> __device__ inline void cp_async_wait() {
