@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each step directly")
-    ap.add_argument("--variant", default="auto", choices=["auto", "generic", "tma"],
+    ap.add_argument("--variant", default="auto", choices=["auto", "generic", "tma", "split"],
                     help="attention kernel (auto: persistent TMA pipeline where the shape allows)")
     return ap.parse_args()
 
@@ -73,8 +73,12 @@ def algorithmic(w: synth.Workload):
     # the routing read, the LCE parameters
     attn_unique = 4.0 * T * w.C * b + w.N * w.regions * w.topk * 4 + w.C * 26 * b
     pool_bytes = 2.0 * T * w.C * b + 2 * w.N * w.regions * w.C * 4
+    # the one-kernel forward: q, k, v read once, out written once, r_idx and r_weight,
+    # the LCE parameters
+    fused_bytes = 4.0 * T * w.C * b + route_bytes + w.C * 26 * b
     return {"tokens": T, "flops": flops, "gathered_bytes": gathered, "attn_bytes": attn_unique,
-            "pool_bytes": pool_bytes, "route_bytes": route_bytes, "elem_bytes": b}
+            "pool_bytes": pool_bytes, "route_bytes": route_bytes, "fused_bytes": fused_bytes,
+            "elem_bytes": b}
 
 
 def load_peaks():
@@ -98,10 +102,11 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the attention kernel from a committed ncu summary,
-    if it was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "attn_bf16_%s.txt" % workload)
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary
+    (profiles/<kernel>_<workload>.txt), if it was taken on the current kernel source
+    (else None)."""
+    path = os.path.join(ROOT, "profiles", "%s_%s.txt" % (kernel, workload))
     if not os.path.exists(path):
         return None, None
     vals = {}
@@ -269,7 +274,7 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     bra.set_kernel_variant({"auto": bra.VARIANT_AUTO, "generic": bra.VARIANT_GENERIC,
-                            "tma": bra.VARIANT_TMA}[args.variant])
+                            "tma": bra.VARIANT_TMA, "split": bra.VARIANT_SPLIT}[args.variant])
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -418,13 +423,16 @@ def main():
     tflops = acc["flops"] * world * args.steps / (ms / 1e3) / 1e12
 
     peaks, peak_kind = load_peaks()
-    attn_name = "attn_bf16_kernel" if w.dtype == "bf16" else "attn_f32_kernel"
+    # the dominant kernel (largest share of device time) and its algorithmic bytes
+    attn_name = max((v[0], k) for k, v in trace.items() if v[1])[1]
     t_ms, t_n = trace[attn_name]
     attn_s = t_ms / max(t_n, 1) / 1e3
+    alg_bytes = {"bra_image_kernel": acc["fused_bytes"], "region_mean_kernel": acc["pool_bytes"],
+                 "route_kernel": acc["route_bytes"]}.get(attn_name, acc["attn_bytes"])
     step_traced_ms = sum(v[0] for v in trace.values()) / traced_steps
     share = {k: round(v[0] / max(1e-12, sum(x[0] for x in trace.values())), 4) for k, v in trace.items() if v[1]}
-    achieved = acc["attn_bytes"] / attn_s / 1e9
-    traffic, _ = profiled_traffic(w.name)
+    achieved = alg_bytes / attn_s / 1e9
+    traffic, _ = profiled_traffic(attn_name, w.name)
     # the roofline the method's own accounting states: slower of the FLOP term at the
     # tensor peak and the gathered K/V bytes at HBM bandwidth
     t_flop = acc["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
@@ -446,7 +454,7 @@ def main():
         "gpu_launches": gpu_launches,
         "roofline": {"bound": "hbm", "kernel": attn_name, "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": acc["attn_bytes"],
+                     "algorithmic_bytes_per_launch": alg_bytes,
                      "avg_launch_us": attn_s * 1e6, "peak_source": peak_kind},
         "roofline_gathered": {"definition": "max(attention FLOP / bf16 peak, gathered K/V bytes / HBM)",
                               "bound": ns_bound, "roofline_us": max(t_flop, t_gath) * 1e6,

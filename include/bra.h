@@ -150,7 +150,8 @@ enum {
     BRA_KERNEL_ROUTE = 1,       /* steps 2-3: affinity row, top-k, softmax        */
     BRA_KERNEL_ATTN_BF16 = 2,   /* steps 4-5, bfloat16 tensor-core kernel         */
     BRA_KERNEL_ATTN_F32 = 3,    /* steps 4-5, float32 SIMT kernel                 */
-    BRA_KERNEL_CLASSES = 4
+    BRA_KERNEL_FUSED_IMAGE = 4, /* steps 1-5 in one kernel (small images)         */
+    BRA_KERNEL_CLASSES = 5
 };
 
 /* Number of kernels this library has launched since it was loaded (all threads,
@@ -181,18 +182,25 @@ const char *bra_kernel_name(int kernel_class);
 /* ---------------------------------------------------------------------------
  * Kernel selection and device status.
  *
- * bfloat16 attention runs in one of three kernels that compute the same function.
- * By default (BRA_VARIANT_AUTO) it is the persistent pipeline kernel (tile boxes
- * fetched by the tensor memory accelerator into multi-stage shared memory by a
- * producer warp, consumed by attention warps) where the shape allows it (64 or 128
- * channels per CTA, every stage within the shared-memory budget, 4-byte aligned
- * lce_w and lce_b), else the generic kernel (16-byte cp.async pieces, one CTA per
- * work unit). BRA_VARIANT_TMA selects the one-unit-per-CTA TMA kernel (same shape
- * rules as the pipeline), BRA_VARIANT_GENERIC the generic kernel. */
-enum { BRA_VARIANT_AUTO = 0, BRA_VARIANT_GENERIC = 1, BRA_VARIANT_TMA = 2 };
+ * By default (BRA_VARIANT_AUTO) a bfloat16 forward whose images are small runs as
+ * ONE kernel (pooling, routing, attention and LCE fused; one thread-block cluster of
+ * `heads` CTAs per image): this needs d = 32, regions of 4x4 or 2x2 tokens, S*S <= 64,
+ * topk <= 32, heads <= 8 and one head's Q, K and V slices of a whole image within one
+ * CTA's shared memory. Otherwise the forward runs as three kernels (region means,
+ * routing, attention), and bfloat16 attention runs in the persistent pipeline kernel
+ * (tile boxes fetched by the tensor memory accelerator into multi-stage shared memory
+ * by a producer warp, consumed by attention warps and LCE warps) where the shape
+ * allows it (64 or 128 channels per CTA, every stage within the shared-memory budget,
+ * 4-byte aligned lce_w and lce_b), else in the generic kernel (16-byte cp.async
+ * pieces, one CTA per work unit). BRA_VARIANT_SPLIT keeps the three-kernel path
+ * with the automatic attention kernel; BRA_VARIANT_TMA selects the one-unit-per-CTA
+ * TMA attention kernel (same shape rules as the pipeline), BRA_VARIANT_GENERIC the
+ * generic kernel. All variants compute the same function. */
+enum { BRA_VARIANT_AUTO = 0, BRA_VARIANT_GENERIC = 1, BRA_VARIANT_TMA = 2, BRA_VARIANT_SPLIT = 3 };
 
 /* Select the attention kernel for all later calls in this process (for testing and
- * comparison): BRA_VARIANT_AUTO (default), BRA_VARIANT_GENERIC or BRA_VARIANT_TMA.
+ * comparison): BRA_VARIANT_AUTO (default), BRA_VARIANT_GENERIC, BRA_VARIANT_TMA or
+ * BRA_VARIANT_SPLIT.
  * Returns the previous setting, or -1 for an unknown variant. */
 int bra_set_kernel_variant(int variant);
 

@@ -44,21 +44,22 @@ def _lib(bra_lib):
     return bra_lib
 
 
-VARIANTS = {"auto": 0, "generic": 1, "tma": 2}
+VARIANTS = {"auto": 0, "generic": 1, "tma": 2, "split": 3}
 
 
-@pytest.fixture(params=["auto", "generic"])
+@pytest.fixture(params=["auto", "split", "generic"])
 def variant(request):
-    """Run a test under the automatic kernel choice (persistent TMA pipeline where the
-    shape allows) and again with the generic cp.async kernel forced."""
+    """Run a test under the automatic kernel choice (the fused one-kernel forward for
+    small images, else region means + routing + persistent attention pipeline), the
+    three-kernel path forced, and the generic cp.async attention kernel forced."""
     prev = bra.set_kernel_variant(VARIANTS[request.param])
     yield request.param
     bra.set_kernel_variant(prev)
 
 
-@pytest.fixture(params=["auto", "generic", "tma"])
+@pytest.fixture(params=["auto", "split", "generic", "tma"])
 def any_variant(request):
-    """All three attention kernels, including the one-unit-per-CTA TMA kernel."""
+    """Every kernel variant, including the one-unit-per-CTA TMA attention kernel."""
     prev = bra.set_kernel_variant(VARIANTS[request.param])
     yield request.param
     bra.set_kernel_variant(prev)
@@ -84,6 +85,9 @@ SMALL = [
     (2, 12, 18, 128, 2, 3, 4, "f32"),     # f32, d = 64, non-square
     (1, 16, 16, 64, 2, 16, 3, "f32"),     # f32 one-token regions, S = 16
     (1, 60, 60, 96, 3, 5, 2, "bf16"),     # 3 heads, 12x12 regions split over 6 CTAs
+    (1, 12, 12, 64, 2, 6, 5, "bf16"),     # 2x2 regions, 20 keys (ragged chunk), fused path
+    (2, 8, 8, 256, 8, 2, 2, "bf16"),      # 8 heads: a cluster of 8 CTAs per image
+    (3, 20, 20, 64, 2, 5, 7, "bf16"),     # 4x4 regions, 112 keys (two chunks), borders
 ]
 
 

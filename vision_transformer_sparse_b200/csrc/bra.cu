@@ -29,6 +29,7 @@
 #include "attn.cuh"
 #include "attn_pipe.cuh"
 #include "attn_tma.cuh"
+#include "fused_image.cuh"
 #include "route.cuh"
 
 namespace bra {
@@ -336,17 +337,20 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // (N,H,W,C) bf16 map, boxes of (64 channels, bw columns, bh rows, 1 image), 128-byte
 // swizzle, zero fill outside the map.
-static bool encode_map(CUtensorMap *m, const void *base, const Shape &s, int bw, int bh, bool swizzle = true) {
+static bool encode_map_box(CUtensorMap *m, const void *base, const Shape &s, int inner, int bw, int bh,
+                           CUtensorMapSwizzle swizzle) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)s.C, (cuuint64_t)s.W, (cuuint64_t)s.H, (cuuint64_t)s.N};
     cuuint64_t strides[3] = {(cuuint64_t)s.C * 2, (cuuint64_t)s.W * s.C * 2, (cuuint64_t)s.H * s.W * s.C * 2};
-    cuuint32_t box[4] = {64u, (cuuint32_t)bw, (cuuint32_t)bh, 1u};
+    cuuint32_t box[4] = {(cuuint32_t)inner, (cuuint32_t)bw, (cuuint32_t)bh, 1u};
     cuuint32_t es[4] = {1u, 1u, 1u, 1u};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+static bool encode_map(CUtensorMap *m, const void *base, const Shape &s, int bw, int bh, bool swizzle = true) {
+    return encode_map_box(m, base, s, 64, bw, bh, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // TMA kernel shape: 64 or 128 channels (HG heads) and RB region rows per CTA, at most
@@ -509,7 +513,7 @@ static int launch_attend_pipe(const Shape &s, const void *q, const void *k, cons
                               const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st,
                               bool *used) {
     *used = false;
-    if (g_variant.load() != BRA_VARIANT_AUTO) return BRA_OK;
+    if (g_variant.load() != BRA_VARIANT_AUTO && g_variant.load() != BRA_VARIANT_SPLIT) return BRA_OK;
     if (!aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
     PipePlan pl;
     if (!plan_pipe(s, pl)) return BRA_OK;
@@ -572,6 +576,70 @@ static int launch_attend(const Shape &s, const void *q, const void *k, const voi
                      : launch_kernel(attn_f32_kernel<64>, BRA_KERNEL_ATTN_F32, blocks, threads, smem, st, p);
 }
 
+// ----------------------------------------------------------------------------- fused small-image path
+
+constexpr int kImageWarps = 16;
+
+// The whole forward in one cluster launch when the shape allows it (see include/bra.h).
+static int launch_fused_image(const Shape &s, const void *q, const void *k, const void *v, const void *w,
+                              const void *b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st,
+                              bool *used) {
+    *used = false;
+    if (g_variant.load() != BRA_VARIANT_AUTO) return BRA_OK;
+    if (s.dtype != BRA_BF16 || s.d != 32 || s.P > 64 || s.topk > 32 || s.heads > 8) return BRA_OK;
+    if (!((s.hr == 4 && s.wr == 4) || (s.hr == 2 && s.wr == 2))) return BRA_OK;
+    if (s.H + 4 > 256 || s.W + 4 > 256 || !aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
+    const ImageSmem L = image_smem_layout(s.H, s.W, s.P, s.topk, s.w2, kImageWarps);
+    if (L.total > kMaxSmem) return BRA_OK;
+    ImageParams p;
+    memset(&p, 0, sizeof(p));
+    if (!encode_map_box(&p.tmQ, q, s, 32, s.W, s.H, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_map_box(&p.tmK, k, s, 32, s.W, s.H, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_map_box(&p.tmV, v, s, 32, s.W + 4, s.H + 4, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return BRA_OK;
+    p.lce_w = static_cast<const __nv_bfloat16 *>(w);
+    p.lce_b = static_cast<const __nv_bfloat16 *>(b);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.r_idx = r_idx;
+    p.r_weight = r_weight;
+    p.N = s.N;
+    p.H = s.H;
+    p.W = s.W;
+    p.C = s.C;
+    p.heads = s.heads;
+    p.S = s.S;
+    p.topk = s.topk;
+    p.P = s.P;
+    p.scale = (float)(1.0 / std::sqrt((double)s.d));
+    p.scale_log2 = (float)(1.0 / std::sqrt((double)s.d) * 1.4426950408889634);
+    p.wait_limit = kWaitLimit;
+    p.div_S = FastDiv((uint32_t)s.S);
+    p.div_W = FastDiv((uint32_t)s.W);
+    auto kern = s.hr == 4 ? bra_image_kernel<4, 4> : bra_image_kernel<2, 2>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(s.N * s.heads);
+    cfg.blockDim = dim3(kImageWarps * 32);
+    cfg.dynamicSmemBytes = L.total;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = s.heads;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+        cudaGetLastError();  // not schedulable here: the three-kernel path runs instead
+        return BRA_OK;
+    }
+    *used = true;
+    LaunchScope ls(BRA_KERNEL_FUSED_IMAGE, st);
+    return cudaLaunchKernelEx(&cfg, kern, p) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
 // Everything a shape must pass before any CUDA call is made.
 static int check_plan(const Shape &s) {
     int rc = check_shape(s);
@@ -591,7 +659,7 @@ extern "C" {
 int bra_version(void) { return (1 << 16) | 1; }
 
 int bra_set_kernel_variant(int variant) {
-    if (variant != BRA_VARIANT_AUTO && variant != BRA_VARIANT_GENERIC && variant != BRA_VARIANT_TMA) return -1;
+    if (variant < BRA_VARIANT_AUTO || variant > BRA_VARIANT_SPLIT) return -1;
     return g_variant.exchange(variant);
 }
 
@@ -670,6 +738,7 @@ const char *bra_kernel_name(int kernel_class) {
         case BRA_KERNEL_ROUTE: return "route_kernel";
         case BRA_KERNEL_ATTN_BF16: return "attn_bf16_kernel";
         case BRA_KERNEL_ATTN_F32: return "attn_f32_kernel";
+        case BRA_KERNEL_FUSED_IMAGE: return "bra_image_kernel";
         default: return "unknown";
     }
 }
@@ -711,6 +780,9 @@ int bra_route(const void *q, const void *k, int N, int H, int W, int C, int head
 // route and attention kernels on the stream.
 static int forward_device(const Shape &s, const void *q, const void *k, const void *v, const void *lce_w,
                           const void *lce_b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st) {
+    bool fused = false;
+    int frc = launch_fused_image(s, q, k, v, lce_w, lce_b, out, r_idx, r_weight, st, &fused);
+    if (frc || fused) return frc;
     float *ws = nullptr;
     if (cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * (size_t)s.N * s.P * s.C * sizeof(float), st) !=
         cudaSuccess)
