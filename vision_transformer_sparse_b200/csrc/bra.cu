@@ -169,14 +169,26 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
         if (total >= INT_MAX - kPoolThreads) return BRA_ERR_SHAPE;
         const unsigned blocks = (unsigned)((total + kPoolThreads - 1) / kPoolThreads);
         LaunchScope ls(BRA_KERNEL_REGION_MEAN, st);
-        if (s.dtype == BRA_BF16)
-            region_mean_kernel<__nv_bfloat16><<<blocks, kPoolThreads, 0, st>>>(
-                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled, s.N,
-                s.H, s.W, s.C, s.S, l, (int)total);
-        else
-            region_mean_kernel<float><<<blocks, kPoolThreads, 0, st>>>(static_cast<const float *>(q),
-                                                                      static_cast<const float *>(k), ws,
-                                                                      ws + pooled, s.N, s.H, s.W, s.C, s.S, l, (int)total);
+        const bool big = s.w2 >= 64 && s.C / V <= kPoolThreads;  // one CTA per region
+        if (s.dtype == BRA_BF16) {
+            if (big)
+                region_mean_big_kernel<__nv_bfloat16><<<s.N * s.P, kPoolThreads, 0, st>>>(
+                    static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled,
+                    s.H, s.W, s.C, s.S);
+            else
+                region_mean_kernel<__nv_bfloat16><<<blocks, kPoolThreads, 0, st>>>(
+                    static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled,
+                    s.N, s.H, s.W, s.C, s.S, l, (int)total);
+        } else {
+            if (big)
+                region_mean_big_kernel<float><<<s.N * s.P, kPoolThreads, 0, st>>>(
+                    static_cast<const float *>(q), static_cast<const float *>(k), ws, ws + pooled, s.H, s.W, s.C, s.S);
+            else
+                region_mean_kernel<float><<<blocks, kPoolThreads, 0, st>>>(static_cast<const float *>(q),
+                                                                          static_cast<const float *>(k), ws,
+                                                                          ws + pooled, s.N, s.H, s.W, s.C, s.S, l,
+                                                                          (int)total);
+        }
         if (cudaGetLastError() != cudaSuccess) return BRA_ERR_CUDA;
     }
     const float scale = 1.0f / sqrtf((float)s.d);

@@ -85,6 +85,65 @@ region_mean_kernel(const T *__restrict__ q, const T *__restrict__ k, float *__re
     }
 }
 
+// Large regions (w2 >= 64): one CTA per (image, region). Thread = (16-byte channel
+// group g, token slot s) over q and k; slots stride the region's tokens with eight
+// independent loads in flight; partial sums meet in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(kPoolThreads)
+region_mean_big_kernel(const T *__restrict__ q, const T *__restrict__ k, float *__restrict__ q_r,
+                       float *__restrict__ k_r, int H, int W, int C, int S) {
+    constexpr int V = Elem<T>::kVec;
+    __shared__ float red[2][kPoolThreads * V];  // [tensor][slots][C]
+    const int P = S * S, np = blockIdx.x;
+    const int n = np / P, p = np - n * P;
+    const int j = p / S, i = p - j * S;
+    const int hr = H / S, wr = W / S, w2 = hr * wr;
+    const int G = C / V, slots = kPoolThreads / G;
+    const int g = threadIdx.x % G, sl = threadIdx.x / G;
+    const size_t org = (((size_t)n * H + j * hr) * W + i * wr) * C + g * V;
+    float aq[V], ak[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) aq[e] = ak[e] = 0.f;
+    if (sl < slots) {
+        for (int t0 = sl; t0 < w2; t0 += 8 * slots) {
+            uint4 bq[8], bk[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                const int t = t0 + b * slots;
+                bq[b] = bk[b] = make_uint4(0u, 0u, 0u, 0u);
+                if (t < w2) {
+                    const int th = t / wr, tw = t - th * wr;
+                    const size_t off = org + ((size_t)th * W + tw) * C;
+                    bq[b] = __ldg(reinterpret_cast<const uint4 *>(q + off));
+                    bk[b] = __ldg(reinterpret_cast<const uint4 *>(k + off));
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                float f[V];
+                unpack16(bq[b], f, q);
+#pragma unroll
+                for (int e = 0; e < V; ++e) aq[e] += f[e];
+                unpack16(bk[b], f, k);
+#pragma unroll
+                for (int e = 0; e < V; ++e) ak[e] += f[e];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            red[0][sl * C + g * V + e] = aq[e];
+            red[1][sl * C + g * V + e] = ak[e];
+        }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < 2 * C; c += kPoolThreads) {
+        const int tensor = c >= C, cc = c - tensor * C;
+        float sum = 0.f;
+        for (int t = 0; t < slots; ++t) sum += red[tensor][t * C + cc];
+        (tensor ? k_r : q_r)[(size_t)np * C + cc] = sum / (float)w2;
+    }
+}
+
 // ----------------------------------------------------------------------------- top-k
 
 // Strict total order used by the routing: larger logit first, equal logits ->
