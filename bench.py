@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each step directly")
-    ap.add_argument("--variant", default="auto", choices=["auto", "generic", "tma", "split"],
+    ap.add_argument("--variant", default="auto", choices=["auto", "generic", "tma", "split", "pipe"],
                     help="attention kernel (auto: persistent TMA pipeline where the shape allows)")
     return ap.parse_args()
 
@@ -274,7 +274,8 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     bra.set_kernel_variant({"auto": bra.VARIANT_AUTO, "generic": bra.VARIANT_GENERIC,
-                            "tma": bra.VARIANT_TMA, "split": bra.VARIANT_SPLIT}[args.variant])
+                            "tma": bra.VARIANT_TMA, "split": bra.VARIANT_SPLIT,
+                            "pipe": bra.VARIANT_PIPE}[args.variant])
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

@@ -151,7 +151,8 @@ enum {
     BRA_KERNEL_ATTN_BF16 = 2,   /* steps 4-5, bfloat16 tensor-core kernel         */
     BRA_KERNEL_ATTN_F32 = 3,    /* steps 4-5, float32 SIMT kernel                 */
     BRA_KERNEL_FUSED_IMAGE = 4, /* steps 1-5 in one kernel (small images)         */
-    BRA_KERNEL_CLASSES = 5
+    BRA_KERNEL_ATTN_UMMA = 5,   /* steps 4-5, tcgen05 kernel (large regions)       */
+    BRA_KERNEL_CLASSES = 6
 };
 
 /* Number of kernels this library has launched since it was loaded (all threads,
@@ -187,20 +188,30 @@ const char *bra_kernel_name(int kernel_class);
  * `heads` CTAs per image): this needs d = 32, regions of 4x4 or 2x2 tokens, S*S <= 64,
  * topk <= 32, heads <= 8 and one head's Q, K and V slices of a whole image within one
  * CTA's shared memory. Otherwise the forward runs as three kernels (region means,
- * routing, attention), and bfloat16 attention runs in the persistent pipeline kernel
- * (tile boxes fetched by the tensor memory accelerator into multi-stage shared memory
- * by a producer warp, consumed by attention warps and LCE warps) where the shape
- * allows it (64 or 128 channels per CTA, every stage within the shared-memory budget,
- * 4-byte aligned lce_w and lce_b), else in the generic kernel (16-byte cp.async
- * pieces, one CTA per work unit). BRA_VARIANT_SPLIT keeps the three-kernel path
- * with the automatic attention kernel; BRA_VARIANT_TMA selects the one-unit-per-CTA
- * TMA attention kernel (same shape rules as the pipeline), BRA_VARIANT_GENERIC the
- * generic kernel. All variants compute the same function. */
-enum { BRA_VARIANT_AUTO = 0, BRA_VARIANT_GENERIC = 1, BRA_VARIANT_TMA = 2, BRA_VARIANT_SPLIT = 3 };
+ * routing, attention). The bfloat16 attention then runs, in this order of preference:
+ *  - on the 5th-generation tensor cores (tcgen05: scores and probabilities in tensor
+ *    memory, one CTA per SM) when d = 32, a region holds 128 or 256 tokens (H/S a
+ *    multiple of 8, W/S even) and topk * (H/S) * (W/S) <= 256;
+ *  - in the persistent pipeline kernel (tile boxes fetched by the tensor memory
+ *    accelerator into multi-stage shared memory by a producer warp, consumed by
+ *    mma.sync attention warps and LCE warps) where the shape allows it (64 or 128
+ *    channels per CTA, every stage within the shared-memory budget);
+ *  - else in the generic kernel (16-byte cp.async pieces, one CTA per work unit).
+ * The first two need 4-byte aligned lce_w and lce_b. BRA_VARIANT_SPLIT keeps the
+ * three-kernel path with the automatic attention kernel; BRA_VARIANT_PIPE skips the
+ * tcgen05 kernel (pipeline, else generic); BRA_VARIANT_TMA selects the
+ * one-unit-per-CTA TMA attention kernel (same shape rules as the pipeline),
+ * BRA_VARIANT_GENERIC the generic kernel. All variants compute the same function. */
+enum {
+    BRA_VARIANT_AUTO = 0,
+    BRA_VARIANT_GENERIC = 1,
+    BRA_VARIANT_TMA = 2,
+    BRA_VARIANT_SPLIT = 3,
+    BRA_VARIANT_PIPE = 4
+};
 
 /* Select the attention kernel for all later calls in this process (for testing and
- * comparison): BRA_VARIANT_AUTO (default), BRA_VARIANT_GENERIC, BRA_VARIANT_TMA or
- * BRA_VARIANT_SPLIT.
+ * comparison): one of the BRA_VARIANT_* values above.
  * Returns the previous setting, or -1 for an unknown variant. */
 int bra_set_kernel_variant(int variant);
 

@@ -44,20 +44,22 @@ def _lib(bra_lib):
     return bra_lib
 
 
-VARIANTS = {"auto": 0, "generic": 1, "tma": 2, "split": 3}
+VARIANTS = {"auto": 0, "generic": 1, "tma": 2, "split": 3, "pipe": 4}
 
 
-@pytest.fixture(params=["auto", "split", "generic"])
+@pytest.fixture(params=["auto", "split", "pipe", "generic"])
 def variant(request):
     """Run a test under the automatic kernel choice (the fused one-kernel forward for
-    small images, else region means + routing + persistent attention pipeline), the
-    three-kernel path forced, and the generic cp.async attention kernel forced."""
+    small images, else region means + routing + the tcgen05 attention kernel for
+    128/256-token regions or the persistent mma.sync pipeline), the three-kernel path
+    forced, the mma.sync pipeline forced, and the generic cp.async attention kernel
+    forced."""
     prev = bra.set_kernel_variant(VARIANTS[request.param])
     yield request.param
     bra.set_kernel_variant(prev)
 
 
-@pytest.fixture(params=["auto", "split", "generic", "tma"])
+@pytest.fixture(params=["auto", "split", "pipe", "generic", "tma"])
 def any_variant(request):
     """Every kernel variant, including the one-unit-per-CTA TMA attention kernel."""
     prev = bra.set_kernel_variant(VARIANTS[request.param])
@@ -88,6 +90,10 @@ SMALL = [
     (1, 12, 12, 64, 2, 6, 5, "bf16"),     # 2x2 regions, 20 keys (ragged chunk), fused path
     (2, 8, 8, 256, 8, 2, 2, "bf16"),      # 8 heads: a cluster of 8 CTAs per image
     (3, 20, 20, 64, 2, 5, 7, "bf16"),     # 4x4 regions, 112 keys (two chunks), borders
+    (1, 32, 32, 64, 2, 2, 1, "bf16"),     # 256-token regions, 256 keys: tcgen05 kernel
+    (2, 16, 32, 64, 2, 2, 2, "bf16"),     # 8x16 regions, topk 2 -> 256 keys: tcgen05
+    (1, 16, 32, 128, 4, 2, 1, "bf16"),    # 8x16 regions, 128 keys, 4 heads: tcgen05
+    (3, 48, 48, 96, 3, 3, 1, "bf16"),     # 16x16 regions, 3 heads, 3 images: tcgen05
 ]
 
 
@@ -159,6 +165,54 @@ def test_attend_rejects_out_of_range_region_index(any_variant):
     r_idx.clamp_(0, w.regions - 1)
     bra.attend(d["q"], d["k"], d["v"], d["lce_w"], d["lce_b"], w.heads, w.S, r_idx)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("shape", [(2, 32, 32, 64, 2, 2, 1), (2, 16, 32, 64, 2, 2, 2)], ids=["w256k1", "w128k2"])
+def test_tcgen05_attend_duplicates_and_bad_index(shape):
+    """128/256-token regions (the tcgen05 kernel): duplicated routed regions count
+    twice; an out-of-range index is reported (status 6) and its keys are masked."""
+    N, H, W, C, heads, S, topk = shape
+    w = synth.Workload("small", 77, N, H, W, C, heads, S, topk, "bf16", region_bias=0.5, lce_b_std=0.05,
+                       lce_w_std=0.1)
+    inp = synth.make_inputs(w)
+    d = to_dev(inp, w.dtype)
+    rng = np.random.Generator(np.random.PCG64(9))
+    r_idx = rng.integers(0, w.regions, size=(w.N, w.regions, w.topk)).astype(np.int32)
+    if topk > 1:
+        r_idx[:, 1:, 1] = r_idx[:, 1:, 0]
+    out = bra.attend(d["q"], d["k"], d["v"], d["lce_w"], d["lce_b"], w.heads, w.S, torch.from_numpy(r_idx).cuda())
+    ref = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], w.heads, w.S, r_idx)
+    rep = compare.Report()
+    compare.check_output(out.float().cpu().numpy(), ref, w.dtype, rep)
+    assert rep.ok, rep.notes
+    bad = torch.from_numpy(r_idx).cuda()
+    bad[0, 1, 0] = w.regions
+    with pytest.raises(bra.BraError) as e:
+        bra.attend(d["q"], d["k"], d["v"], d["lce_w"], d["lce_b"], w.heads, w.S, bad)
+    assert e.value.status == 6
+    assert bra.device_status() == 0
+
+
+def test_tcgen05_row_with_dominant_far_key_is_exact():
+    """256-token regions (the tcgen05 kernel): one query whose logit for a key far down
+    the row exceeds every logit of the first keys by hundreds, so that probabilities
+    taken relative to the first keys would overflow; the row must still match the
+    oracle (the kernel recomputes such a row with its true max)."""
+    w = synth.Workload("small", 91, 1, 32, 32, 64, 2, 2, 1, "bf16", region_bias=0.0, lce_b_std=0.05, lce_w_std=0.1)
+    inp = synth.make_inputs(w)
+    e = np.full(32, 30.0 / np.sqrt(32.0))
+    inp["q"][0, 5, 19, 0:32] = e          # query token 5*16+3 of region 1 (head 0)
+    inp["k"][0, 28, 24, 0:32] = e         # key 200 of region 3
+    inp = {k: synth.round_bf16(v) if k in ("q", "k", "v") else v for k, v in inp.items()}
+    d = to_dev(inp, w.dtype)
+    r_idx = np.array([[[2], [3], [0], [1]]], dtype=np.int32)
+    out = bra.attend(d["q"], d["k"], d["v"], d["lce_w"], d["lce_b"], w.heads, w.S, torch.from_numpy(r_idx).cuda())
+    ref = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], w.heads, w.S, r_idx)
+    rep = compare.Report()
+    got = out.float().cpu().numpy()
+    compare.check_output(got, ref, w.dtype, rep)
+    assert rep.ok, rep.notes
+    assert np.all(np.isfinite(got))
 
 
 def test_host_entry_point_matches_device_entry_point():

@@ -20,14 +20,14 @@ _lib = None
 BRA_F32, BRA_BF16 = 0, 1
 STATUS = {0: "BRA_OK", 1: "BRA_ERR_NULL", 2: "BRA_ERR_SHAPE", 3: "BRA_ERR_ALIGN", 4: "BRA_ERR_DTYPE",
           5: "BRA_ERR_CUDA", 6: "BRA_ERR_INDEX", 7: "BRA_ERR_SCRATCH", 8: "BRA_ERR_TIMEOUT"}
-VARIANT_AUTO, VARIANT_GENERIC, VARIANT_TMA, VARIANT_SPLIT = 0, 1, 2, 3
+VARIANT_AUTO, VARIANT_GENERIC, VARIANT_TMA, VARIANT_SPLIT, VARIANT_PIPE = 0, 1, 2, 3, 4
 STATIC_SCRATCH_FLOATS = 4 * 1024 * 1024
 # entry points declared in include/bra.h
 SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
            "bra_status_string",
            "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name",
            "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout", "bra_trace_read")
-KERNEL_CLASSES = 5
+KERNEL_CLASSES = 6
 
 
 class BraError(RuntimeError):

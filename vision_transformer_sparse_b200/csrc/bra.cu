@@ -29,6 +29,7 @@
 #include "attn.cuh"
 #include "attn_pipe.cuh"
 #include "attn_tma.cuh"
+#include "attn_umma.cuh"
 #include "fused_image.cuh"
 #include "route.cuh"
 
@@ -525,7 +526,8 @@ static int launch_attend_pipe(const Shape &s, const void *q, const void *k, cons
                               const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st,
                               bool *used) {
     *used = false;
-    if (g_variant.load() != BRA_VARIANT_AUTO && g_variant.load() != BRA_VARIANT_SPLIT) return BRA_OK;
+    const int var = g_variant.load();
+    if (var != BRA_VARIANT_AUTO && var != BRA_VARIANT_SPLIT && var != BRA_VARIANT_PIPE) return BRA_OK;
     if (!aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
     PipePlan pl;
     if (!plan_pipe(s, pl)) return BRA_OK;
@@ -567,10 +569,76 @@ static int launch_attend_pipe(const Shape &s, const void *q, const void *k, cons
     return launch_pdl(kern, dim3(ctas), dim3(pl.threads), pl.smem, st, pp) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
 }
 
+// ----------------------------------------------------------------------------- tcgen05 attention
+
+// The tcgen05 kernel takes bf16 heads of 32 channels, regions of 128 or 256 tokens
+// (hr a multiple of 8, wr even) and at most 256 keys per query.
+static bool umma_shape_ok(const Shape &s) {
+    return s.dtype == BRA_BF16 && s.d == 32 && s.w2 % 128 == 0 && s.topk * s.w2 <= 256 &&
+           s.hr % kUmmaRows == 0 && s.wr % 2 == 0 && 128 % s.wr == 0 && s.hr + 4 <= 256 && s.wr + 4 <= 256;
+}
+
+static int launch_attend_umma(const Shape &s, const void *q, const void *k, const void *v, const void *w,
+                              const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st,
+                              bool *used) {
+    *used = false;
+    const int var = g_variant.load();
+    if (var != BRA_VARIANT_AUTO && var != BRA_VARIANT_SPLIT) return BRA_OK;
+    if (!umma_shape_ok(s) || !aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
+    const UmmaSmem L = umma_smem_layout(s.topk, s.w2, s.hr, s.wr);
+    if (L.total > kMaxSmem) return BRA_OK;
+    UmmaParams p;
+    memset(&p, 0, sizeof(p));
+    if (!encode_map_box(&p.tmQ, q, s, 32, s.wr, s.hr, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_map_box(&p.tmK, k, s, 32, s.wr, s.hr, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_map_box(&p.tmV, v, s, 32, s.wr, s.hr, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_map_box(&p.tmH, v, s, 32, s.wr + 4, s.hr + 4, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_map_box(&p.tmO, out, s, 32, s.wr, 128 / s.wr, CU_TENSOR_MAP_SWIZZLE_64B))
+        return BRA_OK;
+    p.lce_w = static_cast<const __nv_bfloat16 *>(w);
+    p.lce_b = static_cast<const __nv_bfloat16 *>(b);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.r_idx = r_idx;
+    p.err_flag = err;
+    p.H = s.H;
+    p.W = s.W;
+    p.C = s.C;
+    p.heads = s.heads;
+    p.S = s.S;
+    p.topk = s.topk;
+    p.hr = s.hr;
+    p.wr = s.wr;
+    p.w2 = s.w2;
+    p.P = s.P;
+    p.regions = s.N * s.P;
+    p.scale_log2 = (float)(1.0 / std::sqrt((double)s.d) * 1.4426950408889634);
+    p.wait_limit = kWaitLimit;
+    p.div_P = FastDiv((uint32_t)s.P);
+    p.div_S = FastDiv((uint32_t)s.S);
+    p.div_wr = FastDiv((uint32_t)s.wr);
+    p.div_wx = FastDiv((uint32_t)(s.wr / 2));
+    auto kern = attn_umma_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    // one CTA per SM (the whole tensor memory); a CTA keeps one head
+    int ctas = std::min(sms, s.heads * p.regions);
+    ctas -= ctas % s.heads;
+    if (ctas < s.heads) ctas = s.heads;
+    *used = true;
+    LaunchScope ls(BRA_KERNEL_ATTN_UMMA, st);
+    return launch_pdl(kern, dim3(ctas), dim3(kUmmaThreads), L.total, st, p) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
 static int launch_attend(const Shape &s, const void *q, const void *k, const void *v, const void *w,
                          const void *b, void *out, const int32_t *r_idx, int *err, cudaStream_t st) {
     bool used = false;
-    int rc = launch_attend_pipe(s, q, k, v, w, b, out, r_idx, err, st, &used);
+    int rc = launch_attend_umma(s, q, k, v, w, b, out, r_idx, err, st, &used);
+    if (rc || used) return rc;
+    rc = launch_attend_pipe(s, q, k, v, w, b, out, r_idx, err, st, &used);
     if (rc || used) return rc;
     rc = launch_attend_tma(s, q, k, v, w, b, out, r_idx, err, st, &used);
     if (rc || used) return rc;
@@ -671,7 +739,7 @@ extern "C" {
 int bra_version(void) { return (1 << 16) | 1; }
 
 int bra_set_kernel_variant(int variant) {
-    if (variant < BRA_VARIANT_AUTO || variant > BRA_VARIANT_SPLIT) return -1;
+    if (variant < BRA_VARIANT_AUTO || variant > BRA_VARIANT_PIPE) return -1;
     return g_variant.exchange(variant);
 }
 
@@ -751,6 +819,7 @@ const char *bra_kernel_name(int kernel_class) {
         case BRA_KERNEL_ATTN_BF16: return "attn_bf16_kernel";
         case BRA_KERNEL_ATTN_F32: return "attn_f32_kernel";
         case BRA_KERNEL_FUSED_IMAGE: return "bra_image_kernel";
+        case BRA_KERNEL_ATTN_UMMA: return "attn_umma_kernel";
         default: return "unknown";
     }
 }
