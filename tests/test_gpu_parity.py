@@ -94,6 +94,8 @@ SMALL = [
     (2, 16, 32, 64, 2, 2, 2, "bf16"),     # 8x16 regions, topk 2 -> 256 keys: tcgen05
     (1, 16, 32, 128, 4, 2, 1, "bf16"),    # 8x16 regions, 128 keys, 4 heads: tcgen05
     (3, 48, 48, 96, 3, 3, 1, "bf16"),     # 16x16 regions, 3 heads, 3 images: tcgen05
+    (1, 32, 32, 64, 2, 16, 20, "bf16"),   # 256 regions (column-per-lane routing), topk 20 (sort)
+    (6, 16, 16, 64, 2, 16, 2, "bf16"),    # 256 regions, 6 images (8 routing rows per CTA)
 ]
 
 

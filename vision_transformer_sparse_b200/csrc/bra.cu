@@ -200,7 +200,9 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
         return BRA_ERR_CUDA;
     int rpw = 4;
     while (rpw > 1 && (long long)s.N * ((s.P + kRouteWarps * rpw - 1) / (kRouteWarps * rpw)) < sms) rpw >>= 1;
-    const int rows = kRouteWarps * rpw;
+    // more than 128 regions: the column-per-lane kernel with 4 or 8 rows per CTA
+    const int cols_rows = (long long)s.N * ((s.P + 7) / 8) >= sms ? 8 : 4;
+    const int rows = E == 8 ? cols_rows : kRouteWarps * rpw;
     int cc = route_chunk(32 * E, rows, s.C);
     while (s.C % cc) cc -= 32;  // equal passes: one divisor for the staging index
     const int smem = route_smem_bytes(32 * E, rows, cc);
@@ -236,8 +238,10 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
         by_rpw(std::integral_constant<int, 2>{});
     else if (E == 4)
         by_rpw(std::integral_constant<int, 4>{});
+    else if (cols_rows == 8)
+        go(route_cols_kernel<8>);
     else
-        by_rpw(std::integral_constant<int, 8>{});
+        go(route_cols_kernel<4>);
     return rc;
 }
 

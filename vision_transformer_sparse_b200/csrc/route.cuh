@@ -86,10 +86,11 @@ region_mean_kernel(const T *__restrict__ q, const T *__restrict__ k, float *__re
 }
 
 // Large regions (w2 >= 64): one CTA per (image, region). Thread = (16-byte channel
-// group g, token slot s) over q and k; slots stride the region's tokens with eight
-// independent loads in flight; partial sums meet in shared memory.
+// group g, token slot s) over q and k; slots stride the region's tokens with four
+// independent loads of each tensor in flight (few registers, so four CTAs share an
+// SM); partial sums meet in shared memory.
 template <typename T>
-__global__ void __launch_bounds__(kPoolThreads)
+__global__ void __launch_bounds__(kPoolThreads, 4)
 region_mean_big_kernel(const T *__restrict__ q, const T *__restrict__ k, float *__restrict__ q_r,
                        float *__restrict__ k_r, int H, int W, int C, int S) {
     constexpr int V = Elem<T>::kVec;
@@ -105,10 +106,10 @@ region_mean_big_kernel(const T *__restrict__ q, const T *__restrict__ k, float *
 #pragma unroll
     for (int e = 0; e < V; ++e) aq[e] = ak[e] = 0.f;
     if (sl < slots) {
-        for (int t0 = sl; t0 < w2; t0 += 8 * slots) {
-            uint4 bq[8], bk[8];
+        for (int t0 = sl; t0 < w2; t0 += 4 * slots) {
+            uint4 bq[4], bk[4];
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
+            for (int b = 0; b < 4; ++b) {
                 const int t = t0 + b * slots;
                 bq[b] = bk[b] = make_uint4(0u, 0u, 0u, 0u);
                 if (t < w2) {
@@ -119,7 +120,7 @@ region_mean_big_kernel(const T *__restrict__ q, const T *__restrict__ k, float *
                 }
             }
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
+            for (int b = 0; b < 4; ++b) {
                 float f[V];
                 unpack16(bq[b], f, q);
 #pragma unroll
@@ -165,6 +166,123 @@ inline int route_smem_bytes(int PP, int rows, int cc) {
     const int dots = rows * PP;  // reuses the k_r tile when it fits
     const int tile = PP * (cc + 4) + rows * cc;
     return (tile > dots ? tile : dots) * 4;
+}
+
+// Top-k selection and softmax of one affinity row (dots: the row's PP = 32E logits in
+// shared memory), run by one warp; writes topk (index, weight) pairs at out_idx /
+// out_w. topk <= 8 by repeated warp argmax, larger topk by a bitonic sort of all 32E
+// (value, index) pairs. Order: larger logit first, equal logits -> lower index first.
+template <int E>
+__device__ __forceinline__ void route_select_row(const float *dots, int P, int topk, int lane, int32_t *out_idx,
+                                                 float *out_w) {
+    constexpr int PP = 32 * E;
+    float val[E];
+    int id[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int col = lane + 32 * e;
+        val[e] = col < P ? dots[col] : -INFINITY;
+        id[e] = col;  // padding columns carry unique indices >= P and lose every comparison
+    }
+    if (topk <= 8) {
+        // topk rounds of warp argmax; lane `round` keeps that round's winner
+        unsigned taken = 0;
+        float my_v = 0.f;
+        int my_i = 0;
+        float v0 = 0.f;
+        for (int round = 0; round < topk; ++round) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                if (!(taken & (1u << e)) && (id[e] < P) && route_before(val[e], id[e], bv, bi)) {
+                    bv = val[e];
+                    bi = id[e];
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (route_before(ov, oi, bv, bi)) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (lane == round) {
+                my_v = bv;
+                my_i = bi;
+            }
+            if (round == 0) v0 = bv;
+        }
+        const float ex = lane < topk ? expf(my_v - v0) : 0.f;
+        float z = ex;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        if (lane < topk) {
+            out_idx[lane] = my_i;
+            out_w[lane] = ex / z;
+        }
+        return;
+    }
+
+    // Bitonic sort of the PP pairs into route_before order; element index = e*32 + lane.
+#pragma unroll
+    for (int kk = 2; kk <= PP; kk <<= 1) {
+#pragma unroll
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            if (jj >= 32) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int e2 = e ^ (jj >> 5);
+                    if (e2 > e) {
+                        const bool up = ((e * 32 + lane) & kk) == 0;
+                        const bool sw = up ? route_before(val[e2], id[e2], val[e], id[e])
+                                           : route_before(val[e], id[e], val[e2], id[e2]);
+                        if (sw) {
+                            const float tv = val[e];
+                            val[e] = val[e2];
+                            val[e2] = tv;
+                            const int ti = id[e];
+                            id[e] = id[e2];
+                            id[e2] = ti;
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const float pv = __shfl_xor_sync(0xffffffffu, val[e], jj);
+                    const int pi = __shfl_xor_sync(0xffffffffu, id[e], jj);
+                    const bool up = ((e * 32 + lane) & kk) == 0;
+                    const bool lower = (lane & jj) == 0;
+                    const bool mine_first = route_before(val[e], id[e], pv, pi);
+                    const bool keep = (up == lower) ? mine_first : !mine_first;
+                    if (!keep) {
+                        val[e] = pv;
+                        id[e] = pi;
+                    }
+                }
+            }
+        }
+    }
+    // softmax over the first topk sorted logits; position 0 holds the maximum
+    const float vmax = __shfl_sync(0xffffffffu, val[0], 0);
+    float z = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (e * 32 + lane < topk) z += expf(val[e] - vmax);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    const float inv_z = 1.0f / z;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int pos = e * 32 + lane;
+        if (pos < topk) {
+            out_idx[pos] = id[e];
+            out_w[pos] = expf(val[e] - vmax) * inv_z;
+        }
+    }
 }
 
 // One CTA per (image n, block of 8*RPW affinity rows). Each warp owns RPW rows and each
@@ -267,114 +385,95 @@ route_kernel(const float *__restrict__ q_r, const float *__restrict__ k_r, int C
     for (int r = 0; r < RPW; ++r) {
         const int row = warp * RPW + r, p = p0 + row;
         if (p >= P) break;
-        float val[E];
-        int id[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int col = lane + 32 * e;
-            val[e] = col < P ? dots[row * PP + col] : -INFINITY;
-            id[e] = col;  // padding columns carry unique indices >= P and lose every comparison
-        }
         const size_t base = ((size_t)n * P + p) * topk;
-        if (topk <= 8) {
-            // topk rounds of warp argmax; lane `round` keeps that round's winner
-            unsigned taken = 0;
-            float my_v = 0.f;
-            int my_i = 0;
-            float v0 = 0.f;
-            for (int round = 0; round < topk; ++round) {
-                float bv = -INFINITY;
-                int bi = 0x7fffffff;
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    if (!(taken & (1u << e)) && (id[e] < P) && route_before(val[e], id[e], bv, bi)) {
-                        bv = val[e];
-                        bi = id[e];
-                    }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                    if (route_before(ov, oi, bv, bi)) {
-                        bv = ov;
-                        bi = oi;
-                    }
-                }
-                if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-                if (lane == round) {
-                    my_v = bv;
-                    my_i = bi;
-                }
-                if (round == 0) v0 = bv;
-            }
-            const float ex = lane < topk ? expf(my_v - v0) : 0.f;
-            float z = ex;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-            if (lane < topk) {
-                r_idx[base + lane] = my_i;
-                r_weight[base + lane] = ex / z;
-            }
-            continue;
-        }
+        route_select_row<E>(dots + row * PP, P, topk, lane, r_idx + base, r_weight + base);
+    }
+}
 
-        // Bitonic sort of the PP pairs into route_before order; element index = e*32 + lane.
+// Many regions (32E = 256 columns): one CTA per (image n, block of ROWS affinity rows),
+// eight warps; warp w owns the 32 columns 32w + lane for all ROWS rows, so every key
+// float4 read from shared memory feeds 4*ROWS FMAs (the query float4s are broadcast).
+// Staging, layout and the selection are those of route_kernel.
+template <int ROWS>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+route_cols_kernel(const float *__restrict__ q_r, const float *__restrict__ k_r, int C, int P, int topk, int cc,
+                  float scale, int32_t *__restrict__ r_idx, float *__restrict__ r_weight, FastDiv div_q4) {
+    extern __shared__ __align__(16) float route_s[];
+    constexpr int E = 8, PP = 32 * E;
+    griddep_wait();               // pooled means come from the preceding kernel
+    griddep_launch_dependents();  // the attention kernel may start its prologue
+    const int n = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int p0 = blockIdx.x * ROWS;
+    const float *kimg = k_r + (size_t)n * P * C;
+    const float *qimg = q_r + (size_t)n * P * C;
+    const int kp = cc + 4;
+    float *kr_s = route_s;           // [PP][kp]
+    float *q_s = route_s + PP * kp;  // [ROWS][cc]
+    const int col = warp * 32 + lane;
+
+    float dot[ROWS];
 #pragma unroll
-        for (int kk = 2; kk <= PP; kk <<= 1) {
+    for (int r = 0; r < ROWS; ++r) dot[r] = 0.f;
+
+    for (int c0 = 0; c0 < C; c0 += cc) {
+        const int cw = min(cc, C - c0), q4 = cw >> 2;
+        __syncthreads();
+        for (int i0 = threadIdx.x; i0 < (PP + ROWS) * q4; i0 += 8 * blockDim.x) {
+            float4 buf[8];
+            int rr[8], cc4[8];
 #pragma unroll
-            for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-                if (jj >= 32) {
+            for (int b = 0; b < 8; ++b) {
+                const int idx = i0 + b * blockDim.x;
+                uint32_t cm;
+                rr[b] = (int)div_q4.divmod((uint32_t)idx, cm);
+                cc4[b] = (int)cm * 4;
+                buf[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (rr[b] < P) {
+                    buf[b] = __ldg(reinterpret_cast<const float4 *>(kimg + (size_t)rr[b] * C + c0 + cc4[b]));
+                } else if (rr[b] >= PP && rr[b] < PP + ROWS) {
+                    buf[b] = __ldg(reinterpret_cast<const float4 *>(qimg + (size_t)min(p0 + rr[b] - PP, P - 1) * C + c0 +
+                                                                   cc4[b]));
+                }
+            }
 #pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        const int e2 = e ^ (jj >> 5);
-                        if (e2 > e) {
-                            const bool up = ((e * 32 + lane) & kk) == 0;
-                            const bool sw = up ? route_before(val[e2], id[e2], val[e], id[e])
-                                               : route_before(val[e], id[e], val[e2], id[e2]);
-                            if (sw) {
-                                const float tv = val[e];
-                                val[e] = val[e2];
-                                val[e2] = tv;
-                                const int ti = id[e];
-                                id[e] = id[e2];
-                                id[e2] = ti;
-                            }
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        const float pv = __shfl_xor_sync(0xffffffffu, val[e], jj);
-                        const int pi = __shfl_xor_sync(0xffffffffu, id[e], jj);
-                        const bool up = ((e * 32 + lane) & kk) == 0;
-                        const bool lower = (lane & jj) == 0;
-                        const bool mine_first = route_before(val[e], id[e], pv, pi);
-                        const bool keep = (up == lower) ? mine_first : !mine_first;
-                        if (!keep) {
-                            val[e] = pv;
-                            id[e] = pi;
-                        }
-                    }
+            for (int b = 0; b < 8; ++b) {
+                if (rr[b] < PP) {
+                    *reinterpret_cast<float4 *>(kr_s + rr[b] * kp + cc4[b]) = buf[b];
+                } else if (rr[b] < PP + ROWS) {
+                    float4 v = buf[b];
+                    v.x *= scale;  // the walk-through scales the region query before the product
+                    v.y *= scale;
+                    v.z *= scale;
+                    v.w *= scale;
+                    *reinterpret_cast<float4 *>(q_s + (rr[b] - PP) * cc + cc4[b]) = v;
                 }
             }
         }
-        // softmax over the first topk sorted logits; position 0 holds the maximum
-        const float vmax = __shfl_sync(0xffffffffu, val[0], 0);
-        float z = 0.f;
+        __syncthreads();
+        for (int c = 0; c < cw; c += 4) {
+            const float4 kv = *reinterpret_cast<const float4 *>(kr_s + col * kp + c);
 #pragma unroll
-        for (int e = 0; e < E; ++e)
-            if (e * 32 + lane < topk) z += expf(val[e] - vmax);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-        const float inv_z = 1.0f / z;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int pos = e * 32 + lane;
-            if (pos < topk) {
-                r_idx[base + pos] = id[e];
-                r_weight[base + pos] = expf(val[e] - vmax) * inv_z;
+            for (int r = 0; r < ROWS; ++r) {
+                const float4 qv = *reinterpret_cast<const float4 *>(q_s + r * cc + c);
+                dot[r] = fmaf(qv.x, kv.x, dot[r]);
+                dot[r] = fmaf(qv.y, kv.y, dot[r]);
+                dot[r] = fmaf(qv.z, kv.z, dot[r]);
+                dot[r] = fmaf(qv.w, kv.w, dot[r]);
             }
         }
+    }
+
+    __syncthreads();
+    float *dots = route_s;  // [ROWS][PP]
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) dots[r * PP + col] = dot[r];
+    __syncthreads();
+    for (int row = warp; row < ROWS; row += kRouteWarps) {
+        const int p = p0 + row;
+        if (p >= P) break;
+        const size_t base = ((size_t)n * P + p) * topk;
+        route_select_row<E>(dots + row * PP, P, topk, lane, r_idx + base, r_weight + base);
     }
 }
 
