@@ -105,8 +105,11 @@ int bra_attend(const void *q, const void *k, const void *v, const void *lce_w, c
  * device (pinned host memory gives asynchronous copies), runs the forward on
  * `stream`, copies out, r_idx and r_weight back to the host buffers and
  * synchronises `stream` before returning. Device buffers are taken from and
- * returned to the device's default memory pool, stream-ordered. Same shapes,
- * dtypes and error codes as bra_forward; host pointers need no alignment. */
+ * returned to a stream-ordered memory pool that the library creates once per
+ * device and that keeps its memory between calls (so repeated calls do not map
+ * device memory again); that memory stays reserved until the process exits.
+ * Same shapes, dtypes and error codes as bra_forward; host pointers need no
+ * alignment. */
 int bra_forward_host(const void *q, const void *k, const void *v, const void *lce_w,
                      const void *lce_b, int N, int H, int W, int C, int heads, int S, int topk,
                      int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream);

@@ -18,7 +18,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <type_traits>
 #include <utility>
 #include <vector>
@@ -148,6 +150,108 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// ----------------------------------------------------------------------------- launch facts
+// Attribute and occupancy queries cost far more than a launch (a cluster-occupancy query
+// takes milliseconds), and their answers depend only on (device, kernel, block, shared
+// memory): each is made once per key and kept.
+
+static std::mutex g_facts_mu;
+static std::map<int, int> g_sms;                                          // device -> SMs
+static std::map<std::pair<int, const void *>, int> g_smem_set;            // (device, kernel) -> bytes allowed
+static std::map<std::tuple<int, const void *, int, int, int>, int> g_occ;  // (device, kernel, threads, smem, cluster)
+
+static int sm_count(int *sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BRA_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_facts_mu);
+    auto it = g_sms.find(dev);
+    if (it == g_sms.end()) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BRA_ERR_CUDA;
+        it = g_sms.emplace(dev, n).first;
+    }
+    *sms = it->second;
+    return BRA_OK;
+}
+
+// Allow `bytes` of dynamic shared memory for `kern` on the current device.
+template <typename K> static cudaError_t allow_smem(K kern, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_pair(dev, reinterpret_cast<const void *>(kern));
+    std::lock_guard<std::mutex> g(g_facts_mu);
+    auto it = g_smem_set.find(key);
+    if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) g_smem_set[key] = bytes;
+    return e;
+}
+
+// Resident CTAs per SM (cluster = 0) or resident clusters on the device (cluster > 0,
+// for the launch configuration cfg).
+template <typename K>
+static cudaError_t occupancy(int *out, K kern, int threads, int smem, int cluster, const cudaLaunchConfig_t *cfg) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_tuple(dev, reinterpret_cast<const void *>(kern), threads, smem, cluster);
+    {
+        std::lock_guard<std::mutex> g(g_facts_mu);
+        auto it = g_occ.find(key);
+        if (it != g_occ.end()) {
+            *out = it->second;
+            return cudaSuccess;
+        }
+    }
+    int v = 0;
+    e = cluster > 0 ? cudaOccupancyMaxActiveClusters(&v, kern, cfg)
+                    : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> g(g_facts_mu);
+    g_occ[key] = v;
+    *out = v;
+    return cudaSuccess;
+}
+
+// Device buffers of bra_forward_host come from a library-owned stream-ordered pool per
+// device whose memory is kept between calls (release threshold = unlimited): the
+// default pool returns its memory at every synchronisation, and mapping tens of MB
+// again on the next call costs milliseconds.
+struct HostCallRes {
+    cudaMemPool_t pool;
+    cudaStream_t up, back;  // non-blocking streams for the host-to-device and device-to-host copies
+};
+static std::map<int, HostCallRes> g_host_pools;
+
+// The pool and the two copy streams, per device.
+static int host_call_pool(cudaMemPool_t *pool, cudaStream_t *up, cudaStream_t *back) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BRA_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_facts_mu);
+    auto it = g_host_pools.find(dev);
+    if (it == g_host_pools.end()) {
+        cudaMemPoolProps props;
+        memset(&props, 0, sizeof(props));
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p = nullptr;
+        if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return BRA_ERR_CUDA;
+        uint64_t keep = UINT64_MAX;
+        if (cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) return BRA_ERR_CUDA;
+        cudaStream_t u = nullptr, b = nullptr;
+        if (cudaStreamCreateWithFlags(&u, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking) != cudaSuccess)
+            return BRA_ERR_CUDA;
+        it = g_host_pools.emplace(dev, HostCallRes{p, u, b}).first;
+    }
+    *pool = it->second.pool;
+    *up = it->second.up;
+    *back = it->second.back;
+    return BRA_OK;
+}
+
 // Token slots per (region, channel group) for the region-mean kernel: ns divides wr,
 // G*ns divides 32, and each thread keeps at least 4 tokens.
 static int pool_ns_log2(const Shape &s) {
@@ -195,9 +299,8 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
     const float scale = 1.0f / sqrtf((float)s.d);
     const int E = s.P <= 32 ? 1 : s.P <= 64 ? 2 : s.P <= 128 ? 4 : 8;
     // rows per CTA: as many as still leave about one CTA per SM
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return BRA_ERR_CUDA;
+    int sms = 148;
+    if (sm_count(&sms) != BRA_OK) return BRA_ERR_CUDA;
     int rpw = 4;
     while (rpw > 1 && (long long)s.N * ((s.P + kRouteWarps * rpw - 1) / (kRouteWarps * rpw)) < sms) rpw >>= 1;
     // more than 128 regions: the column-per-lane kernel with 4 or 8 rows per CTA
@@ -209,7 +312,7 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
     const FastDiv div_q4((uint32_t)(cc / 4));
     int rc = BRA_OK;
     auto go = [&](auto kern) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+        if (allow_smem(kern, smem) != cudaSuccess) {
             rc = BRA_ERR_CUDA;
             return;
         }
@@ -327,8 +430,7 @@ static bool plan_f32(const Shape &s, AttnParams &p, int &threads, int &smem) {
 template <typename K>
 static int launch_kernel(K kern, int kid, int blocks, int threads, int smem, cudaStream_t st,
                          const AttnParams &p) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return BRA_ERR_CUDA;
+    if (allow_smem(kern, smem) != cudaSuccess) return BRA_ERR_CUDA;
     LaunchScope ls(kid, st);
     kern<<<blocks, threads, smem, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
@@ -433,8 +535,7 @@ static int launch_attend_tma(const Shape &s, const void *q, const void *k, const
     p.wait_limit = kWaitLimit;
     const int blocks = s.N * s.P * p.n_rb * p.n_hg;
     auto kern = s.d == 32 ? attn_tma_kernel<32> : attn_tma_kernel<64>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return BRA_ERR_CUDA;
+    if (allow_smem(kern, smem) != cudaSuccess) return BRA_ERR_CUDA;
     *used = true;
     LaunchScope ls(BRA_KERNEL_ATTN_BF16, st);
     return launch_pdl(kern, dim3(blocks), dim3(threads), smem, st, p) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
@@ -557,12 +658,9 @@ static int launch_attend_pipe(const Shape &s, const void *q, const void *k, cons
     pp.div_wx = FastDiv((uint32_t)(s.wr / pp.XT));
     auto kern = pl.threads <= 160 ? (s.d == 32 ? attn_pipe_kernel<32, 160, 4> : attn_pipe_kernel<64, 160, 4>)
                                   : (s.d == 32 ? attn_pipe_kernel<32, 512, 1> : attn_pipe_kernel<64, 512, 1>);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
-        return BRA_ERR_CUDA;
-    int dev = 0, sms = 0, occ = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, pl.threads, pl.smem) != cudaSuccess)
+    if (allow_smem(kern, pl.smem) != cudaSuccess) return BRA_ERR_CUDA;
+    int sms = 0, occ = 0;
+    if (sm_count(&sms) != BRA_OK || occupancy(&occ, kern, pl.threads, pl.smem, 0, nullptr) != cudaSuccess)
         return BRA_ERR_CUDA;
     if (occ < 1) return BRA_OK;
     int ctas = std::min(pp.units, sms * occ);
@@ -622,12 +720,9 @@ static int launch_attend_umma(const Shape &s, const void *q, const void *k, cons
     p.div_wr = FastDiv((uint32_t)s.wr);
     p.div_wx = FastDiv((uint32_t)(s.wr / 2));
     auto kern = attn_umma_kernel;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total) != cudaSuccess)
-        return BRA_ERR_CUDA;
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return BRA_ERR_CUDA;
+    if (allow_smem(kern, L.total) != cudaSuccess) return BRA_ERR_CUDA;
+    int sms = 0;
+    if (sm_count(&sms) != BRA_OK) return BRA_ERR_CUDA;
     // one CTA per SM (the whole tensor memory); a CTA keeps one head
     int ctas = std::min(sms, s.heads * p.regions);
     ctas -= ctas % s.heads;
@@ -700,8 +795,7 @@ static int launch_fused_image(const Shape &s, const void *q, const void *k, cons
     p.div_S = FastDiv((uint32_t)s.S);
     p.div_W = FastDiv((uint32_t)s.W);
     auto kern = s.hr == 4 ? bra_image_kernel<4, 4> : bra_image_kernel<2, 2>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total) != cudaSuccess)
-        return BRA_ERR_CUDA;
+    if (allow_smem(kern, L.total) != cudaSuccess) return BRA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(s.N * s.heads);
     cfg.blockDim = dim3(kImageWarps * 32);
@@ -715,7 +809,7 @@ static int launch_fused_image(const Shape &s, const void *q, const void *k, cons
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+    if (occupancy(&clusters, kern, kImageWarps * 32, L.total, s.heads, &cfg) != cudaSuccess || clusters < 1) {
         cudaGetLastError();  // not schedulable here: the three-kernel path runs instead
         return BRA_OK;
     }
@@ -863,18 +957,21 @@ int bra_route(const void *q, const void *k, int N, int H, int W, int C, int head
 // The forward with its scratch taken from (and returned to) the stream-ordered pool;
 // the scratch is released after the attention launch so that nothing separates the
 // route and attention kernels on the stream.
+// ws_given: scratch of 2*N*S*S*C floats owned by the caller, or NULL to take it from the
+// stream-ordered default pool for the duration of the call.
 static int forward_device(const Shape &s, const void *q, const void *k, const void *v, const void *lce_w,
-                          const void *lce_b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st) {
+                          const void *lce_b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st,
+                          float *ws_given = nullptr) {
     bool fused = false;
     int frc = launch_fused_image(s, q, k, v, lce_w, lce_b, out, r_idx, r_weight, st, &fused);
     if (frc || fused) return frc;
-    float *ws = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * (size_t)s.N * s.P * s.C * sizeof(float), st) !=
-        cudaSuccess)
+    float *ws = ws_given;
+    if (!ws && cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * (size_t)s.N * s.P * s.C * sizeof(float), st) !=
+                   cudaSuccess)
         return BRA_ERR_CUDA;
     int rc = launch_route_into(s, q, k, r_idx, r_weight, ws, st);
     if (rc == BRA_OK) rc = launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, nullptr, st);
-    if (cudaFreeAsync(ws, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    if (!ws_given && cudaFreeAsync(ws, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     return rc;
 }
 
@@ -931,32 +1028,71 @@ int bra_forward_host(const void *q, const void *k, const void *v, const void *lc
     if (!q || !k || !v || !lce_w || !lce_b || !out || !r_idx || !r_weight) return BRA_ERR_NULL;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t es = dtype == BRA_BF16 ? 2 : 4;
-    const size_t map = (size_t)N * H * W * C * es, wb = (size_t)C * 25 * es, bb = (size_t)C * es;
-    const size_t route = (size_t)N * s.P * topk * 4;
+    const size_t img = (size_t)H * W * C * es, map = (size_t)N * img, wb = (size_t)C * 25 * es, bb = (size_t)C * es;
+    const size_t rimg = (size_t)s.P * topk * 4, route = (size_t)N * rimg;
+    const size_t scratch = 2 * (size_t)N * s.P * C * sizeof(float);
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    const size_t total = 4 * up(map) + up(wb) + up(bb) + 2 * up(route);
+    const size_t total = 4 * up(map) + up(wb) + up(bb) + 2 * up(route) + up(scratch);
+    cudaMemPool_t pool = nullptr;
+    cudaStream_t up_st = nullptr, back = nullptr;
+    if (host_call_pool(&pool, &up_st, &back) != BRA_OK) return BRA_ERR_CUDA;
     char *base = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&base), total, st) != cudaSuccess) return BRA_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&base), total, pool, st) != cudaSuccess) return BRA_ERR_CUDA;
     char *dq = base, *dk = dq + up(map), *dv = dk + up(map), *dout = dv + up(map), *dw = dout + up(map);
     char *db = dw + up(wb), *di = db + up(bb), *dr = di + up(route);
+    float *dws = reinterpret_cast<float *>(dr + up(route));
+    // Images are independent: the batch goes in chunks over three streams. The inputs
+    // stream in back to back on one copy stream, chunk c is computed on `stream` once its
+    // inputs are in, and its results go back on a second copy stream while later chunks
+    // are still coming in.
+    const int nchunk = N < 8 ? N : 8, per = (N + nchunk - 1) / nchunk;
+    std::vector<cudaEvent_t> ev;
+    auto event = [&](cudaEvent_t *e) {
+        if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+        ev.push_back(*e);
+        return true;
+    };
     rc = BRA_OK;
-    const struct {
-        void *dst;
-        const void *src;
-        size_t n;
-    } h2d[] = {{dq, q, map}, {dk, k, map}, {dv, v, map}, {dw, lce_w, wb}, {db, lce_b, bb}};
-    for (const auto &c : h2d)
-        if (rc == BRA_OK && cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, st) != cudaSuccess)
-            rc = BRA_ERR_CUDA;
-    if (rc == BRA_OK)
-        rc = forward_device(s, dq, dk, dv, dw, db, dout, reinterpret_cast<int32_t *>(di),
-                            reinterpret_cast<float *>(dr), st);
-    if (rc == BRA_OK && cudaMemcpyAsync(out, dout, map, cudaMemcpyDeviceToHost, st) != cudaSuccess) rc = BRA_ERR_CUDA;
-    if (rc == BRA_OK && cudaMemcpyAsync(r_idx, di, route, cudaMemcpyDeviceToHost, st) != cudaSuccess) rc = BRA_ERR_CUDA;
-    if (rc == BRA_OK && cudaMemcpyAsync(r_weight, dr, route, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    cudaEvent_t e_alloc = nullptr;
+    if (!event(&e_alloc) || cudaEventRecord(e_alloc, st) != cudaSuccess ||
+        cudaStreamWaitEvent(up_st, e_alloc, 0) != cudaSuccess ||
+        cudaMemcpyAsync(dw, lce_w, wb, cudaMemcpyHostToDevice, up_st) != cudaSuccess ||
+        cudaMemcpyAsync(db, lce_b, bb, cudaMemcpyHostToDevice, up_st) != cudaSuccess)
         rc = BRA_ERR_CUDA;
+    for (int n0 = 0; n0 < N && rc == BRA_OK; n0 += per) {
+        const int nb = N - n0 < per ? N - n0 : per;
+        const size_t o = (size_t)n0 * img, ob = (size_t)nb * img, ro = (size_t)n0 * rimg, rb = (size_t)nb * rimg;
+        cudaEvent_t e_in = nullptr, e_out = nullptr;
+        if (!event(&e_in) || !event(&e_out) ||
+            cudaMemcpyAsync(dq + o, static_cast<const char *>(q) + o, ob, cudaMemcpyHostToDevice, up_st) != cudaSuccess ||
+            cudaMemcpyAsync(dk + o, static_cast<const char *>(k) + o, ob, cudaMemcpyHostToDevice, up_st) != cudaSuccess ||
+            cudaMemcpyAsync(dv + o, static_cast<const char *>(v) + o, ob, cudaMemcpyHostToDevice, up_st) != cudaSuccess ||
+            cudaEventRecord(e_in, up_st) != cudaSuccess || cudaStreamWaitEvent(st, e_in, 0) != cudaSuccess) {
+            rc = BRA_ERR_CUDA;
+            break;
+        }
+        Shape sc = s;
+        sc.N = nb;
+        rc = forward_device(sc, dq + o, dk + o, dv + o, dw, db, dout + o, reinterpret_cast<int32_t *>(di + ro),
+                            reinterpret_cast<float *>(dr + ro), st, dws + (size_t)n0 * 2 * s.P * C);
+        if (rc != BRA_OK) break;
+        if (cudaEventRecord(e_out, st) != cudaSuccess || cudaStreamWaitEvent(back, e_out, 0) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<char *>(out) + o, dout + o, ob, cudaMemcpyDeviceToHost, back) != cudaSuccess ||
+            cudaMemcpyAsync(reinterpret_cast<char *>(r_idx) + ro, di + ro, rb, cudaMemcpyDeviceToHost, back) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(reinterpret_cast<char *>(r_weight) + ro, dr + ro, rb, cudaMemcpyDeviceToHost, back) !=
+                cudaSuccess)
+            rc = BRA_ERR_CUDA;
+    }
+    // `stream` takes over both copy streams, then releases the buffers
+    cudaEvent_t e_up = nullptr, e_back = nullptr;
+    if (!event(&e_up) || !event(&e_back) || cudaEventRecord(e_up, up_st) != cudaSuccess ||
+        cudaEventRecord(e_back, back) != cudaSuccess || cudaStreamWaitEvent(st, e_up, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(st, e_back, 0) != cudaSuccess)
+        rc = rc == BRA_OK ? BRA_ERR_CUDA : rc;
     if (cudaFreeAsync(base, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
     return rc;
 }
 
