@@ -189,7 +189,7 @@ const char *bra_kernel_name(int kernel_class);
  * By default (BRA_VARIANT_AUTO) a bfloat16 forward whose images are small runs as
  * ONE kernel (pooling, routing, attention and LCE fused; one thread-block cluster of
  * `heads` CTAs per image): this needs d = 32, regions of 4x4 or 2x2 tokens, S*S <= 64,
- * topk <= 32, heads <= 8 and one head's Q, K and V slices of a whole image within one
+ * topk <= 64, heads <= 8 and one head's Q, K and V slices of a whole image within one
  * CTA's shared memory. Otherwise the forward runs as three kernels (region means,
  * routing, attention). The bfloat16 attention then runs, in this order of preference:
  *  - on the 5th-generation tensor cores (tcgen05: scores and probabilities in tensor

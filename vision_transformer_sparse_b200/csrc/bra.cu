@@ -765,10 +765,14 @@ static int launch_fused_image(const Shape &s, const void *q, const void *k, cons
                               bool *used) {
     *used = false;
     if (g_variant.load() != BRA_VARIANT_AUTO) return BRA_OK;
-    if (s.dtype != BRA_BF16 || s.d != 32 || s.P > 64 || s.topk > 32 || s.heads > 8) return BRA_OK;
+    if (s.dtype != BRA_BF16 || s.d != 32 || s.P > 64 || s.topk > 64 || s.heads > 8) return BRA_OK;
     if (!((s.hr == 4 && s.wr == 4) || (s.hr == 2 && s.wr == 2))) return BRA_OK;
     if (s.H + 4 > 256 || s.W + 4 > 256 || !aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
-    const ImageSmem L = image_smem_layout(s.H, s.W, s.P, s.topk, s.w2, kImageWarps);
+    // 16 warps when one CTA fills an SM's shared memory; 8 when two fit (the kernel's
+    // 128 registers per thread then allow two CTAs per SM)
+    int nwarps = kImageWarps;
+    if (image_smem_layout(s.H, s.W, s.P, s.topk, s.w2, kImageWarps / 2).total <= kMaxSmem / 2) nwarps = kImageWarps / 2;
+    const ImageSmem L = image_smem_layout(s.H, s.W, s.P, s.topk, s.w2, nwarps);
     if (L.total > kMaxSmem) return BRA_OK;
     ImageParams p;
     memset(&p, 0, sizeof(p));
@@ -798,7 +802,7 @@ static int launch_fused_image(const Shape &s, const void *q, const void *k, cons
     if (allow_smem(kern, L.total) != cudaSuccess) return BRA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(s.N * s.heads);
-    cfg.blockDim = dim3(kImageWarps * 32);
+    cfg.blockDim = dim3(nwarps * 32);
     cfg.dynamicSmemBytes = L.total;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
@@ -809,7 +813,7 @@ static int launch_fused_image(const Shape &s, const void *q, const void *k, cons
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int clusters = 0;
-    if (occupancy(&clusters, kern, kImageWarps * 32, L.total, s.heads, &cfg) != cudaSuccess || clusters < 1) {
+    if (occupancy(&clusters, kern, nwarps * 32, L.total, s.heads, &cfg) != cudaSuccess || clusters < 1) {
         cudaGetLastError();  // not schedulable here: the three-kernel path runs instead
         return BRA_OK;
     }

@@ -263,10 +263,11 @@ __global__ void __launch_bounds__(512, 1) bra_image_kernel(const __grid_constant
                 val[e] = col < P ? s : -INFINITY;
             }
         }
-        // topk rounds of warp argmax (larger logit first, ties to the lower region index)
+        // topk rounds of warp argmax (larger logit first, ties to the lower region index);
+        // round r's winner is kept by lane r % 32 in slot r / 32 (topk <= 64)
         unsigned taken = 0;
-        float my_v = 0.f, v0 = 0.f;
-        int my_i = 0;
+        float my_v[2] = {0.f, 0.f}, v0 = 0.f;
+        int my_i[2] = {0, 0};
         for (int round = 0; round < topk; ++round) {
             float bv = -INFINITY;
             int bi = 0x7fffffff;
@@ -287,21 +288,28 @@ __global__ void __launch_bounds__(512, 1) bra_image_kernel(const __grid_constant
             }
             if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
             if (lane == (round & 31)) {
-                my_v = bv;
-                my_i = bi;
+                my_v[round >> 5] = bv;
+                my_i[round >> 5] = bi;
             }
             if (round == 0) v0 = bv;
         }
-        // r_weight: softmax of the selected logits (topk <= 32 here)
-        const float ex = lane < topk ? expf(my_v - v0) : 0.f;
-        float z = ex;
+        // r_weight: softmax of the selected logits
+        float ex[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) ex[e] = lane + 32 * e < topk ? expf(my_v[e] - v0) : 0.f;
+        float z = ex[0] + ex[1];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-        if (lane < topk) {
-            const size_t o = ((size_t)n * P + p) * topk + lane;
-            prm.r_idx[o] = my_i;
-            prm.r_weight[o] = ex / z;
-            for (int r = 0; r < prm.heads; ++r) st_dsmem_s32(Rloc + (p * topk + lane) * 4, (uint32_t)r, my_i);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int slot = lane + 32 * e;
+            if (slot < topk) {
+                const size_t o = ((size_t)n * P + p) * topk + slot;
+                prm.r_idx[o] = my_i[e];
+                prm.r_weight[o] = ex[e] / z;
+                for (int r = 0; r < prm.heads; ++r)
+                    st_dsmem_s32(Rloc + (p * topk + slot) * 4, (uint32_t)r, my_i[e]);
+            }
         }
     }
     cluster_arrive();  // every row's routing is in every CTA; the partial affinities are no longer read
