@@ -184,53 +184,86 @@ __global__ void __launch_bounds__(512, 1) bra_image_kernel(const __grid_constant
     }
 
     // ---------------------------------------------------------------- 2. means, partial affinity
-    // one warp per (tensor, region): lane = (channel pair lane & 15, token parity lane >> 4);
-    // the two parities read neighbouring pixels (conflict-free) and meet by a shuffle
-    for (int it = warp; it < 2 * P; it += nwarps) {
-        const int tensor = it >= P, p = it - tensor * P;
-        const uint32_t tile = tensor ? tK : tQ;
-        const int c2 = lane & 15;
-        float sx = 0.f, sy = 0.f;
+    // region sums as column sums on the tensor cores: one warp per (tensor, region),
+    // D[16 x 32] = ones[16 x W2] * X[W2 x 32] (bf16 in, fp32 accumulate: exact products,
+    // fp32 sums), X read with ldmatrix.trans like the V operand of the attention; every
+    // row of D holds the sums, lanes 0-3 write row 0.
+    {
+        const int kc = 2 * (lane & 3);  // this lane's k (token) pair in the A fragment
+        const uint32_t one2 = 0x3F803F80u;
+        uint32_t a1[4];
+        a1[0] = a1[1] = kc < W2 ? one2 : 0u;          // tokens kc, kc+1
+        a1[2] = a1[3] = kc + 8 < W2 ? one2 : 0u;      // tokens kc+8, kc+9
+        const int tl = (lane & 7) + ((lane >> 3) & 1) * 8;  // token row this lane addresses
+        const int tt = tl < W2 ? tl : 0;                     // rows past W2 meet zeros in A
+        const int toff = (tt / WR) * W + (tt % WR);
+        for (int it = warp; it < 2 * P; it += nwarps) {
+            const int tensor = it >= P, p = it - tensor * P;
+            const uint32_t tile = tensor ? tK : tQ;
+            const int row = rbase[p] + toff;
+            float d[4][4];
 #pragma unroll
-        for (int t = lane >> 4; t < W2; t += 2) {
-            const int row = rbase[p] + (t / WR) * W + (t % WR);
-            const float2 f = bf16x2_to_float2(ld_shared_u32(swz64(tile, row, c2 >> 2) + (c2 & 3) * 4));
-            sx += f.x;
-            sy += f.y;
-        }
-        sx += __shfl_xor_sync(0xffffffffu, sx, 16);
-        sy += __shfl_xor_sync(0xffffffffu, sy, 16);
-        if (lane < 16) {
-            if (tensor) {
-                kr[p * 36 + 2 * c2] = sx / (float)W2;
-                kr[p * 36 + 2 * c2 + 1] = sy / (float)W2;
-            } else {
-                qr[p * 32 + 2 * c2] = prm.scale * (sx / (float)W2);  // scale*q_r, as the walk-through
-                qr[p * 32 + 2 * c2 + 1] = prm.scale * (sy / (float)W2);
+            for (int t = 0; t < 4; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+#pragma unroll
+            for (int dp = 0; dp < 2; ++dp) {
+                uint32_t b0, b1, b2, b3;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                             : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3)
+                             : "r"(swz64(tile, row, dp * 2 + ((lane >> 4) & 1))));
+                mma_bf16_16816(d[2 * dp], a1, b0, b1);
+                mma_bf16_16816(d[2 * dp + 1], a1, b2, b3);
+            }
+            if (lane < 4) {
+                const float inv = 1.f / (float)W2;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int c = 8 * t + kc;
+                    if (tensor) {
+                        *reinterpret_cast<float2 *>(kr + p * 36 + c) = make_float2(d[t][0] * inv, d[t][1] * inv);
+                    } else {  // scale * q_r, as the walk-through
+                        *reinterpret_cast<float2 *>(qr + p * 32 + c) =
+                            make_float2(prm.scale * (d[t][0] * inv), prm.scale * (d[t][1] * inv));
+                    }
+                }
             }
         }
     }
     __syncthreads();
-    // one warp per affinity row p, lane = columns lane and lane + 32
-    for (int p = warp; p < P; p += nwarps) {
-        float acc0 = 0.f, acc1 = 0.f;
-        const int c1 = lane, cB = lane + 32 < P ? lane + 32 : lane;
+    // affinity rows two at a time per warp (they share the key loads), lane = columns
+    // lane and lane + 32; one partial sum per float4 component keeps the chains short
+    for (int p = 2 * warp; p < P; p += 2 * nwarps) {
+        const int p2 = p + 1 < P ? p + 1 : p;
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
+        const int c1 = lane < P ? lane : 0, cB = lane + 32 < P ? lane + 32 : lane;
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
             const float4 qv = *reinterpret_cast<const float4 *>(qr + p * 32 + c);
-            const float4 k0 = *reinterpret_cast<const float4 *>(kr + (c1 < P ? c1 : 0) * 36 + c);
+            const float4 qw = *reinterpret_cast<const float4 *>(qr + p2 * 32 + c);
+            const float4 k0 = *reinterpret_cast<const float4 *>(kr + c1 * 36 + c);
             const float4 k1 = *reinterpret_cast<const float4 *>(kr + cB * 36 + c);
-            acc0 = fmaf(qv.x, k0.x, acc0);
-            acc0 = fmaf(qv.y, k0.y, acc0);
-            acc0 = fmaf(qv.z, k0.z, acc0);
-            acc0 = fmaf(qv.w, k0.w, acc0);
-            acc1 = fmaf(qv.x, k1.x, acc1);
-            acc1 = fmaf(qv.y, k1.y, acc1);
-            acc1 = fmaf(qv.z, k1.z, acc1);
-            acc1 = fmaf(qv.w, k1.w, acc1);
+            a0.x = fmaf(qv.x, k0.x, a0.x);
+            a0.y = fmaf(qv.y, k0.y, a0.y);
+            a0.z = fmaf(qv.z, k0.z, a0.z);
+            a0.w = fmaf(qv.w, k0.w, a0.w);
+            a1.x = fmaf(qv.x, k1.x, a1.x);
+            a1.y = fmaf(qv.y, k1.y, a1.y);
+            a1.z = fmaf(qv.z, k1.z, a1.z);
+            a1.w = fmaf(qv.w, k1.w, a1.w);
+            b0.x = fmaf(qw.x, k0.x, b0.x);
+            b0.y = fmaf(qw.y, k0.y, b0.y);
+            b0.z = fmaf(qw.z, k0.z, b0.z);
+            b0.w = fmaf(qw.w, k0.w, b0.w);
+            b1.x = fmaf(qw.x, k1.x, b1.x);
+            b1.y = fmaf(qw.y, k1.y, b1.y);
+            b1.z = fmaf(qw.z, k1.z, b1.z);
+            b1.w = fmaf(qw.w, k1.w, b1.w);
         }
-        if (c1 < P) A[p * P + c1] = acc0;
-        if (lane + 32 < P) A[p * P + lane + 32] = acc1;
+        if (lane < P) A[p * P + lane] = (a0.x + a0.y) + (a0.z + a0.w);
+        if (lane + 32 < P) A[p * P + lane + 32] = (a1.x + a1.y) + (a1.z + a1.w);
+        if (p2 != p) {
+            if (lane < P) A[p2 * P + lane] = (b0.x + b0.y) + (b0.z + b0.w);
+            if (lane + 32 < P) A[p2 * P + lane + 32] = (b1.x + b1.y) + (b1.z + b1.w);
+        }
     }
 
     // ---------------------------------------------------------------- 3. routing
