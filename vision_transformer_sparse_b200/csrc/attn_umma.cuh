@@ -10,26 +10,34 @@
 // Shapes: bf16, head dim 32, regions of 128 or 256 tokens (hr a multiple of 8, wr
 // even), topk * w2 <= 256 keys per query. Work unit = (image n, query region p, head
 // h); a CTA (one per SM) keeps one head and walks its units through two shared-memory
-// stages. Warp roles:
+// stages. Each 128-query tile t owns 256 TMEM columns, used as two halves of 128: the
+// scores of keys 0..127 of unit k go to half F(k) = k mod 2, those of keys 128..255 to the
+// other half G(k). O(k) accumulates in the first 32 columns of F(k) and every P is
+// written over scores already read, so the next unit's first-half scores (into G(k)) can
+// be computed as soon as O(k) is complete, while O(k) itself is still being read.
+// Warp roles:
 //   - warp 0, lane 0: TMA producer. Per unit: the Q tile (w2 rows of 32 channels,
 //     64-byte swizzle), the K and V tiles of the routed regions (same layout) and the
 //     V halo of the query region ((hr+4) x (wr+4) pixels, no swizzle, zero outside the
 //     image) onto the stage's "full" barrier.
-//   - warps 1 and 2, lane 0: MMA issuers, one per 128-query tile t (TMEM buffer t of
-//     256 columns): S_t = Q_t K^T (N = topk * w2), then O_t = P_t V with P_t read from
-//     TMEM (the A operand) and V from shared memory (MN-major), four 16-key steps per
-//     64-key chunk pair as soon as that pair's P is stored. The two issuers run
-//     independently, so one tile's softmax never waits for the other's.
-//   - warps 3..10: softmax, two warpgroups; warpgroup t owns TMEM buffer t and each
-//     thread one query row. One pass over the scores, two 32-key chunks at a time:
+//   - warps 1 and 2, lane 0: MMA issuers, one per tile t: S_F = Q_t K_{0..127}^T, then
+//     (once the epilogue has read the previous O) S_G = Q_t K_{128..255}^T, then
+//     O_t = P_t V with P_t read from TMEM (the A operand) and V from shared memory
+//     (MN-major), four 16-key steps per 64-key chunk pair as soon as that pair's P is
+//     stored.
+//   - warps 3..10: softmax, two warpgroups; warpgroup t owns tile t, each thread one
+//     query row, and does nothing but the passes: two 32-key chunks at a time,
 //     p = 2^((s - m) * scale * log2 e) on the MUFU with m the max of the first valid
-//     chunk, row sum in fp32, P packed to bf16 over scores already read. A row whose
-//     p, sum or O is not finite (a later key far above m) is recomputed exactly from
-//     the stage's Q, K, V. Epilogue: O / l + LCE, rounded once to bf16, written to a
-//     64B-swizzled smem tile that one thread stores with the TMA.
-//   - warps 11..14: LCE. The depthwise 5x5 convolution plus bias of the unit's pixels
-//     in fp32 (one channel pair per thread, weights in registers, 8 rows x 2 columns
-//     per item) into an fp32 staging tile that the softmax epilogue adds.
+//     chunk, row sum in fp32, P packed to bf16 over scores already read; the row sum
+//     goes to shared memory before the last pair is signalled.
+//   - warps 11..: LCE and epilogue, kUmmaLceWarps / 4 warpgroups. The depthwise 5x5 convolution
+//     plus bias of the unit's pixels in fp32 (one channel pair per thread, weights in
+//     registers, 8 rows x 2 columns per item) into an fp32 staging tile; then warpgroup
+//     g finishes tiles g, g + groups, ..., one query row per thread (the warp's TMEM lane quarter): O read
+//     from TMEM, O / l + LCE rounded once to bf16 into a 64B-swizzled smem tile that
+//     one thread stores with the TMA.
+//     A row whose p, sum or O is not finite (a later key far above m) is recomputed
+//     exactly from the stage's Q, K, V.
 // Every wait is bounded; a wait that runs out raises the device timeout flag and the
 // role leaves its loop. Tensor memory is released on every path.
 #pragma once
@@ -39,7 +47,7 @@
 
 namespace bra {
 
-constexpr int kUmmaLceWarps = 4;
+constexpr int kUmmaLceWarps = 4;  // one or two warpgroups
 constexpr int kUmmaSoftWarp0 = 3;                      // first softmax warp
 constexpr int kUmmaLceWarp0 = kUmmaSoftWarp0 + 8;      // first LCE warp
 constexpr int kUmmaThreads = (kUmmaLceWarp0 + kUmmaLceWarps) * 32;
@@ -49,23 +57,27 @@ constexpr int kUmmaRows = 8;         // LCE output rows per item (two pixel colu
 // barrier slots
 enum {
     kUbFull = 0,      // [2] stage loaded (TMA bytes)
-    kUbEmpty = 2,     // [2] stage free: MMA commits + every LCE and softmax thread
-    kUbSFull = 4,     // [2] S_t in TMEM
-    kUbOFull = 6,     // [2] O_t in TMEM
-    kUbSEmpty = 8,    // [2] TMEM buffer t read (O taken)
-    kUbDrain = 10,    // [2] MMA drain before the TMEM is released
-    kUbOTFree = 12,   // [2] output tile t free (the previous unit's store has read it)
-    kUbOTReady = 14,  // [2] output tile t written by all 128 rows
-    kUbLFull = 16,    // LCE staging written
-    kUbLEmpty = 17,   // LCE staging consumed
-    kUbP = 18,        // [2][4] P of chunk pair j of tile t stored
-    kUbCount = 26
+    kUbEmpty = 2,     // [2] stage free: MMA commits + every LCE/epilogue thread
+    kUbSFullF = 4,    // [2] first-half scores of tile t in TMEM
+    kUbSFullG = 6,    // [2] second-half scores of tile t in TMEM
+    kUbOFull = 8,     // [2] O_t complete in TMEM
+    kUbOEmpty = 10,   // [2] O_t read by the epilogue
+    kUbDrain = 12,    // [2] MMA drain before the TMEM is released
+    kUbOTFree = 14,   // [2] output tile t free (the previous unit's store has read it)
+    kUbOTReady = 16,  // [2] output tile t written by all 128 rows
+    kUbGRead = 18,    // [2] second-half scores of tile t read by the pass
+    kUbPFree = 20,    // [2] P of pair 0 of tile t consumed by the MMA
+    kUbLFull = 22,    // LCE staging written
+    kUbLEmpty = 23,   // LCE staging consumed
+    kUbP = 24,        // [2][4] P of chunk pair j of tile t stored
+    kUbCount = 32
 };
 
 struct UmmaSmem {
     int q, k, v, halo, stage_bytes;  // offsets inside a stage; stage size (1024-aligned)
     int staging;                     // fp32 [w2][kUmmaStagePitch]: LCE + bias
     int otile;                       // bf16 output tiles [2 tiles][128 rows][32] (64B swizzle)
+    int rsum;                        // fp32 [2 tiles][128]: row sums of the current pass
     int idx;                         // int [2][topk]: routing of the unit in each stage
     int bars, tslot, total;
 };
@@ -79,7 +91,8 @@ __host__ __device__ inline UmmaSmem umma_smem_layout(int topk, int w2, int hr, i
     L.stage_bytes = L.halo + (((hr + 4) * (wr + 4) * 64 + 1023) & ~1023);
     L.staging = 2 * L.stage_bytes;
     L.otile = L.staging + ((w2 * kUmmaStagePitch * 4 + 1023) & ~1023);
-    L.idx = L.otile + 2 * 128 * 64;
+    L.rsum = L.otile + 2 * 128 * 64;
+    L.idx = L.rsum + 2 * 128 * 4;
     L.bars = L.idx + ((2 * topk * 4 + 7) & ~7);
     L.tslot = L.bars + kUbCount * 8;
     L.total = L.tslot + 16 + 1024;  // + alignment of the dynamic base to 1024
@@ -232,17 +245,20 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(bars + 8 * (kUbFull + s), 1);
-            mbar_init(bars + 8 * (kUbEmpty + s), nT + 32 * kUmmaLceWarps + 128 * nT);
-            mbar_init(bars + 8 * (kUbSFull + s), 1);
+            mbar_init(bars + 8 * (kUbEmpty + s), nT + 32 * kUmmaLceWarps);
+            mbar_init(bars + 8 * (kUbSFullF + s), 1);
+            mbar_init(bars + 8 * (kUbSFullG + s), 1);
             mbar_init(bars + 8 * (kUbOFull + s), 1);
-            mbar_init(bars + 8 * (kUbSEmpty + s), 128);
+            mbar_init(bars + 8 * (kUbOEmpty + s), 128);
             mbar_init(bars + 8 * (kUbDrain + s), 1);
             mbar_init(bars + 8 * (kUbOTFree + s), 1);
             mbar_init(bars + 8 * (kUbOTReady + s), 128);
+            mbar_init(bars + 8 * (kUbGRead + s), 128);
+            mbar_init(bars + 8 * (kUbPFree + s), 1);
             for (int j = 0; j < 4; ++j) mbar_init(bars + 8 * (kUbP + 4 * s + j), 128);
         }
         mbar_init(bars + 8 * kUbLFull, 32 * kUmmaLceWarps);
-        mbar_init(bars + 8 * kUbLEmpty, 128 * nT);
+        mbar_init(bars + 8 * kUbLEmpty, 32 * kUmmaLceWarps);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -302,44 +318,71 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
         }
     } else if (warp < kUmmaSoftWarp0) {
         // ------------------------------------------------------------ MMA issuers (one per tile)
-        // TMEM buffer t (256 columns at tbase + 256 t): S_t over all of it, then P_t in
-        // place (pair 0 in columns 32..63, pair j > 0 in 64 j .. 64 j + 31) and O_t in
-        // columns 0..31, whose scores are read before the first PV step.
+        // Unit k of tile t: half F = k mod 2 of the tile's 256 columns takes the scores of
+        // keys 0..127 and O (its columns 0..31), half G the scores of keys 128..255. P of
+        // pair j goes to F + 32 (j + 1) for j < 3 and, once pair 0's MMAs are done, over
+        // P_0 for j = 3, so G holds nothing but scores: the next unit's first-half scores
+        // (into G) are issued as soon as the pass has read them, before the last PV steps.
+        // Writing G(k) = F(k-1) needs unit k-1's MMAs complete and O(k-1) read. With 128
+        // keys (no second half) the next unit's scores wait for that read as well.
         const int t = warp - 1;
         if (lane == 0 && t < nT) {
-            const uint32_t idS = idesc_bf16_f32(128, Lk, 0, 0);
+            const uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
             const uint32_t idV = idesc_bf16_f32(128, 32, 0, 1);
             const uint32_t d = tbase + 256 * t;
             bool ok = true;
             int k = 0;
+            auto issue_s = [&](uint32_t dst, uint32_t stage, int key0) {
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk)
+                    umma_ss(dst, smem_desc(stage + L.q + t * 8192 + 32 * kk, 16, 512, kDescSwizzle64B),
+                            smem_desc(stage + L.k + key0 * 64 + 32 * kk, 16, 512, kDescSwizzle64B), idS, (uint32_t)kk);
+            };
             for (int ru = ru0; ru < prm.regions && ok; ru += stride_ru, ++k) {
                 const int s = k & 1, use = k >> 1;
                 const uint32_t st = base + s * L.stage_bytes;
+                const uint32_t F = d + 128 * (k & 1), G = d + 128 * ((k & 1) ^ 1);
+                const bool next = ru + stride_ru < prm.regions;
                 if (!mbar_wait_bounded(bars + 8 * (kUbFull + s), use & 1, lim) ||
-                    (k > 0 && !mbar_wait_bounded(bars + 8 * (kUbSEmpty + t), (k - 1) & 1, lim))) {
+                    (k > 0 && !mbar_wait_bounded(bars + 8 * (kUbOFull + t), (k - 1) & 1, lim)) ||
+                    (k > 0 && !mbar_wait_bounded(bars + 8 * (kUbOEmpty + t), (k - 1) & 1, lim))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk)
-                    umma_ss(d, smem_desc(st + L.q + t * 8192 + 32 * kk, 16, 512, kDescSwizzle64B),
-                            smem_desc(st + L.k + 32 * kk, 16, 512, kDescSwizzle64B), idS, (uint32_t)kk);
-                umma_commit(bars + 8 * (kUbSFull + t));
+                if (np < 4 || k == 0) {  // otherwise issued during the previous unit
+                    issue_s(F, st, 0);
+                    umma_commit(bars + 8 * (kUbSFullF + t));
+                }
+                if (np == 4) {
+                    issue_s(G, st, 128);
+                    umma_commit(bars + 8 * (kUbSFullG + t));
+                }
                 // O_t = P_t V, one chunk pair (four 16-key steps) as soon as its P is stored
                 for (int j = 0; j < np; ++j) {
+                    if (j == 3 && next) {  // the next unit's first half, into G
+                        if (!mbar_wait_bounded(bars + 8 * (kUbGRead + t), k & 1, lim) ||
+                            !mbar_wait_bounded(bars + 8 * (kUbFull + (s ^ 1)), ((k + 1) >> 1) & 1, lim)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_s(G, base + (s ^ 1) * L.stage_bytes, 0);
+                        umma_commit(bars + 8 * (kUbSFullF + t));
+                    }
                     if (!mbar_wait_bounded(bars + 8 * (kUbP + 4 * t + j), k & 1, lim)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t pcol = d + (j == 0 ? 32 : 64 * j);
+                    const uint32_t pcol = F + 32 * (j < 3 ? j + 1 : 1);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int kk = 4 * j + i;
-                        umma_ts(d, pcol + 8 * i, smem_desc(st + L.v + 1024 * kk, 0, 512, kDescSwizzle64B), idV,
+                        umma_ts(F, pcol + 8 * i, smem_desc(st + L.v + 1024 * kk, 0, 512, kDescSwizzle64B), idV,
                                 (uint32_t)(kk > 0));
                     }
+                    if (j == 0 && np == 4) umma_commit(bars + 8 * (kUbPFree + t));
                 }
                 if (!ok) break;
                 umma_commit(bars + 8 * (kUbOFull + t));
@@ -354,131 +397,134 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
         // ------------------------------------------------------------ softmax warpgroups
         const int t = (warp - kUmmaSoftWarp0) >> 2, sub = warp & 3;
         if (t < nT) {
-            const int row = 32 * sub + lane, qi = t * 128 + row;
+            const int row = 32 * sub + lane;
             const uint32_t trow = tbase + ((uint32_t)(32 * sub) << 16) + 256 * t;
             const float sl2 = prm.scale_log2;
-            const float4 *srow = reinterpret_cast<const float4 *>(sStage + qi * kUmmaStagePitch);
-            const bool leader = row == 0;
-            const uint32_t ot = base + L.otile + t * 8192;
+            float *rsum = reinterpret_cast<float *>(sm + L.rsum) + t * 128 + row;
             int k = 0;
             for (int ru = ru0; ru < prm.regions; ru += stride_ru, ++k) {
                 const int s = k & 1, use = k >> 1;
                 if (!umma_wait_warp(bars + 8 * (kUbFull + s), use & 1, lim)) break;
                 const bool v0 = sIdx[s * prm.topk] >= 0;
                 const bool v1 = prm.topk > 1 ? sIdx[s * prm.topk + 1] >= 0 : true;
-                if (!umma_wait_warp(bars + 8 * (kUbSFull + t), k & 1, lim)) break;
+                const uint32_t F = trow + 128 * (k & 1), G = trow + 128 * ((k & 1) ^ 1);
+                if (!umma_wait_warp(bars + 8 * (kUbSFullF + t), k & 1, lim)) break;
                 tc_fence_after();
+                bool gready = np < 4, fail = false;
+                auto wait_g = [&]() {
+                    if (!gready) {
+                        if (!umma_wait_warp(bars + 8 * (kUbSFullG + t), k & 1, lim)) return false;
+                        tc_fence_after();
+                        gready = true;
+                    }
+                    return true;
+                };
                 // reference: the exact max of the first valid 32-key chunk. Every p is
                 // taken relative to it; a row whose later keys exceed it by so much that p,
                 // the row sum or O overflows is recomputed exactly in the epilogue.
-                const int cv = v0 ? 0 : ((prm.topk > 1 && v1) ? (prm.w2 >> 5) : -1);
                 uint32_t ra[32], rb[32];
                 float m = -INFINITY;
-                if (cv == 0) {
-                    tmem_ld32_nowait(trow, ra);
-                    tmem_ld32_nowait(trow + 32, rb);
+                bool have = false;  // ra, rb hold the scores of the next pair
+                if (v0) {
+                    tmem_ld32_nowait(F, ra);
+                    tmem_ld32_nowait(F + 32, rb);
                     tmem_wait_ld(ra);
                     tmem_regs_after_wait(rb);
                     m = max32(ra, -INFINITY);
-                } else if (cv > 0) {
-                    tmem_ld32(trow + 32 * cv, ra);
+                    have = true;
+                } else if (np == 4 && prm.topk > 1 && v1) {  // keys 128..255: the second region
+                    if (!wait_g()) break;
+                    tmem_ld32(G, ra);
                     m = max32(ra, -INFINITY);
                 }
                 // single pass over chunk pairs (64 independent exponentials in flight per
-                // thread): probabilities, row sum, P (bf16) over scores already read; each
-                // pair's P is handed to the MMA issuer as soon as it is stored
+                // thread): probabilities, row sum, P (bf16) over scores already read. Each
+                // pair's P is handed to the MMA issuer as soon as it is stored, the next
+                // pair's scores being loaded meanwhile.
                 const float mneg = m == -INFINITY ? 0.f : -m * sl2;
                 const float2 sl2v = make_float2(sl2, sl2), mnv = make_float2(mneg, mneg);
                 float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
                 float2 lc = make_float2(0.f, 0.f), ld = make_float2(0.f, 0.f);
                 for (int j = 0; j < np; ++j) {
-                    if (j > 0 || cv != 0) {
-                        tmem_ld32_nowait(trow + 64 * j, ra);
-                        tmem_ld32_nowait(trow + 64 * j + 32, rb);
+                    const bool valid = (j << 6) < prm.w2 ? v0 : v1;  // both chunks of a pair lie in one region
+                    if (valid && !have) {
+                        if (j >= 2 && !wait_g()) {
+                            fail = true;
+                            break;
+                        }
+                        const uint32_t c = j < 2 ? F + 64 * j : G + 64 * (j - 2);
+                        tmem_ld32_nowait(c, ra);
+                        tmem_ld32_nowait(c + 32, rb);
                         tmem_wait_ld(ra);
                         tmem_regs_after_wait(rb);
                     }
+                    if (j == 3) {  // every score of G has been read: the next unit may take G
+                        if (!wait_g()) {
+                            fail = true;
+                            break;
+                        }
+                        tc_fence_before();
+                        umma_arrive(bars + 8 * (kUbGRead + t));
+                    }
                     uint32_t pa[16], pb[16];
-                    if ((j << 6) < prm.w2 ? v0 : v1) {  // both chunks of a pair lie in one region
+                    if (valid) {
                         exp32(ra, sl2v, mnv, la, lb, pa);
                         exp32(rb, sl2v, mnv, lc, ld, pb);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pa[e] = pb[e] = 0u;
                     }
-                    const uint32_t pcol = trow + (j == 0 ? 32 : 64 * j);
+                    if (j == 3) {  // P_3 goes over P_0: wait for pair 0's MMAs
+                        if (!umma_wait_warp(bars + 8 * (kUbPFree + t), k & 1, lim)) {
+                            fail = true;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    const uint32_t pcol = F + 32 * (j < 3 ? j + 1 : 1);
                     tmem_st16_nowait(pcol, pa);
                     tmem_st16_nowait(pcol + 16, pb);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    umma_arrive(bars + 8 * (kUbP + 4 * t + j));
-                }
-                if (leader) {
-                    bulk_wait_read<0>();  // the previous unit's store has read the output tile
-                    umma_arrive(bars + 8 * (kUbOTFree + t));
-                }
-                // epilogue: O / l + LCE + bias -> out
-                if (!umma_wait_warp(bars + 8 * (kUbOFull + t), k & 1, lim)) break;
-                tc_fence_after();
-                uint32_t o[32];
-                tmem_ld32(trow, o);
-                tc_fence_before();
-                umma_arrive(bars + 8 * (kUbSEmpty + t));  // the buffer may take the next S
-                float l = ((la.x + la.y) + (lb.x + lb.y)) + ((lc.x + lc.y) + (ld.x + ld.y));
-                float ck[4] = {l, 0.f, 0.f, 0.f};  // NaN unless l and every O value are finite
-#pragma unroll
-                for (int e = 0; e < 32; ++e) ck[e & 3] = fmaf(__uint_as_float(o[e]), 0.f, ck[e & 3]);
-                if (!(fabsf((ck[0] + ck[1]) + (ck[2] + ck[3])) <= 3.0e38f)) {
-                    float of[32];
-                    umma_exact_row(sm + s * L.stage_bytes, L, qi, prm.w2, prm.topk, v0, v1, sl2, of, l);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(of[e]);
-                }
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                if (!umma_wait_warp(bars + 8 * kUbLFull, k & 1, lim)) break;
-                uint4 ov[4];
-                uint32_t *ow = reinterpret_cast<uint32_t *>(ov);
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    const float4 a = srow[q4];
-                    ow[2 * q4] = pack_bf16x2(fmaf(__uint_as_float(o[4 * q4]), inv, a.x),
-                                             fmaf(__uint_as_float(o[4 * q4 + 1]), inv, a.y));
-                    ow[2 * q4 + 1] = pack_bf16x2(fmaf(__uint_as_float(o[4 * q4 + 2]), inv, a.z),
-                                                 fmaf(__uint_as_float(o[4 * q4 + 3]), inv, a.w));
-                }
-                umma_arrive(bars + 8 * kUbLEmpty);  // staging row consumed
-                // the row goes to the tile's smem image; one thread stores the whole tile
-                if (!umma_wait_warp(bars + 8 * (kUbOTFree + t), k & 1, lim)) break;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + (ot - base) + row * 64 + ((q4 ^ ((row >> 1) & 3)) << 4)) = ov[q4];
-                fence_proxy_async();  // the rows are read by the tensor store
-                umma_arrive(bars + 8 * (kUbOTReady + t));
-                if (sub == 0) {  // the leader's warp: keep its control flow uniform
-                    bool stored = true;
-                    if (leader) {
-                        stored = mbar_wait_bounded(bars + 8 * (kUbOTReady + t), k & 1, lim);
-                        if (stored) {
-                            uint32_t pr, ir;
-                            const int n = (int)prm.div_P.divmod((uint32_t)ru, pr);
-                            const int j = (int)prm.div_S.divmod(pr, ir);
-                            tma_store_4d(&prm.tmO, ot, c0, (int)ir * prm.wr, j * prm.hr + t * (128 / prm.wr), n);
-                            bulk_commit();
-                        }
+                    // the next pair's scores are loaded while the stores drain (the load and
+                    // its wait stay in one branch, so no copy of a pending register is made)
+                    const int jn = j + 1;
+                    have = jn < np && ((jn << 6) < prm.w2 ? v0 : v1);
+                    if (have && jn >= 2 && !wait_g()) {
+                        fail = true;
+                        have = false;
                     }
-                    if (!__shfl_sync(0xffffffffu, stored, 0)) break;
+                    if (have) {
+                        const uint32_t c = jn < 2 ? F + 64 * jn : G + 64 * (jn - 2);
+                        tmem_ld32_nowait(c, ra);
+                        tmem_ld32_nowait(c + 32, rb);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        umma_arrive(bars + 8 * (kUbP + 4 * t + j));
+                        tmem_wait_ld(ra);
+                        tmem_regs_after_wait(rb);
+                    } else {
+                        tmem_wait_st();
+                        if (j == np - 1) *rsum = ((la.x + la.y) + (lb.x + lb.y)) + ((lc.x + lc.y) + (ld.x + ld.y));
+                        tc_fence_before();
+                        umma_arrive(bars + 8 * (kUbP + 4 * t + j));
+                    }
+                    if (fail) break;
                 }
-                umma_arrive(bars + 8 * (kUbEmpty + s));  // Q, K, V of the stage no longer needed
+                if (fail) break;
             }
             if (lane == 0 && ru0 + k * stride_ru < prm.regions) atomicExch(&g_bra_timeout_flag, 1);
-            if (leader) bulk_wait<0>();  // the output tiles are written before the CTA exits
         }
     } else {
-        // ------------------------------------------------------------ LCE warps
-        // Item = (channel pair, two adjacent pixel columns, 8 rows): the 12 x 6 halo
-        // values it reads feed all 16 of its outputs.
+        // ------------------------------------------------------------ LCE + epilogue warps
+        // LCE item = (channel pair, two adjacent pixel columns, 8 rows): the 12 x 6 halo
+        // values it reads feed all 16 of its outputs, split over both warpgroups.
+        // Epilogue: warpgroup t finishes tile t, one query row per thread (the warp's TMEM
+        // lane quarter).
         const int lt = tid - kUmmaLceWarp0 * 32;
         const int pair = lt & 15;
+        const int erow = 32 * (warp & 3) + lane;
+        const int tw = lt >> 7;  // the warpgroup: the epilogue's first tile
+        const uint32_t etm = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
+        const float *sRsum = reinterpret_cast<const float *>(sm + L.rsum);
         const int c = c0 + 2 * pair;
         float2 wt[25];
         {
@@ -537,9 +583,91 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
                 }
             }
             umma_arrive(bars + 8 * kUbLFull);
-            umma_arrive(bars + 8 * (kUbEmpty + s));  // halo of the stage is read
+            if (!umma_wait_warp(bars + 8 * kUbLFull, k & 1, lim)) break;  // every staging row written
+            // ---- epilogue, tiles t = warpgroup, warpgroup + warpgroups, ...: O / l + LCE + bias -> out
+            bool fail = false;
+            for (int t = tw; t < nT; t += kUmmaLceWarps / 4) {
+                const bool leader = lt == 128 * tw;  // stores the warpgroup's tiles
+                if (leader) {
+                    // the previous unit's store of this tile has read it (a warpgroup that
+                    // owns both tiles has just issued this unit's store of tile 0)
+                    if (t > tw)
+                        bulk_wait_read<1>();
+                    else
+                        bulk_wait_read<0>();
+                    umma_arrive(bars + 8 * (kUbOTFree + t));
+                }
+                const int qi = t * 128 + erow;
+                if (!umma_wait_warp(bars + 8 * (kUbOFull + t), k & 1, lim) ||
+                    !umma_wait_warp(bars + 8 * (kUbP + 4 * t + np - 1), k & 1, lim)) {  // row sums stored
+                    fail = true;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t o[32];
+                tmem_ld32(etm + 256 * t + 128 * (k & 1), o);
+                float l = sRsum[t * 128 + erow];
+                tc_fence_before();
+                umma_arrive(bars + 8 * (kUbOEmpty + t));  // the half may take the next scores
+                float ck[4] = {l, 0.f, 0.f, 0.f};  // NaN unless l and every O value are finite
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ck[e & 3] = fmaf(__uint_as_float(o[e]), 0.f, ck[e & 3]);
+                if (!(fabsf((ck[0] + ck[1]) + (ck[2] + ck[3])) <= 3.0e38f)) {
+                    const bool v0 = sIdx[s * prm.topk] >= 0;
+                    const bool v1 = prm.topk > 1 ? sIdx[s * prm.topk + 1] >= 0 : true;
+                    float of[32];
+                    umma_exact_row(sm + s * L.stage_bytes, L, qi, prm.w2, prm.topk, v0, v1, prm.scale_log2, of, l);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(of[e]);
+                }
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                const float4 *srow = reinterpret_cast<const float4 *>(sStage + qi * kUmmaStagePitch);
+                uint4 ov[4];
+                uint32_t *ow = reinterpret_cast<uint32_t *>(ov);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 a = srow[q4];
+                    ow[2 * q4] = pack_bf16x2(fmaf(__uint_as_float(o[4 * q4]), inv, a.x),
+                                             fmaf(__uint_as_float(o[4 * q4 + 1]), inv, a.y));
+                    ow[2 * q4 + 1] = pack_bf16x2(fmaf(__uint_as_float(o[4 * q4 + 2]), inv, a.z),
+                                                 fmaf(__uint_as_float(o[4 * q4 + 3]), inv, a.w));
+                }
+                // the row goes to the tile's smem image; one thread stores the whole tile
+                if (!umma_wait_warp(bars + 8 * (kUbOTFree + t), k & 1, lim)) {
+                    fail = true;
+                    break;
+                }
+                unsigned char *otile = sm + L.otile + t * 8192;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(otile + erow * 64 + ((q4 ^ ((erow >> 1) & 3)) << 4)) = ov[q4];
+                fence_proxy_async();  // the rows are read by the tensor store
+                umma_arrive(bars + 8 * (kUbOTReady + t));
+                if (warp == kUmmaLceWarp0 + 4 * tw) {  // the storing thread's warp: keep its control flow uniform
+                    bool stored = true;
+                    if (lane == 0) {
+                        stored = mbar_wait_bounded(bars + 8 * (kUbOTReady + t), k & 1, lim);
+                        if (stored) {
+                            uint32_t pr, ir;
+                            const int n = (int)prm.div_P.divmod((uint32_t)ru, pr);
+                            const int j = (int)prm.div_S.divmod(pr, ir);
+                            tma_store_4d(&prm.tmO, base + L.otile + t * 8192, c0, (int)ir * prm.wr,
+                                         j * prm.hr + t * (128 / prm.wr), n);
+                            bulk_commit();
+                        }
+                    }
+                    if (!__shfl_sync(0xffffffffu, stored, 0)) {
+                        fail = true;
+                        break;
+                    }
+                }
+            }
+            if (fail) break;
+            umma_arrive(bars + 8 * kUbLEmpty);       // staging rows consumed
+            umma_arrive(bars + 8 * (kUbEmpty + s));  // halo, Q, K, V of the stage no longer needed
         }
         if (lane == 0 && ru0 + k * stride_ru < prm.regions) atomicExch(&g_bra_timeout_flag, 1);
+        if (lt == 128 * tw) bulk_wait<0>();  // the output tiles are written before the CTA exits
     }
 
     tc_fence_before();
