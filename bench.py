@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch each step directly")
     ap.add_argument("--variant", default="auto", choices=["auto", "generic", "tma", "split", "pipe"],
                     help="attention kernel (auto: persistent TMA pipeline where the shape allows)")
+    ap.add_argument("--source-hash", metavar="KERNEL",
+                    help="print the source hash of a traced kernel class (for a profiles/ summary) and exit")
     return ap.parse_args()
 
 
@@ -92,13 +94,44 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+# The header that defines each traced kernel class; a class's source is that header and
+# every header it includes from csrc/, so a committed profile stays valid until one of
+# those files changes.
+KERNEL_HEADERS = {
+    "attn_umma_kernel": ["attn_umma.cuh"],
+    "bra_image_kernel": ["fused_image.cuh"],
+    "attn_bf16_kernel": ["attn_pipe.cuh", "attn_tma.cuh", "attn.cuh"],
+    "attn_f32_kernel": ["attn.cuh"],
+    "region_mean_kernel": ["route.cuh"],
+    "route_kernel": ["route.cuh"],
+}
+
+
+def kernel_sources(kernel: str):
+    """Sorted csrc/ headers that make up `kernel` (its #include closure)."""
+    csrc = os.path.join(ROOT, "vision_transformer_sparse_b200", "csrc")
+    todo, seen = list(KERNEL_HEADERS.get(kernel, [])), set()
+    if not todo:
+        todo = [n for n in os.listdir(csrc) if n.endswith(".cuh")]
+    while todo:
+        name = todo.pop()
+        if name in seen or not os.path.exists(os.path.join(csrc, name)):
+            continue
+        seen.add(name)
+        with open(os.path.join(csrc, name)) as f:
+            for line in f:
+                line = line.strip()
+                if line.startswith("#include \"") and line.endswith("\""):
+                    todo.append(line[len("#include \""):-1])
+    return sorted(seen)
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "vision_transformer_sparse_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith(".cuh"):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in kernel_sources(kernel):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -116,7 +149,7 @@ def profiled_traffic(kernel: str, workload: str):
                                                                    "units_scale"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
-    if vals.get("source_hash") != kernel_source_hash() or "dram_bytes_per_launch" not in vals:
+    if vals.get("source_hash") != kernel_source_hash(kernel) or "dram_bytes_per_launch" not in vals:
         return None, path
     return float(vals["dram_bytes_per_launch"]), path
 
@@ -251,6 +284,10 @@ def cpu_baseline(w: synth.Workload, budget_s: float = 12.0):
 
 def main():
     args = parse()
+    if args.source_hash:
+        print("%s %s (%s)" % (args.source_hash, kernel_source_hash(args.source_hash),
+                              " ".join(kernel_sources(args.source_hash))))
+        return
     w = synth.WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
