@@ -24,7 +24,13 @@ def to_dev(inp, dtype):
 
 def run_forward(w: synth.Workload, inp):
     d = to_dev(inp, w.dtype)
-    out, r_idx, r_w = bra.forward(d["q"], d["k"], d["v"], d["lce_w"], d["lce_b"], w.heads, w.S, w.topk)
+    # outputs start as NaN / -1, so that an element the kernels leave unwritten fails
+    # instead of passing on whatever an earlier test left in that memory
+    out = torch.full_like(d["q"], float("nan"))
+    r_idx = torch.full((w.N, w.regions, w.topk), -1, dtype=torch.int32, device="cuda")
+    r_w = torch.full((w.N, w.regions, w.topk), float("nan"), dtype=torch.float32, device="cuda")
+    bra.forward(d["q"], d["k"], d["v"], d["lce_w"], d["lce_b"], w.heads, w.S, w.topk, out=out, r_idx=r_idx,
+                r_weight=r_w)
     torch.cuda.synchronize()
     return out.float().cpu().numpy(), r_idx.cpu().numpy(), r_w.cpu().numpy()
 

@@ -34,7 +34,8 @@ struct PipeSmem {
     int q, halo, k, v;                // offsets inside a stage
     int q_half, halo_half, kv_half;
     int stages;                       // offset of stage 0 (from the aligned base)
-    int o;                            // O tile: -1 = inside the stage (over its dead K/V)
+    int o;                            // O tiles: -1 = inside the stage (over its dead K/V), else
+    int o_stride;                     //   one per stage at o + s * o_stride
     int rowmap, idx, flags, bars;     // small arrays: shared / per stage (bars: full, oready, empty)
     int total;
 };
@@ -55,11 +56,15 @@ __host__ __device__ inline PipeSmem pipe_smem_layout(int NS, int topk, int w2, i
     s.stages = 0;
     int end = NS * s.stage_bytes;
     const int o_bytes = QT * 16 * (CH + 4) * 4;
+    s.o_stride = align16(o_bytes);
     if (o_bytes <= 2 * nh * s.kv_half) {
         s.o = -1;  // K/V of the stage are dead once every warp has finished its attention
     } else {
+        // one O tile per stage: the attention warps write unit k+1's O while the
+        // epilogue warps still read unit k's, and a stage is only reused after its
+        // epilogue has released it
         s.o = end;
-        end += align16(o_bytes);
+        end += NS * s.o_stride;
     }
     s.rowmap = end;
     end += align16(kpad * 4);
@@ -455,7 +460,7 @@ __global__ void __launch_bounds__(MAXT, MINB) attn_pipe_kernel(const __grid_cons
             const float inv0 = l_i[0] > 0.f ? 1.f / l_i[0] : 0.f;
             const float inv1 = l_i[1] > 0.f ? 1.f / l_i[1] : 0.f;
             bar_sync_named(2, nAT);  // every attention warp is done with this stage's K/V
-            float *sO = reinterpret_cast<float *>(sm + (L.o >= 0 ? L.o : s * L.stage_bytes + L.k));
+            float *sO = reinterpret_cast<float *>(sm + (L.o >= 0 ? L.o + s * L.o_stride : s * L.stage_bytes + L.k));
             {
                 const int r0 = mt * 16 + (lane >> 2);
 #pragma unroll
@@ -511,7 +516,8 @@ __global__ void __launch_bounds__(MAXT, MINB) attn_pipe_kernel(const __grid_cons
         decode_unit(pp, u, rb, p, n, j, i);
         const int y0 = j * prm.hr + rb * prm.RB, x0 = i * prm.wr;
         const uint32_t st = base + L.stages + s * L.stage_bytes;
-        const float *sO = reinterpret_cast<const float *>(sm + (L.o >= 0 ? L.o : s * L.stage_bytes + L.k));
+        const float *sO =
+            reinterpret_cast<const float *>(sm + (L.o >= 0 ? L.o + s * L.o_stride : s * L.stage_bytes + L.k));
         __nv_bfloat16 *opx = prm.out + (((size_t)n * prm.H + y0) * prm.W + x0) * prm.C + c0;
         for (int item = et; item < items; item += nET) {
             const int cp = item & (npairs - 1);
