@@ -759,20 +759,40 @@ static int launch_attend(const Shape &s, const void *q, const void *k, const voi
 
 constexpr int kImageWarps = 16;
 
-// The whole forward in one cluster launch when the shape allows it (see include/bra.h).
-static int launch_fused_image(const Shape &s, const void *q, const void *k, const void *v, const void *w,
-                              const void *b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st,
-                              bool *used) {
+// Small images: attention and LCE of one (image, head) from shared memory (see
+// include/bra.h), in one of two forms. Cluster form: everything in one launch, each
+// cluster pooling, scoring and selecting its own image's routing. Routed form: the
+// routing kernels first, then this kernel (programmatic dependent launch; its tile
+// copies overlap the routing). The cluster form repeats its top-k rounds (one warp
+// argmax per selected region) in every CTA, so past 8 routed regions the routed form
+// is faster (measured: 14x14 maps, topk 16: 122 vs 150 us; 28x28, topk 4: 61 vs 59 us).
+static bool fused_routed(const Shape &s) { return s.topk > 8; }
+
+static bool fused_image_shape_ok(const Shape &s, const void *w, const void *b) {
+    if (g_variant.load() != BRA_VARIANT_AUTO) return false;
+    if (s.dtype != BRA_BF16 || s.d != 32 || s.P > 64 || s.topk > 64 || s.heads > 8) return false;
+    if (!((s.hr == 4 && s.wr == 4) || (s.hr == 2 && s.wr == 2))) return false;
+    return s.H + 4 <= 256 && s.W + 4 <= 256 && aligned(w, 4) && aligned(b, 4);
+}
+
+// 16 warps when one CTA fills an SM's shared memory; 8 when two fit (the kernel's 128
+// registers per thread then allow two CTAs per SM).
+static ImageSmem fused_image_layout(const Shape &s, bool routed, int *nwarps) {
+    *nwarps = kImageWarps;
+    if (image_smem_layout(s.H, s.W, s.P, s.topk, s.w2, kImageWarps / 2, routed).total <= kMaxSmem / 2)
+        *nwarps = kImageWarps / 2;
+    return image_smem_layout(s.H, s.W, s.P, s.topk, s.w2, *nwarps, routed);
+}
+
+// routed: r_idx already holds (or, on the stream, will hold) the routing; the kernel
+// reads it and writes neither r_idx nor r_weight.
+static int launch_fused_image(const Shape &s, bool routed, const void *q, const void *k, const void *v,
+                              const void *w, const void *b, void *out, int32_t *r_idx, float *r_weight,
+                              cudaStream_t st, bool *used) {
     *used = false;
-    if (g_variant.load() != BRA_VARIANT_AUTO) return BRA_OK;
-    if (s.dtype != BRA_BF16 || s.d != 32 || s.P > 64 || s.topk > 64 || s.heads > 8) return BRA_OK;
-    if (!((s.hr == 4 && s.wr == 4) || (s.hr == 2 && s.wr == 2))) return BRA_OK;
-    if (s.H + 4 > 256 || s.W + 4 > 256 || !aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
-    // 16 warps when one CTA fills an SM's shared memory; 8 when two fit (the kernel's
-    // 128 registers per thread then allow two CTAs per SM)
-    int nwarps = kImageWarps;
-    if (image_smem_layout(s.H, s.W, s.P, s.topk, s.w2, kImageWarps / 2).total <= kMaxSmem / 2) nwarps = kImageWarps / 2;
-    const ImageSmem L = image_smem_layout(s.H, s.W, s.P, s.topk, s.w2, nwarps);
+    if (!fused_image_shape_ok(s, w, b)) return BRA_OK;
+    int nwarps = 0;
+    const ImageSmem L = fused_image_layout(s, routed, &nwarps);
     if (L.total > kMaxSmem) return BRA_OK;
     ImageParams p;
     memset(&p, 0, sizeof(p));
@@ -798,7 +818,20 @@ static int launch_fused_image(const Shape &s, const void *q, const void *k, cons
     p.wait_limit = kWaitLimit;
     p.div_S = FastDiv((uint32_t)s.S);
     p.div_W = FastDiv((uint32_t)s.W);
-    auto kern = s.hr == 4 ? bra_image_kernel<4, 4> : bra_image_kernel<2, 2>;
+    if (routed) {
+        auto kern = s.hr == 4 ? bra_image_kernel<4, 4, true> : bra_image_kernel<2, 2, true>;
+        int per_sm = 0;
+        if (allow_smem(kern, L.total) != cudaSuccess ||
+            occupancy(&per_sm, kern, nwarps * 32, L.total, 0, nullptr) != cudaSuccess || per_sm < 1) {
+            cudaGetLastError();
+            return BRA_OK;
+        }
+        *used = true;
+        LaunchScope ls(BRA_KERNEL_FUSED_IMAGE, st);
+        return launch_pdl(kern, dim3(s.N * s.heads), dim3(nwarps * 32), L.total, st, p) == cudaSuccess ? BRA_OK
+                                                                                                      : BRA_ERR_CUDA;
+    }
+    auto kern = s.hr == 4 ? bra_image_kernel<4, 4, false> : bra_image_kernel<2, 2, false>;
     if (allow_smem(kern, L.total) != cudaSuccess) return BRA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(s.N * s.heads);
@@ -967,14 +1000,18 @@ static int forward_device(const Shape &s, const void *q, const void *k, const vo
                           const void *lce_b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st,
                           float *ws_given = nullptr) {
     bool fused = false;
-    int frc = launch_fused_image(s, q, k, v, lce_w, lce_b, out, r_idx, r_weight, st, &fused);
-    if (frc || fused) return frc;
+    const bool routed = fused_routed(s) && fused_image_shape_ok(s, lce_w, lce_b);
+    if (!routed) {
+        const int frc = launch_fused_image(s, false, q, k, v, lce_w, lce_b, out, r_idx, r_weight, st, &fused);
+        if (frc || fused) return frc;
+    }
     float *ws = ws_given;
     if (!ws && cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * (size_t)s.N * s.P * s.C * sizeof(float), st) !=
                    cudaSuccess)
         return BRA_ERR_CUDA;
     int rc = launch_route_into(s, q, k, r_idx, r_weight, ws, st);
-    if (rc == BRA_OK) rc = launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, nullptr, st);
+    if (rc == BRA_OK && routed) rc = launch_fused_image(s, true, q, k, v, lce_w, lce_b, out, r_idx, r_weight, st, &fused);
+    if (rc == BRA_OK && !fused) rc = launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, nullptr, st);
     if (!ws_given && cudaFreeAsync(ws, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     return rc;
 }

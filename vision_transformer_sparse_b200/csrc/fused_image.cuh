@@ -54,7 +54,9 @@ struct ImageSmem {
 
 // Byte offsets from a 1024-aligned base. Q and K: H*W pixels of 64 bytes; V: the
 // (H+4) x (W+4) zero-bordered image (the convolution's padding comes with the copy).
-__host__ __device__ inline ImageSmem image_smem_layout(int H, int W, int P, int topk, int w2, int nwarps) {
+// routed: the routing comes from global memory, so no pooling or affinity buffers.
+__host__ __device__ inline ImageSmem image_smem_layout(int H, int W, int P, int topk, int w2, int nwarps,
+                                                       bool routed = false) {
     ImageSmem s;
     const int tile = ((H * W * 64 + 1023) / 1024) * 1024;
     const int vtile = (((H + 4) * (W + 4) * 64 + 1023) / 1024) * 1024;
@@ -63,12 +65,13 @@ __host__ __device__ inline ImageSmem image_smem_layout(int H, int W, int P, int 
     s.k = s.q + tile;
     s.v = s.k + tile;
     int end = s.v + vtile;
+    const int rp = routed ? 0 : P;
     s.qr = end;  // [P][32] fp32 region means of the head's q channels
-    end += align16(P * 32 * 4);
+    end += align16(rp * 32 * 4);
     s.kr = end;  // [P][36]: pitch of 9 16-byte units, conflict-free float4 reads
-    end += align16(P * 36 * 4);
+    end += align16(rp * 36 * 4);
     s.a = end;  // [P][P] partial affinity of this head (read by the cluster peers)
-    end += align16(P * P * 4);
+    end += align16(rp * P * 4);
     s.ridx = end;  // [P][topk]
     end += align16(P * topk * 4);
     s.base = end;  // [P] first pixel row of each region
@@ -109,8 +112,11 @@ __device__ __forceinline__ uint32_t swz64(uint32_t tile, int row, int ck) {
     return tile + row * 64 + (((ck ^ (row >> 1)) & 3) << 4);
 }
 
-// HR x WR regions, 32 channels per head.
-template <int HR, int WR>
+// HR x WR regions, 32 channels per head. kRouted: steps 1-3 ran in the routing kernels
+// before this one (launched with programmatic dependent launch): the kernel copies its
+// tiles while they finish, then takes r_idx from global memory and runs step 4-5 only;
+// no cluster, no pooling, no affinity.
+template <int HR, int WR, bool kRouted>
 __global__ void __launch_bounds__(512, 1) bra_image_kernel(const __grid_constant__ ImageParams prm) {
     constexpr int D = 32, W2 = HR * WR;
     static_assert(W2 <= 16, "a region's queries fill at most one 16-row tile");
@@ -121,9 +127,9 @@ __global__ void __launch_bounds__(512, 1) bra_image_kernel(const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
     const int H = prm.H, W = prm.W, HW = H * W, P = prm.P, topk = prm.topk;
     const int L = topk * W2, kpad = (L + kKC - 1) / kKC * kKC;
-    const ImageSmem Ls = image_smem_layout(H, W, P, topk, W2, nwarps);
+    const ImageSmem Ls = image_smem_layout(H, W, P, topk, W2, nwarps, kRouted);
     const int WP = W + 4;  // padded V row pitch (pixels)
-    const int m = (int)cluster_ctarank();
+    const int m = kRouted ? (int)(blockIdx.x % prm.heads) : (int)cluster_ctarank();
     const int n = blockIdx.x / prm.heads;
     const int c0 = m * D;
     float *qr = reinterpret_cast<float *>(sm + Ls.qr);
@@ -171,182 +177,194 @@ __global__ void __launch_bounds__(512, 1) bra_image_kernel(const __grid_constant
         }
         bias = bf16x2_to_float2(__ldg(reinterpret_cast<const uint32_t *>(prm.lce_b + c)));
     }
+    if constexpr (kRouted) {
+        griddep_wait();  // r_idx comes from the preceding routing kernel
+        const int32_t *src = prm.r_idx + (size_t)n * P * topk;
+        for (int i = tid; i < P * topk; i += blockDim.x) {
+            const int r = __ldcg(src + i);
+            ridx[i] = r >= 0 && r < P ? r : 0;  // the routing kernels only write indices in range
+        }
+    }
     const bool ok = __syncthreads_and(mbar_wait_bounded(bar, 0, prm.wait_limit));
     if (!ok) {
         if (tid == 0) atomicExch(&g_bra_timeout_flag, 1);
         mbar_wait_bounded(bar, 0, prm.wait_limit);
-        // keep the cluster's barrier sequence intact before leaving
-        cluster_arrive();
-        cluster_wait();
-        cluster_arrive();
-        cluster_wait();
+        if constexpr (!kRouted) {
+            // keep the cluster's barrier sequence intact before leaving
+            cluster_arrive();
+            cluster_wait();
+            cluster_arrive();
+            cluster_wait();
+        }
         return;
     }
 
-    // ---------------------------------------------------------------- 2. means, partial affinity
-    // region sums as column sums on the tensor cores: one warp per (tensor, region),
-    // D[16 x 32] = ones[16 x W2] * X[W2 x 32] (bf16 in, fp32 accumulate: exact products,
-    // fp32 sums), X read with ldmatrix.trans like the V operand of the attention; every
-    // row of D holds the sums, lanes 0-3 write row 0.
-    {
-        const int kc = 2 * (lane & 3);  // this lane's k (token) pair in the A fragment
-        const uint32_t one2 = 0x3F803F80u;
-        uint32_t a1[4];
-        a1[0] = a1[1] = kc < W2 ? one2 : 0u;          // tokens kc, kc+1
-        a1[2] = a1[3] = kc + 8 < W2 ? one2 : 0u;      // tokens kc+8, kc+9
-        const int tl = (lane & 7) + ((lane >> 3) & 1) * 8;  // token row this lane addresses
-        const int tt = tl < W2 ? tl : 0;                     // rows past W2 meet zeros in A
-        const int toff = (tt / WR) * W + (tt % WR);
-        for (int it = warp; it < 2 * P; it += nwarps) {
-            const int tensor = it >= P, p = it - tensor * P;
-            const uint32_t tile = tensor ? tK : tQ;
-            const int row = rbase[p] + toff;
-            float d[4][4];
+    if constexpr (!kRouted) {
+        // ---------------------------------------------------------------- 2. means, partial affinity
+        // region sums as column sums on the tensor cores: one warp per (tensor, region),
+        // D[16 x 32] = ones[16 x W2] * X[W2 x 32] (bf16 in, fp32 accumulate: exact products,
+        // fp32 sums), X read with ldmatrix.trans like the V operand of the attention; every
+        // row of D holds the sums, lanes 0-3 write row 0.
+        {
+            const int kc = 2 * (lane & 3);  // this lane's k (token) pair in the A fragment
+            const uint32_t one2 = 0x3F803F80u;
+            uint32_t a1[4];
+            a1[0] = a1[1] = kc < W2 ? one2 : 0u;          // tokens kc, kc+1
+            a1[2] = a1[3] = kc + 8 < W2 ? one2 : 0u;      // tokens kc+8, kc+9
+            const int tl = (lane & 7) + ((lane >> 3) & 1) * 8;  // token row this lane addresses
+            const int tt = tl < W2 ? tl : 0;                     // rows past W2 meet zeros in A
+            const int toff = (tt / WR) * W + (tt % WR);
+            for (int it = warp; it < 2 * P; it += nwarps) {
+                const int tensor = it >= P, p = it - tensor * P;
+                const uint32_t tile = tensor ? tK : tQ;
+                const int row = rbase[p] + toff;
+                float d[4][4];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
+                for (int t = 0; t < 4; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.f;
 #pragma unroll
-            for (int dp = 0; dp < 2; ++dp) {
-                uint32_t b0, b1, b2, b3;
-                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                             : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3)
-                             : "r"(swz64(tile, row, dp * 2 + ((lane >> 4) & 1))));
-                mma_bf16_16816(d[2 * dp], a1, b0, b1);
-                mma_bf16_16816(d[2 * dp + 1], a1, b2, b3);
-            }
-            if (lane < 4) {
-                const float inv = 1.f / (float)W2;
+                for (int dp = 0; dp < 2; ++dp) {
+                    uint32_t b0, b1, b2, b3;
+                    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                                 : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3)
+                                 : "r"(swz64(tile, row, dp * 2 + ((lane >> 4) & 1))));
+                    mma_bf16_16816(d[2 * dp], a1, b0, b1);
+                    mma_bf16_16816(d[2 * dp + 1], a1, b2, b3);
+                }
+                if (lane < 4) {
+                    const float inv = 1.f / (float)W2;
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const int c = 8 * t + kc;
-                    if (tensor) {
-                        *reinterpret_cast<float2 *>(kr + p * 36 + c) = make_float2(d[t][0] * inv, d[t][1] * inv);
-                    } else {  // scale * q_r, as the walk-through
-                        *reinterpret_cast<float2 *>(qr + p * 32 + c) =
-                            make_float2(prm.scale * (d[t][0] * inv), prm.scale * (d[t][1] * inv));
+                    for (int t = 0; t < 4; ++t) {
+                        const int c = 8 * t + kc;
+                        if (tensor) {
+                            *reinterpret_cast<float2 *>(kr + p * 36 + c) = make_float2(d[t][0] * inv, d[t][1] * inv);
+                        } else {  // scale * q_r, as the walk-through
+                            *reinterpret_cast<float2 *>(qr + p * 32 + c) =
+                                make_float2(prm.scale * (d[t][0] * inv), prm.scale * (d[t][1] * inv));
+                        }
                     }
                 }
             }
         }
-    }
-    __syncthreads();
-    // affinity rows two at a time per warp (they share the key loads), lane = columns
-    // lane and lane + 32; one partial sum per float4 component keeps the chains short
-    for (int p = 2 * warp; p < P; p += 2 * nwarps) {
-        const int p2 = p + 1 < P ? p + 1 : p;
-        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
-        const int c1 = lane < P ? lane : 0, cB = lane + 32 < P ? lane + 32 : lane;
+        __syncthreads();
+        // affinity rows two at a time per warp (they share the key loads), lane = columns
+        // lane and lane + 32; one partial sum per float4 component keeps the chains short
+        for (int p = 2 * warp; p < P; p += 2 * nwarps) {
+            const int p2 = p + 1 < P ? p + 1 : p;
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
+            const int c1 = lane < P ? lane : 0, cB = lane + 32 < P ? lane + 32 : lane;
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-            const float4 qv = *reinterpret_cast<const float4 *>(qr + p * 32 + c);
-            const float4 qw = *reinterpret_cast<const float4 *>(qr + p2 * 32 + c);
-            const float4 k0 = *reinterpret_cast<const float4 *>(kr + c1 * 36 + c);
-            const float4 k1 = *reinterpret_cast<const float4 *>(kr + cB * 36 + c);
-            a0.x = fmaf(qv.x, k0.x, a0.x);
-            a0.y = fmaf(qv.y, k0.y, a0.y);
-            a0.z = fmaf(qv.z, k0.z, a0.z);
-            a0.w = fmaf(qv.w, k0.w, a0.w);
-            a1.x = fmaf(qv.x, k1.x, a1.x);
-            a1.y = fmaf(qv.y, k1.y, a1.y);
-            a1.z = fmaf(qv.z, k1.z, a1.z);
-            a1.w = fmaf(qv.w, k1.w, a1.w);
-            b0.x = fmaf(qw.x, k0.x, b0.x);
-            b0.y = fmaf(qw.y, k0.y, b0.y);
-            b0.z = fmaf(qw.z, k0.z, b0.z);
-            b0.w = fmaf(qw.w, k0.w, b0.w);
-            b1.x = fmaf(qw.x, k1.x, b1.x);
-            b1.y = fmaf(qw.y, k1.y, b1.y);
-            b1.z = fmaf(qw.z, k1.z, b1.z);
-            b1.w = fmaf(qw.w, k1.w, b1.w);
+            for (int c = 0; c < 32; c += 4) {
+                const float4 qv = *reinterpret_cast<const float4 *>(qr + p * 32 + c);
+                const float4 qw = *reinterpret_cast<const float4 *>(qr + p2 * 32 + c);
+                const float4 k0 = *reinterpret_cast<const float4 *>(kr + c1 * 36 + c);
+                const float4 k1 = *reinterpret_cast<const float4 *>(kr + cB * 36 + c);
+                a0.x = fmaf(qv.x, k0.x, a0.x);
+                a0.y = fmaf(qv.y, k0.y, a0.y);
+                a0.z = fmaf(qv.z, k0.z, a0.z);
+                a0.w = fmaf(qv.w, k0.w, a0.w);
+                a1.x = fmaf(qv.x, k1.x, a1.x);
+                a1.y = fmaf(qv.y, k1.y, a1.y);
+                a1.z = fmaf(qv.z, k1.z, a1.z);
+                a1.w = fmaf(qv.w, k1.w, a1.w);
+                b0.x = fmaf(qw.x, k0.x, b0.x);
+                b0.y = fmaf(qw.y, k0.y, b0.y);
+                b0.z = fmaf(qw.z, k0.z, b0.z);
+                b0.w = fmaf(qw.w, k0.w, b0.w);
+                b1.x = fmaf(qw.x, k1.x, b1.x);
+                b1.y = fmaf(qw.y, k1.y, b1.y);
+                b1.z = fmaf(qw.z, k1.z, b1.z);
+                b1.w = fmaf(qw.w, k1.w, b1.w);
+            }
+            if (lane < P) A[p * P + lane] = (a0.x + a0.y) + (a0.z + a0.w);
+            if (lane + 32 < P) A[p * P + lane + 32] = (a1.x + a1.y) + (a1.z + a1.w);
+            if (p2 != p) {
+                if (lane < P) A[p2 * P + lane] = (b0.x + b0.y) + (b0.z + b0.w);
+                if (lane + 32 < P) A[p2 * P + lane + 32] = (b1.x + b1.y) + (b1.z + b1.w);
+            }
         }
-        if (lane < P) A[p * P + lane] = (a0.x + a0.y) + (a0.z + a0.w);
-        if (lane + 32 < P) A[p * P + lane + 32] = (a1.x + a1.y) + (a1.z + a1.w);
-        if (p2 != p) {
-            if (lane < P) A[p2 * P + lane] = (b0.x + b0.y) + (b0.z + b0.w);
-            if (lane + 32 < P) A[p2 * P + lane + 32] = (b1.x + b1.y) + (b1.z + b1.w);
-        }
-    }
 
-    // ---------------------------------------------------------------- 3. routing
-    cluster_arrive();  // our partial affinity is complete and visible to the peers
-    cluster_wait();
-    const uint32_t Aloc = sbase + Ls.a;
-    const uint32_t Rloc = sbase + Ls.ridx;
-    // the cluster's CTAs share the rows: this CTA selects rows m, m + heads, ... and
-    // writes each row's routing into every peer's index table
-    for (int p = m + warp * prm.heads; p < P; p += nwarps * prm.heads) {
-        float val[2];
-        int id[2];
-        {
-            // every peer's partial first (independent remote loads), then the sums in rank order
-            float part[2][8];
+        // ---------------------------------------------------------------- 3. routing
+        cluster_arrive();  // our partial affinity is complete and visible to the peers
+        cluster_wait();
+        const uint32_t Aloc = sbase + Ls.a;
+        const uint32_t Rloc = sbase + Ls.ridx;
+        // the cluster's CTAs share the rows: this CTA selects rows m, m + heads, ... and
+        // writes each row's routing into every peer's index table
+        for (int p = m + warp * prm.heads; p < P; p += nwarps * prm.heads) {
+            float val[2];
+            int id[2];
+            {
+                // every peer's partial first (independent remote loads), then the sums in rank order
+                float part[2][8];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int col = min(lane + 32 * e, P - 1);
+                for (int e = 0; e < 2; ++e) {
+                    const int col = min(lane + 32 * e, P - 1);
 #pragma unroll
-                for (int r = 0; r < 8; ++r) part[e][r] = r < prm.heads ? ld_dsmem_f32(Aloc + (p * P + col) * 4, r) : 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int col = lane + 32 * e;
-                float s = 0.f;
-#pragma unroll
-                for (int r = 0; r < 8; ++r)
-                    if (r < prm.heads) s += part[e][r];
-                id[e] = col;
-                val[e] = col < P ? s : -INFINITY;
-            }
-        }
-        // topk rounds of warp argmax (larger logit first, ties to the lower region index);
-        // round r's winner is kept by lane r % 32 in slot r / 32 (topk <= 64)
-        unsigned taken = 0;
-        float my_v[2] = {0.f, 0.f}, v0 = 0.f;
-        int my_i[2] = {0, 0};
-        for (int round = 0; round < topk; ++round) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-                if (!(taken & (1u << e)) && id[e] < P && route_before(val[e], id[e], bv, bi)) {
-                    bv = val[e];
-                    bi = id[e];
+                    for (int r = 0; r < 8; ++r) part[e][r] = r < prm.heads ? ld_dsmem_f32(Aloc + (p * P + col) * 4, r) : 0.f;
                 }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (route_before(ov, oi, bv, bi)) {
-                    bv = ov;
-                    bi = oi;
+                for (int e = 0; e < 2; ++e) {
+                    const int col = lane + 32 * e;
+                    float s = 0.f;
+#pragma unroll
+                    for (int r = 0; r < 8; ++r)
+                        if (r < prm.heads) s += part[e][r];
+                    id[e] = col;
+                    val[e] = col < P ? s : -INFINITY;
                 }
             }
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-            if (lane == (round & 31)) {
-                my_v[round >> 5] = bv;
-                my_i[round >> 5] = bi;
+            // topk rounds of warp argmax (larger logit first, ties to the lower region index);
+            // round r's winner is kept by lane r % 32 in slot r / 32 (topk <= 64)
+            unsigned taken = 0;
+            float my_v[2] = {0.f, 0.f}, v0 = 0.f;
+            int my_i[2] = {0, 0};
+            for (int round = 0; round < topk; ++round) {
+                float bv = -INFINITY;
+                int bi = 0x7fffffff;
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    if (!(taken & (1u << e)) && id[e] < P && route_before(val[e], id[e], bv, bi)) {
+                        bv = val[e];
+                        bi = id[e];
+                    }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                    if (route_before(ov, oi, bv, bi)) {
+                        bv = ov;
+                        bi = oi;
+                    }
+                }
+                if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+                if (lane == (round & 31)) {
+                    my_v[round >> 5] = bv;
+                    my_i[round >> 5] = bi;
+                }
+                if (round == 0) v0 = bv;
             }
-            if (round == 0) v0 = bv;
-        }
-        // r_weight: softmax of the selected logits
-        float ex[2];
+            // r_weight: softmax of the selected logits
+            float ex[2];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) ex[e] = lane + 32 * e < topk ? expf(my_v[e] - v0) : 0.f;
-        float z = ex[0] + ex[1];
+            for (int e = 0; e < 2; ++e) ex[e] = lane + 32 * e < topk ? expf(my_v[e] - v0) : 0.f;
+            float z = ex[0] + ex[1];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int slot = lane + 32 * e;
-            if (slot < topk) {
-                const size_t o = ((size_t)n * P + p) * topk + slot;
-                prm.r_idx[o] = my_i[e];
-                prm.r_weight[o] = ex[e] / z;
-                for (int r = 0; r < prm.heads; ++r)
-                    st_dsmem_s32(Rloc + (p * topk + slot) * 4, (uint32_t)r, my_i[e]);
+            for (int e = 0; e < 2; ++e) {
+                const int slot = lane + 32 * e;
+                if (slot < topk) {
+                    const size_t o = ((size_t)n * P + p) * topk + slot;
+                    prm.r_idx[o] = my_i[e];
+                    prm.r_weight[o] = ex[e] / z;
+                    for (int r = 0; r < prm.heads; ++r)
+                        st_dsmem_s32(Rloc + (p * topk + slot) * 4, (uint32_t)r, my_i[e]);
+                }
             }
         }
+        cluster_arrive();  // every row's routing is in every CTA; the partial affinities are no longer read
+        cluster_wait();
     }
-    cluster_arrive();  // every row's routing is in every CTA; the partial affinities are no longer read
-    cluster_wait();
 
     // ---------------------------------------------------------------- 4. attention + LCE
     const int nchunks = kpad / kKC;
