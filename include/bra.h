@@ -186,12 +186,14 @@ const char *bra_kernel_name(int kernel_class);
 /* ---------------------------------------------------------------------------
  * Kernel selection and device status.
  *
- * By default (BRA_VARIANT_AUTO) a bfloat16 forward whose images are small runs as
- * ONE kernel (pooling, routing, attention and LCE fused; one thread-block cluster of
- * `heads` CTAs per image): this needs d = 32, regions of 4x4 or 2x2 tokens, S*S <= 64,
- * topk <= 64, heads <= 8 and one head's Q, K and V slices of a whole image within one
- * CTA's shared memory. Otherwise the forward runs as three kernels (region means,
- * routing, attention). The bfloat16 attention then runs, in this order of preference:
+ * By default (BRA_VARIANT_AUTO) a bfloat16 forward whose images are small runs its
+ * attention and LCE in one fused kernel that holds one head's Q, K and V slices of a
+ * whole image in shared memory: this needs d = 32, regions of 4x4 or 2x2 tokens,
+ * S*S <= 64, topk <= 64, heads <= 8 and those slices within one CTA's shared memory.
+ * With topk <= 8 the fused kernel also pools and routes (one thread-block cluster of
+ * `heads` CTAs per image, ONE launch in all); with topk > 8 the routing kernels run
+ * first and the fused kernel follows them. Otherwise the forward runs as three kernels
+ * (region means, routing, attention). The bfloat16 attention then runs, in this order of preference:
  *  - on the 5th-generation tensor cores (tcgen05: scores and probabilities in tensor
  *    memory, one CTA per SM) when d = 32, a region holds 128 or 256 tokens (H/S a
  *    multiple of 8, W/S even) and topk * (H/S) * (W/S) <= 256;
