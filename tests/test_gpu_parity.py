@@ -102,6 +102,8 @@ SMALL = [
     (3, 48, 48, 96, 3, 3, 1, "bf16"),     # 16x16 regions, 3 heads, 3 images: tcgen05
     (1, 32, 32, 64, 2, 16, 20, "bf16"),   # 256 regions (column-per-lane routing), topk 20 (sort)
     (6, 16, 16, 64, 2, 16, 2, "bf16"),    # 256 regions, 6 images (8 routing rows per CTA)
+    (2, 12, 12, 64, 2, 6, 12, "bf16"),    # 2x2 regions, topk 12: per-image routing, routed fused kernel
+    (1, 20, 20, 64, 2, 5, 20, "bf16"),    # 4x4 regions, 25 of them, topk 20: the same, one column warp
 ]
 
 
