@@ -381,10 +381,19 @@ __host__ __device__ inline F32Smem f32_smem_layout(int topk, int nq, int RB, int
     return s;
 }
 
-// One thread per (query, head); float32 FMA throughout (exact enough for 1e-4).
+// F32Lanes<D>::n lanes per (query, head), each taking every n-th key of a chunk with
+// its own online softmax; the lanes' partial states (max, sum, O) merge by shuffles at
+// the end. One lane at d = 64, whose q and O rows already fill the registers.
+// float32 FMA throughout (exact enough for 1e-4).
+template <int D> struct F32Lanes {
+    static constexpr int n = D == 32 ? 2 : 1;
+    static constexpr int max_threads = 256;
+};
+
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(F32Lanes<D>::max_threads)
 attn_f32_kernel(const AttnParams prm) {
+    constexpr int kKSF = F32Lanes<D>::n;
     using T = float;
     extern __shared__ __align__(16) unsigned char smem[];
     const int CH = prm.HG * D;
@@ -413,7 +422,8 @@ attn_f32_kernel(const AttnParams prm) {
     load_halo<T>(prm, vg, n, y0, x0, c0, CH, sHalo);
     cp_async_commit();
 
-    const int tq = threadIdx.x % nq, hl = threadIdx.x / nq;
+    const int sub = threadIdx.x % kKSF, qh = threadIdx.x / kKSF;  // the kKSF lanes of a query are adjacent
+    const int tq = qh % nq, hl = qh / nq;
     const bool active = hl < prm.HG;
     float qv[D], acc[D];
     float m_i = -INFINITY, l_i = 0.f;
@@ -435,18 +445,19 @@ attn_f32_kernel(const AttnParams prm) {
         cp_async_wait<0>();
         __syncthreads();
         if (active) {
-            float s[kKCF];
+            float s[kKCF / kKSF];
             float cmax = -INFINITY;
 #pragma unroll
-            for (int kk = 0; kk < kKCF; ++kk) {
+            for (int kq = 0; kq < kKCF / kKSF; ++kq) {
+                const int kk = kq * kKSF + sub;
                 const float *kr = sK + kk * CH + hl * D;
                 float dot = 0.f;
 #pragma unroll
                 for (int c = 0; c < D; ++c) dot = fmaf(qv[c], kr[c], dot);
                 const int key = k0 + kk;
                 const bool ok = key < Lk && (!bad || sIdx[key / prm.w2] >= 0);
-                s[kk] = ok ? dot * prm.scale_log2 : -INFINITY;
-                cmax = fmaxf(cmax, s[kk]);
+                s[kq] = ok ? dot * prm.scale_log2 : -INFINITY;
+                cmax = fmaxf(cmax, s[kq]);
             }
             const float m_new = fmaxf(m_i, cmax);
             const float mref = m_new == -INFINITY ? 0.f : m_new;
@@ -456,17 +467,32 @@ attn_f32_kernel(const AttnParams prm) {
 #pragma unroll
             for (int c = 0; c < D; ++c) acc[c] *= alpha;
 #pragma unroll
-            for (int kk = 0; kk < kKCF; ++kk) {
-                const float pe = exp2f(s[kk] - mref);
+            for (int kq = 0; kq < kKCF / kKSF; ++kq) {
+                const float pe = exp2f(s[kq] - mref);
                 l_i += pe;
-                const float *vr = sV + kk * CH + hl * D;
+                const float *vr = sV + (kq * kKSF + sub) * CH + hl * D;
 #pragma unroll
                 for (int c = 0; c < D; ++c) acc[c] = fmaf(pe, vr[c], acc[c]);
             }
         }
     }
-    if (active) {
-        const float inv = l_i > 0.f ? 1.f / l_i : 0.f;
+    // merge the lanes' partial states: common max, rescaled sums and O
+    float m = m_i;
+#pragma unroll
+    for (int o = 1; o < kKSF; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float f = m_i == -INFINITY ? 0.f : exp2f(m_i - m);
+    float l = l_i * f;
+#pragma unroll
+    for (int o = 1; o < kKSF; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+        float a = acc[c] * f;
+#pragma unroll
+        for (int o = 1; o < kKSF; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        acc[c] = a;
+    }
+    if (active && sub == 0) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
         for (int c = 0; c < D; ++c) sO[tq * L.o_ld + hl * D + c] = acc[c] * inv;
     }

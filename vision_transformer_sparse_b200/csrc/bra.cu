@@ -403,14 +403,17 @@ static bool plan_bf16(const Shape &s, AttnParams &p, int &threads, int &smem) {
     return false;
 }
 
-// SIMT float32 kernel shape: one thread per (query, head), at most 256 per CTA.
+// SIMT float32 kernel shape: F32Lanes<d>::n threads per (query, head), at most
+// F32Lanes<d>::max_threads per CTA.
 static bool plan_f32(const Shape &s, AttnParams &p, int &threads, int &smem) {
+    const int lanes = s.d == 32 ? F32Lanes<32>::n : F32Lanes<64>::n;
+    const int max_threads = s.d == 32 ? F32Lanes<32>::max_threads : F32Lanes<64>::max_threads;
     for (int hg = largest_divisor_at_most(s.heads, 128 / s.d); hg >= 1; --hg) {
         if (s.heads % hg) continue;
         for (int rb = s.hr; rb >= 1; --rb) {
             if (s.hr % rb) continue;
             const int nq = rb * s.wr;
-            if (nq * hg > 256) continue;
+            if (nq * hg * lanes > max_threads) continue;
             const F32Smem L = f32_smem_layout(s.topk, nq, rb, s.wr, hg * s.d);
             if (L.total > kMaxSmem) continue;
             p.HG = hg;
@@ -419,7 +422,7 @@ static bool plan_f32(const Shape &s, AttnParams &p, int &threads, int &smem) {
             p.stages = 1;
             p.n_hg = s.heads / hg;
             p.n_rb = s.hr / rb;
-            threads = ((nq * hg + 31) / 32) * 32;
+            threads = ((nq * hg * lanes + 31) / 32) * 32;
             smem = L.total;
             return true;
         }
