@@ -1,0 +1,64 @@
+"""Host-side logic of bench.py (no GPU): how a committed ncu summary is matched to the
+source it was captured on, and the algorithmic figures the roofline divides by."""
+import importlib.util
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "vision_transformer_sparse_b200", "csrc")
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def includes(name):
+    with open(os.path.join(CSRC, name)) as f:
+        return re.findall(r'^\s*#include "([^"]+)"', f.read(), flags=re.M)
+
+
+def test_kernel_sources_are_the_include_closure(bench):
+    for kernel, heads in bench.KERNEL_HEADERS.items():
+        got = set(bench.kernel_sources(kernel))
+        assert set(heads) <= got, kernel
+        for name in got:  # closed under #include
+            assert set(includes(name)) <= got, (kernel, name)
+        assert "common.cuh" in got
+
+
+def test_fp32_kernel_does_not_depend_on_the_tensor_core_kernels(bench):
+    got = set(bench.kernel_sources("attn_f32_kernel"))
+    assert "attn_umma.cuh" not in got and "umma.cuh" not in got and "fused_image.cuh" not in got
+
+
+def test_profile_lookup_matches_only_the_current_source(bench, tmp_path, monkeypatch):
+    # a summary is used for traffic only while its hash is the kernel's current one
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    os.makedirs(tmp_path / "profiles")
+    os.makedirs(tmp_path / "vision_transformer_sparse_b200")
+    os.symlink(CSRC, tmp_path / "vision_transformer_sparse_b200" / "csrc")
+    h = bench.kernel_source_hash("attn_umma_kernel")
+    (tmp_path / "profiles" / "attn_umma_kernel_w.txt").write_text(
+        "source_hash: %s\ndram_bytes_per_launch: 1234\n" % h)
+    (tmp_path / "profiles" / "attn_umma_kernel_old.txt").write_text(
+        "source_hash: 0000000000000000\ndram_bytes_per_launch: 99\n")
+    assert bench.profiled_traffic("attn_umma_kernel", "w")[0] == 1234.0
+    assert bench.profiled_traffic("attn_umma_kernel", "old")[0] is None
+    assert bench.profiled_traffic("attn_umma_kernel", "missing") == (None, None)
+
+
+def test_algorithmic_figures_of_the_detection_stage(bench):
+    from vision_transformer_sparse_b200 import synth
+    w = synth.WORKLOADS["det_stage1_1024"]
+    acc = bench.algorithmic(w)
+    T = w.N * w.H * w.W
+    L = w.topk * (w.H // w.S) * (w.W // w.S)
+    assert acc["tokens"] == T
+    assert acc["flops"] == 4 * T * L * w.C
+    assert acc["gathered_bytes"] == w.N * w.S * w.S * L * 2 * w.C * 2
