@@ -144,3 +144,63 @@ def forward(q, k, v, lce_w, lce_b, heads: int, S: int, topk: int
 
 def check_shape(N, H, W, C, heads, S, topk) -> bool:
     return _load().oracle_check_shape(N, H, W, C, heads, S, topk) == 0
+
+
+# ----------------------------------------------------------------------------- attention layer
+# The two steps either side of the path: the qkv projection before it (nn.Linear C -> 3C
+# with bias; q, k and v are consecutive C-wide chunks of its output, in that order) and
+# the output projection `wo` after it (nn.Linear C -> C with bias). Sources: "BiFormer ...
+# 前向传播过程" (niftyadmin), section "BRA模块" (the qkv projection split into q and kv, and
+# the closing linear layer after out + lepe) and section "网络结构" (the module printout:
+# qkv Linear(64 -> 192, bias=True), wo Linear(64 -> 64, bias=True)); Algorithm 1 as
+# described on bernice.tw chunks linear_qkv(x) into query, key, value the same way.
+# Between the steps every tensor is stored in the layer's dtype (a bf16 model keeps its
+# activations in bf16): q, k, v and the attention output are rounded to that dtype before
+# the next step reads them, as the CUDA path stores them.
+
+def round_to(x, dtype: str) -> np.ndarray:
+    """Round float64 values to the storage dtype, nearest with ties to even; float64 out.
+
+    "f32": IEEE single (numpy's conversion). "bf16": bfloat16 straight from the float64
+    value (one rounding): the 52-bit fraction is rounded to 7 bits. Valid for zero and for
+    finite magnitudes in bfloat16's normal range, which the function checks.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    if dtype == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if dtype != "bf16":
+        raise ValueError("dtype must be 'f32' or 'bf16'")
+    a = np.abs(x)
+    if not np.all(np.isfinite(x)) or np.any((a != 0) & ((a < 2.0 ** -126) | (a >= 3.3e38))):
+        raise ValueError("round_to bf16: value outside bfloat16's normal range")
+    u = x.view(np.uint64)
+    drop = np.uint64(45)
+    lsb = (u >> drop) & np.uint64(1)
+    r = (u + (np.uint64(1) << np.uint64(44)) - np.uint64(1) + lsb) & ~((np.uint64(1) << drop) - np.uint64(1))
+    return r.view(np.float64)
+
+
+def linear(x, w, b) -> np.ndarray:
+    """nn.Linear in float64: y = x w^T + b, x (..., K), w (Nout, K), b (Nout)."""
+    x, w, b = _d(x), _d(w), _d(b)
+    return x @ w.T + b
+
+
+def layer_forward(x, w_qkv, b_qkv, w_o, b_o, lce_w, lce_b, heads: int, S: int, topk: int, dtype: str,
+                  intermediates: bool = False):
+    """The attention layer around the path: out = wo(BRA(qkv(x))).
+
+    x (N,H,W,C); w_qkv (3C, C), b_qkv (3C); w_o (C, C), b_o (C); lce_w (C,5,5), lce_b (C).
+    Returns (out, r_idx, r_weight), plus {"q","k","v","o"} (the stored intermediates)
+    when `intermediates` is set. `out` is the float64 value before the final rounding.
+    """
+    x = _d(x)
+    N, H, W, C = x.shape
+    qkv = linear(x.reshape(-1, C), w_qkv, b_qkv)
+    q, k, v = (round_to(qkv[:, i * C:(i + 1) * C], dtype).reshape(N, H, W, C) for i in range(3))
+    o, r_idx, r_w = forward(q, k, v, lce_w, lce_b, heads, S, topk)
+    o = round_to(o, dtype)
+    out = linear(o.reshape(-1, C), w_o, b_o).reshape(N, H, W, C)
+    if intermediates:
+        return out, r_idx, r_w, {"q": q, "k": k, "v": v, "o": o}
+    return out, r_idx, r_w

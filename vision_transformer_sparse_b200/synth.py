@@ -23,6 +23,15 @@ Value recipe (stated once, used everywhere):
     (round-to-nearest-even) when the workload dtype is bf16.
 Seeds: workload c, tensor slot i -> seed 0xB1F0 + 16*c + i, with slots
 q=0, k=1, v=2, lce_w=3, lce_b=4, q/k/v region offsets = 5/6/7.
+
+Attention-layer inputs (make_layer_inputs: the qkv projection before the path and
+the output projection after it) draw the layer input x instead of q, k, v:
+  * x ~ N(0, 1), plus the same kind of per-(image, region, channel) offset for the
+    detection and segmentation workloads;
+  * qkv weight (3C, C) and output weight (C, C) ~ N(0, 1/C), so that q, k, v and the
+    layer output have unit scale; both biases ~ N(0, 0.02^2);
+  * LCE weight and bias as above; slots x=8, x offset=9, qkv weight/bias=10/11,
+    output weight/bias=12/13.
 """
 from __future__ import annotations
 
@@ -31,7 +40,8 @@ from typing import Dict, Optional
 
 import numpy as np
 
-SLOT = {"q": 0, "k": 1, "v": 2, "lce_w": 3, "lce_b": 4, "q_off": 5, "k_off": 6, "v_off": 7}
+SLOT = {"q": 0, "k": 1, "v": 2, "lce_w": 3, "lce_b": 4, "q_off": 5, "k_off": 6, "v_off": 7,
+        "x": 8, "x_off": 9, "w_qkv": 10, "b_qkv": 11, "w_o": 12, "b_o": 13}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -130,4 +140,31 @@ def make_inputs(w: Workload, seed_base: Optional[int] = None, batch: Optional[in
     else:
         b = np.zeros((w.C,))
     out["lce_b"] = _store(b, w.dtype)
+    return out
+
+
+def make_layer_inputs(w: Workload, seed_base: Optional[int] = None, batch: Optional[int] = None
+                      ) -> Dict[str, np.ndarray]:
+    """Return x (N,H,W,C), w_qkv (3C,C), b_qkv (3C), w_o (C,C), b_o (C), lce_w, lce_b.
+
+    float32 arrays whose values are exactly representable in the workload dtype.
+    """
+    N = w.N if batch is None else batch
+    shape = (N, w.H, w.W, w.C)
+    hr, wr = w.H // w.S, w.W // w.S
+    x = _rng(w, "x", seed_base).standard_normal(shape)
+    if w.region_bias > 0:
+        off = _rng(w, "x_off", seed_base).standard_normal((N, w.S, 1, w.S, 1, w.C)) * w.region_bias
+        x = (x.reshape(N, w.S, hr, w.S, wr, w.C) + off).reshape(shape)
+    g = 1.0 / np.sqrt(w.C)
+    out = {
+        "x": _store(x, w.dtype),
+        "w_qkv": _store(_rng(w, "w_qkv", seed_base).standard_normal((3 * w.C, w.C)) * g, w.dtype),
+        "b_qkv": _store(_rng(w, "b_qkv", seed_base).standard_normal((3 * w.C,)) * 0.02, w.dtype),
+        "w_o": _store(_rng(w, "w_o", seed_base).standard_normal((w.C, w.C)) * g, w.dtype),
+        "b_o": _store(_rng(w, "b_o", seed_base).standard_normal((w.C,)) * 0.02, w.dtype),
+    }
+    base = make_inputs(w, seed_base, batch)
+    out["lce_w"] = base["lce_w"]
+    out["lce_b"] = base["lce_b"]
     return out
