@@ -20,6 +20,11 @@ the tokens of all ranks over the slowest rank's time.
 
 --impl reference times the float64 CPU oracle on this host's cores (the only
 reference this method has): each step is a bounded sample of the same workload.
+
+--layer times the attention layer around BRA instead (bra_attention_layer: the qkv
+projection, the BRA forward, the output projection) on the same workload shape, with
+the layer's seeded inputs (x and the two projections' weights); its line carries its
+own metric name.
 """
 from __future__ import annotations
 
@@ -42,6 +47,7 @@ from vision_transformer_sparse_b200 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "BRA fwd tokens/s and TFLOP/s at 1 B200; % of bf16 tensor/HBM roofline"
+METRIC_LAYER = "BRA attention layer fwd (qkv projection + BRA + output projection) tokens/s at 1 B200"
 
 
 def parse():
@@ -54,6 +60,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each step directly")
+    ap.add_argument("--layer", action="store_true",
+                    help="time the whole attention layer (bra_attention_layer) instead of the BRA forward")
     ap.add_argument("--variant", default="auto", choices=["auto", "generic", "tma", "split", "pipe"],
                     help="attention kernel (auto: persistent TMA pipeline where the shape allows)")
     ap.add_argument("--source-hash", metavar="KERNEL",
@@ -78,9 +86,14 @@ def algorithmic(w: synth.Workload):
     # the one-kernel forward: q, k, v read once, out written once, r_idx and r_weight,
     # the LCE parameters
     fused_bytes = 4.0 * T * w.C * b + route_bytes + w.C * 26 * b
+    # the projections (attention layer): qkv reads x and its weight and writes q, k, v;
+    # wo reads the attention output and its weight and writes out. Per launch, averaged
+    # over the two launches of a layer forward.
+    lin_bytes = (4.0 * T * w.C * b + 3 * w.C * w.C * b + 2.0 * T * w.C * b + w.C * w.C * b) / 2
+    lin_flops = 8.0 * T * w.C * w.C
     return {"tokens": T, "flops": flops, "gathered_bytes": gathered, "attn_bytes": attn_unique,
             "pool_bytes": pool_bytes, "route_bytes": route_bytes, "fused_bytes": fused_bytes,
-            "elem_bytes": b}
+            "linear_bytes": lin_bytes, "linear_flops": lin_flops, "elem_bytes": b}
 
 
 def load_peaks():
@@ -104,6 +117,8 @@ KERNEL_HEADERS = {
     "attn_f32_kernel": ["attn.cuh"],
     "region_mean_kernel": ["route.cuh"],
     "route_kernel": ["route.cuh"],
+    "linear_umma_kernel": ["linear.cuh"],
+    "linear_f32_kernel": ["linear.cuh"],
 }
 
 
@@ -230,16 +245,24 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- reference arm
 
+def oracle_step(w: synth.Workload, sample: synth.Workload, layer: bool):
+    """One call of the oracle on `sample` (the BRA forward, or the whole layer)."""
+    import oracle
+    if layer:
+        inp = {k: v.astype(np.float64) for k, v in synth.make_layer_inputs(sample).items()}
+        keys = ("x", "w_qkv", "b_qkv", "w_o", "b_o", "lce_w", "lce_b")
+        return lambda: oracle.layer_forward(*(inp[k] for k in keys), w.heads, w.S, w.topk, w.dtype)
+    inp = {k: v.astype(np.float64) for k, v in synth.make_inputs(sample).items()}
+    return lambda: oracle.forward(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], w.heads, w.S, w.topk)
+
+
 def bench_reference(args, w: synth.Workload, rank: int):
     """The float64 CPU oracle on this host's cores; each step one image of the workload."""
     import oracle
     if rank != 0:
         return None
     sample = w.with_(N=1)
-    inp = {k: v.astype(np.float64) for k, v in synth.make_inputs(sample).items()}
-
-    def step():
-        oracle.forward(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], w.heads, w.S, w.topk)
+    step = oracle_step(w, sample, args.layer)
 
     for _ in range(args.warmup):
         step()
@@ -250,7 +273,7 @@ def bench_reference(args, w: synth.Workload, rank: int):
     value = sample.tokens * args.steps / dt
     cores = oracle.threads()
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
+        "impl": "reference", "metric": METRIC_LAYER if args.layer else METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1), BiFormer stage shape)",
@@ -263,21 +286,22 @@ def bench_reference(args, w: synth.Workload, rank: int):
     return line
 
 
-def cpu_baseline(w: synth.Workload, budget_s: float = 12.0):
+def cpu_baseline(w: synth.Workload, budget_s: float = 12.0, layer: bool = False):
     """The oracle as it stands on a bounded sample: whole images (at most 8), repeated
     until about `budget_s` seconds of host time are used (at least once)."""
     import oracle
     sample = w.with_(N=max(1, min(w.N, 8)))
-    inp = {k: v.astype(np.float64) for k, v in synth.make_inputs(sample).items()}
+    step = oracle_step(w, sample, layer)
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.forward(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], w.heads, w.S, w.topk)
+        step()
         reps += 1
         dt = time.perf_counter() - t0
         if dt > budget_s:
             break
     return {"value": sample.tokens * reps / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": "%d x forward of %d images (%d tokens), %.1f s" % (reps, sample.N, sample.tokens, dt)}
+            "sample": "%d x %s of %d images (%d tokens), %.1f s" % (reps, "layer" if layer else "forward",
+                                                                   sample.N, sample.tokens, dt)}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -322,15 +346,19 @@ def main():
 
     # inputs: this rank's own batch (weak scaling); seeded per rank
     seed = None if rank == 0 else 0xB1F0 + 16 * w.index + 1000 * rank
-    inp = synth.make_inputs(w, seed_base=seed)
+    layer = args.layer
+    inp = synth.make_layer_inputs(w, seed_base=seed) if layer else synth.make_inputs(w, seed_base=seed)
     base = {k: torch.from_numpy(v).to(dev).to(tdt).contiguous() for k, v in inp.items()}
-    set_bytes = 4 * w.tokens * w.C * acc["elem_bytes"]
+    lead = "x" if layer else "q"  # the (N,H,W,C) input whose shape the output takes
+    # bytes of one input set plus its output (the layer's q, k, v and attention output
+    # are the library's scratch, produced and consumed inside the step)
+    set_bytes = (2 if layer else 4) * w.tokens * w.C * acc["elem_bytes"]
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     n_sets = max(2, math.ceil(3 * l2 / set_bytes))
     sets = []
     for _ in range(n_sets):
         s = {k: v.clone() for k, v in base.items()}
-        s["out"] = torch.empty_like(base["q"])
+        s["out"] = torch.empty_like(base[lead])
         s["r_idx"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.int32, device=dev)
         s["r_w"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.float32, device=dev)
         sets.append(s)
@@ -338,8 +366,13 @@ def main():
     stream = torch.cuda.Stream(device=dev)
 
     def fwd(s):
-        bra.forward(s["q"], s["k"], s["v"], s["lce_w"], s["lce_b"], w.heads, w.S, w.topk,
-                    out=s["out"], r_idx=s["r_idx"], r_weight=s["r_w"], stream=stream)
+        if layer:
+            bra.attention_layer(s["x"], s["w_qkv"], s["b_qkv"], s["w_o"], s["b_o"], s["lce_w"], s["lce_b"],
+                                w.heads, w.S, w.topk, out=s["out"], r_idx=s["r_idx"], r_weight=s["r_w"],
+                                stream=stream)
+        else:
+            bra.forward(s["q"], s["k"], s["v"], s["lce_w"], s["lce_b"], w.heads, w.S, w.topk,
+                        out=s["out"], r_idx=s["r_idx"], r_weight=s["r_w"], stream=stream)
 
     # one CUDA graph per input set
     graphs = []
@@ -421,15 +454,28 @@ def main():
     traced_steps = rounds * n_sets
     clocks.stop()
 
-    # ---- end to end through the host-buffer entry point (pinned host memory)
+    # ---- end to end through the public API from pinned host memory: the host-buffer
+    # entry point for the forward; for the layer, copies on the stream around the
+    # device call
     host = {k: v.cpu().pin_memory() for k, v in base.items()}
-    h_out = torch.empty_like(host["q"]).pin_memory()
+    h_out = torch.empty_like(host[lead]).pin_memory()
     h_idx = torch.empty((w.N, w.regions, w.topk), dtype=torch.int32).pin_memory()
     h_w = torch.empty((w.N, w.regions, w.topk), dtype=torch.float32).pin_memory()
+    d_in = sets[0]
 
     def e2e_step():
-        bra.forward_host(host["q"], host["k"], host["v"], host["lce_w"], host["lce_b"], w.heads, w.S, w.topk,
-                         out=h_out, r_idx=h_idx, r_weight=h_w, stream=stream)
+        if layer:
+            with torch.cuda.stream(stream):
+                for k_, v_ in host.items():
+                    d_in[k_].copy_(v_, non_blocking=True)
+                fwd(d_in)
+                h_out.copy_(d_in["out"], non_blocking=True)
+                h_idx.copy_(d_in["r_idx"], non_blocking=True)
+                h_w.copy_(d_in["r_w"], non_blocking=True)
+            stream.synchronize()
+        else:
+            bra.forward_host(host["q"], host["k"], host["v"], host["lce_w"], host["lce_b"], w.heads, w.S, w.topk,
+                             out=h_out, r_idx=h_idx, r_weight=h_w, stream=stream)
 
     for _ in range(3):
         e2e_step()
@@ -466,7 +512,8 @@ def main():
     t_ms, t_n = trace[attn_name]
     attn_s = t_ms / max(t_n, 1) / 1e3
     alg_bytes = {"bra_image_kernel": acc["fused_bytes"], "region_mean_kernel": acc["pool_bytes"],
-                 "route_kernel": acc["route_bytes"]}.get(attn_name, acc["attn_bytes"])
+                 "route_kernel": acc["route_bytes"], "linear_umma_kernel": acc["linear_bytes"],
+                 "linear_f32_kernel": acc["linear_bytes"]}.get(attn_name, acc["attn_bytes"])
     step_traced_ms = sum(v[0] for v in trace.values()) / traced_steps
     share = {k: round(v[0] / max(1e-12, sum(x[0] for x in trace.values())), 4) for k, v in trace.items() if v[1]}
     achieved = alg_bytes / attn_s / 1e9
@@ -477,7 +524,8 @@ def main():
     t_gath = acc["gathered_bytes"] / (peaks["hbm_gbs"] * 1e9)
     ns_bound = "tensor" if t_flop > t_gath else "hbm"
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_LAYER if layer else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1), BiFormer stage shape; no dataset)",
@@ -487,6 +535,8 @@ def main():
                          % (n_sets, set_bytes / 1e6, n_sets * set_bytes / 1e6, l2 / 1e6),
                    "launch": "CUDA graph per step" if graphs else "direct launches",
                    "attention_kernel": args.variant,
+                   "step": "bra_attention_layer (qkv projection, BRA, output projection)" if layer
+                           else "bra_forward",
                    "parallelism": "dp%d (independent images, no collective)" % world},
         "tflops": tflops,
         "gpu_launches": gpu_launches,
@@ -505,10 +555,11 @@ def main():
         "clocks": clocks.summary(),
         "e2e": {"value": tokens_all * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-                "entry": "bra_forward_host (pinned host buffers)"},
+                "entry": "bra_attention_layer with stream copies (pinned host buffers)" if layer
+                         else "bra_forward_host (pinned host buffers)"},
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(w, layer=layer)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -145,6 +145,41 @@ int bra_forward_noalloc(const void *q, const void *k, const void *v, const void 
                         bra_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * The attention layer around BRA: the qkv projection before it and the output
+ * projection `wo` after it, both nn.Linear modules with bias (y = x w^T + b), as
+ * printed in the walk-through's module listing ("BiFormer ... 前向传播过程",
+ * section "网络结构": qkv Linear(64 -> 192, bias=True), wo Linear(64 -> 64,
+ * bias=True)) and used in its section "BRA模块" (q, k, v are consecutive C-wide
+ * chunks of the qkv output; a linear layer closes the block).
+ *
+ * Conventions (besides those above): x, y, q, k, v, out are row-major with one row
+ * per token ((N,H,W,C) maps are (N*H*W) x C matrices); a weight w is (Nout, K)
+ * row-major (the PyTorch Linear weight) and a bias b is (Nout); all in `dtype`.
+ * The products accumulate in float32 (bfloat16 tensor-core products for BRA_BF16,
+ * float32 FMA for BRA_F32); the bias is added in float32 and every stored value is
+ * rounded once to `dtype` (round to nearest even). Supported: 1 <= K, Nout <= 4096;
+ * for BRA_BF16 also K % 32 == 0 and Nout (each third of it for bra_qkv) a multiple
+ * of 32. x, w and the outputs 16-byte aligned; biases aligned to their element. */
+
+/* y (M x Nout) = x (M x K) w^T + b. M may be 0 (nothing is launched). */
+int bra_linear(const void *x, const void *w, const void *b, int M, int K, int Nout, int dtype, void *y,
+               bra_stream_t stream);
+
+/* The qkv projection: [q | k | v] = x w_qkv^T + b_qkv with x (M x C), w_qkv (3C, C),
+ * b_qkv (3C); q, k, v (M x C) each get their C-wide chunk, in that order. */
+int bra_qkv(const void *x, const void *w_qkv, const void *b_qkv, int M, int C, int dtype, void *q, void *k,
+            void *v, bra_stream_t stream);
+
+/* The whole layer: out = wo(BRA(qkv(x))) with x, out (N,H,W,C); q, k, v and the
+ * attention output are stored in `dtype` between the steps (scratch of 4*N*H*W*C
+ * elements taken stream-ordered from the default memory pool, besides the routing
+ * scratch of bra_forward). r_idx and r_weight as in bra_forward. BRA's shape rules
+ * apply, plus those of the projections with K = C. */
+int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, const void *w_o, const void *b_o,
+                        const void *lce_w, const void *lce_b, int N, int H, int W, int C, int heads, int S,
+                        int topk, int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Tracing (measurement support; no part of the computation).
  *
  * Kernel classes the library launches, for bra_trace_end and bra_kernel_name. */
@@ -155,7 +190,9 @@ enum {
     BRA_KERNEL_ATTN_F32 = 3,    /* steps 4-5, float32 SIMT kernel                 */
     BRA_KERNEL_FUSED_IMAGE = 4, /* steps 1-5 in one kernel (small images)         */
     BRA_KERNEL_ATTN_UMMA = 5,   /* steps 4-5, tcgen05 kernel (large regions)       */
-    BRA_KERNEL_CLASSES = 6
+    BRA_KERNEL_LINEAR_BF16 = 6, /* qkv / output projection, tcgen05 GEMM          */
+    BRA_KERNEL_LINEAR_F32 = 7,  /* qkv / output projection, float32 SIMT          */
+    BRA_KERNEL_CLASSES = 8
 };
 
 /* Number of kernels this library has launched since it was loaded (all threads,

@@ -82,3 +82,70 @@ def test_empty_batch_is_a_no_op(bra_lib):
     shape = (0, 56, 56, 64, 2, 7, 1, 1)
     assert fwd(shape, [None] * 8) == 0
     assert bra.raw_call("bra_route", None, None, *shape, None, None, None) == 0
+
+
+# ---------------------------------------------------------------- projections and the layer
+
+def lin(M, K, Nout, dtype, x=FAKE, w=FAKE, b=FAKE, y=FAKE):
+    return bra.raw_call("bra_linear", x, w, b, M, K, Nout, dtype, y, None)
+
+
+@pytest.mark.parametrize("M,K,Nout,dtype,code", [
+    (10, 64, 64, 7, 4),       # dtype
+    (-1, 64, 64, 1, 2),       # M < 0
+    (10, 0, 64, 1, 2),        # K = 0
+    (10, 48, 64, 1, 2),       # bf16 K not a multiple of 32
+    (10, 64, 48, 1, 2),       # bf16 Nout not a multiple of 32
+    (10, 8192, 64, 1, 2),     # K above 4096
+    (10, 64, 8192, 0, 2),     # Nout above 4096
+])
+def test_linear_bad_shapes_rejected(bra_lib, M, K, Nout, dtype, code):
+    assert lin(M, K, Nout, dtype) == code
+
+
+def test_linear_nulls_alignment_and_empty(bra_lib):
+    for i in range(4):
+        ptrs = [FAKE] * 4
+        ptrs[i] = None
+        assert lin(10, 64, 64, 1, *ptrs) == 1
+    for i in (0, 1, 3):   # x, w, y need 16 bytes
+        ptrs = [FAKE] * 4
+        ptrs[i] = ODD
+        assert lin(10, 64, 64, 1, *ptrs) == 3
+    assert lin(10, 64, 64, 1, b=ctypes.c_void_p(0x10001)) == 3   # bias aligned to its element
+    assert lin(0, 64, 64, 1, None, None, None, None) == 0        # nothing to do
+    assert lin(0, 48, 40, 0, None, None, None, None) == 0        # float32 takes any K, Nout
+
+
+def test_qkv_rejects_before_cuda(bra_lib):
+    call = lambda M, C, dt, *p: bra.raw_call("bra_qkv", *(p[:3] if p else [FAKE] * 3), M, C, dt,
+                                             *(p[3:] if p else [FAKE] * 3), None)
+    assert call(10, 48, 1) == 2          # each third must be a multiple of 32 in bf16
+    assert call(10, 2000, 1) == 2        # 3C above 4096
+    assert call(10, 64, 9) == 4
+    assert call(10, 64, 1, FAKE, FAKE, FAKE, FAKE, None, FAKE) == 1
+    assert call(10, 64, 1, FAKE, FAKE, FAKE, FAKE, FAKE, ODD) == 3
+    assert call(0, 64, 1, None, None, None, None, None, None) == 0
+
+
+@pytest.mark.parametrize("shape,code", [
+    ((1, 57, 56, 64, 2, 7, 1, 1), 2),    # H % S
+    ((1, 56, 56, 96, 2, 7, 1, 1), 2),    # d = 48
+    ((1, 56, 56, 64, 2, 7, 50, 1), 2),   # topk > S^2
+    ((1, 56, 56, 64, 2, 7, 1, 7), 4),    # dtype
+])
+def test_layer_bad_shapes_rejected(bra_lib, shape, code):
+    assert bra.raw_call("bra_attention_layer", *[FAKE] * 7, *shape, *[FAKE] * 3, None) == code
+
+
+def test_layer_nulls_and_alignment(bra_lib):
+    shape = (1, 56, 56, 64, 2, 7, 1, 1)
+    for i in range(10):
+        ptrs = [FAKE] * 10
+        ptrs[i] = None
+        assert bra.raw_call("bra_attention_layer", *ptrs[:7], *shape, *ptrs[7:], None) == 1
+    for i in (0, 1, 3, 7):   # x, w_qkv, w_o, out need 16 bytes
+        ptrs = [FAKE] * 10
+        ptrs[i] = ODD
+        assert bra.raw_call("bra_attention_layer", *ptrs[:7], *shape, *ptrs[7:], None) == 3
+    assert bra.raw_call("bra_attention_layer", *[None] * 7, 0, 56, 56, 64, 2, 7, 1, 1, *[None] * 3, None) == 0

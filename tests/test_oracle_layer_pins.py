@@ -224,3 +224,23 @@ def test_workload_layer_inputs_shapes_and_scale():
         a = mid[name].astype(np.float32)
         np.testing.assert_array_equal(a, synth.round_bf16(a))
         assert np.array_equal(a.astype(np.float64), mid[name])
+
+
+def test_layer_checker_accepts_the_oracle_and_rejects_a_kv_swap():
+    """The GPU tests' layer check passes the oracle's own (rounded) result and fails a
+    result computed with the k and v chunks of the projection swapped."""
+    from oracle import compare
+    w = synth.Workload("checker", 50, 1, 14, 14, 64, 2, 7, 4, "bf16", lce_b_std=0.01)
+    inp = synth.make_layer_inputs(w)
+    args = (w.heads, w.S, w.topk, w.dtype)
+    keys = ("x", "w_qkv", "b_qkv", "w_o", "b_o", "lce_w", "lce_b")
+    out, r_idx, r_w = oracle.layer_forward(*(inp[k] for k in keys), *args)
+    rep = compare.check_layer(inp, *args[:3], w.dtype, oracle.round_to(out, "bf16"), r_idx, r_w.astype(np.float32))
+    assert rep.ok, rep.notes
+    C = w.C
+    bad = dict(inp)
+    bad["w_qkv"] = np.vstack([inp["w_qkv"][:C], inp["w_qkv"][2 * C:], inp["w_qkv"][C:2 * C]])
+    bad["b_qkv"] = np.concatenate([inp["b_qkv"][:C], inp["b_qkv"][2 * C:], inp["b_qkv"][C:2 * C]])
+    out2, idx2, w2 = oracle.layer_forward(*(bad[k] for k in keys), *args)
+    rep2 = compare.check_layer(inp, *args[:3], w.dtype, oracle.round_to(out2, "bf16"), idx2, w2.astype(np.float32))
+    assert not rep2.ok

@@ -26,8 +26,9 @@ STATIC_SCRATCH_FLOATS = 4 * 1024 * 1024
 SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
            "bra_status_string",
            "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name",
-           "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout", "bra_trace_read")
-KERNEL_CLASSES = 6
+           "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout", "bra_trace_read",
+           "bra_linear", "bra_qkv", "bra_attention_layer")
+KERNEL_CLASSES = 8
 
 
 class BraError(RuntimeError):
@@ -50,8 +51,11 @@ def lib() -> ctypes.CDLL:
         L.bra_attend.argtypes = [vp] * 5 + shape + [vp, vp, vp]
         L.bra_forward_host.argtypes = [vp] * 5 + shape + [vp, vp, vp, vp]
         L.bra_forward_noalloc.argtypes = [vp] * 5 + shape + [vp, vp, vp, vp]
+        L.bra_linear.argtypes = [vp] * 3 + [i] * 4 + [vp, vp]
+        L.bra_qkv.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
+        L.bra_attention_layer.argtypes = [vp] * 7 + shape + [vp, vp, vp, vp]
         for f in ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
-                  "bra_version"):
+                  "bra_version", "bra_linear", "bra_qkv", "bra_attention_layer"):
             getattr(L, f).restype = i
         L.bra_status_string.argtypes = [i]
         L.bra_status_string.restype = ctypes.c_char_p
@@ -117,6 +121,46 @@ def forward(q, k, v, lce_w, lce_b, heads: int, S: int, topk: int, out=None, r_id
     rc = lib().bra_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(lce_b), N, H, W, C, heads, S, topk,
                            _dtype_code(q), _ptr(out), _ptr(r_idx), _ptr(r_weight), _stream(stream))
     _raise(rc, "bra_forward")
+    return out, r_idx, r_weight
+
+
+def linear(x, w, b, out=None, stream=None) -> torch.Tensor:
+    """bra_linear: x (..., K) rows, w (Nout, K), b (Nout) -> x w^T + b, shape (..., Nout)."""
+    K = x.shape[-1]
+    Nout = w.shape[0]
+    M = x.numel() // K if K else 0
+    out = torch.empty(x.shape[:-1] + (Nout,), dtype=x.dtype, device=x.device) if out is None else out
+    _check_dev(x, w, b, out)
+    rc = lib().bra_linear(_ptr(x), _ptr(w), _ptr(b), M, K, Nout, _dtype_code(x), _ptr(out), _stream(stream))
+    _raise(rc, "bra_linear")
+    return out
+
+
+def qkv(x, w_qkv, b_qkv, q=None, k=None, v=None, stream=None):
+    """bra_qkv: x (..., C), w_qkv (3C, C), b_qkv (3C) -> q, k, v, each of x's shape."""
+    C = x.shape[-1]
+    M = x.numel() // C if C else 0
+    q, k, v = (torch.empty_like(x) if t is None else t for t in (q, k, v))
+    _check_dev(x, w_qkv, b_qkv, q, k, v)
+    rc = lib().bra_qkv(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), M, C, _dtype_code(x), _ptr(q), _ptr(k), _ptr(v),
+                       _stream(stream))
+    _raise(rc, "bra_qkv")
+    return q, k, v
+
+
+def attention_layer(x, w_qkv, b_qkv, w_o, b_o, lce_w, lce_b, heads: int, S: int, topk: int, out=None,
+                    r_idx=None, r_weight=None, stream=None):
+    """bra_attention_layer: out = wo(BRA(qkv(x))) for x (N,H,W,C) -> out, r_idx, r_weight."""
+    N, H, W, C = x.shape
+    P = S * S
+    out = torch.empty_like(x) if out is None else out
+    r_idx = torch.empty((N, P, topk), dtype=torch.int32, device=x.device) if r_idx is None else r_idx
+    r_weight = torch.empty((N, P, topk), dtype=torch.float32, device=x.device) if r_weight is None else r_weight
+    _check_dev(x, w_qkv, b_qkv, w_o, b_o, lce_w, lce_b, out, r_idx, r_weight)
+    rc = lib().bra_attention_layer(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(w_o), _ptr(b_o), _ptr(lce_w),
+                                   _ptr(lce_b), N, H, W, C, heads, S, topk, _dtype_code(x), _ptr(out),
+                                   _ptr(r_idx), _ptr(r_weight), _stream(stream))
+    _raise(rc, "bra_attention_layer")
     return out, r_idx, r_weight
 
 

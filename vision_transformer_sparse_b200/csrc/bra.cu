@@ -33,6 +33,7 @@
 #include "attn_tma.cuh"
 #include "attn_umma.cuh"
 #include "fused_image.cuh"
+#include "linear.cuh"
 #include "route.cuh"
 
 namespace bra {
@@ -858,6 +859,97 @@ static int launch_fused_image(const Shape &s, bool routed, const void *q, const 
     return cudaLaunchKernelEx(&cfg, kern, p) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
 }
 
+// ----------------------------------------------------------------------------- projections
+
+// 2-D bfloat16 map of a row-major (rows x cols) matrix: boxes of 32 columns x box_rows
+// rows, 64-byte swizzle (the MMA operand layout), zero fill past the last row.
+static bool encode_map_rows(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {32u, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output columns per tile: the largest power of two in [32, 256] dividing ny (so that a
+// tile never straddles two output buffers), 0 if none.
+static int linear_tile_n(int ny) {
+    for (int b = 256; b >= 32; b >>= 1)
+        if (ny % b == 0) return b;
+    return 0;
+}
+
+// Shapes the projections take (checked before any CUDA call): y (M x Nout) = x (M x K)
+// w^T + b, output split into nsplit buffers of Nout / nsplit columns.
+static int check_linear(int M, int K, int Nout, int nsplit, int dtype) {
+    if (dtype != BRA_F32 && dtype != BRA_BF16) return BRA_ERR_DTYPE;
+    if (M < 0 || K <= 0 || Nout <= 0 || nsplit < 1 || nsplit > 3 || Nout % nsplit) return BRA_ERR_SHAPE;
+    if (K > 4096 || Nout > 4096) return BRA_ERR_SHAPE;
+    if (dtype == BRA_BF16 && (K % 32 || linear_tile_n(Nout / nsplit) == 0)) return BRA_ERR_SHAPE;
+    return BRA_OK;
+}
+
+// y[i] (M x Nout/nsplit, row-major) = column block i of x w^T + b.
+static int launch_linear(const void *x, const void *w, const void *b, int M, int K, int Nout, int nsplit,
+                         void *const *y, int dtype, cudaStream_t st) {
+    if (M == 0) return BRA_OK;
+    const int ny = Nout / nsplit;
+    if (dtype == BRA_F32) {
+        LinearF32Params p;
+        p.x = static_cast<const float *>(x);
+        p.w = static_cast<const float *>(w);
+        p.b = static_cast<const float *>(b);
+        for (int i = 0; i < 3; ++i) p.y[i] = static_cast<float *>(y[i < nsplit ? i : 0]);
+        p.M = M;
+        p.K = K;
+        p.Nout = Nout;
+        p.Ny = ny;
+        const dim3 grid((Nout + 63) / 64, (unsigned)std::min((M + 63) / 64, 65535));
+        LaunchScope ls(BRA_KERNEL_LINEAR_F32, st);
+        linear_f32_kernel<<<grid, 256, 0, st>>>(p);
+        return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+    }
+    LinearParams p;
+    memset(&p, 0, sizeof(p));
+    p.BN = linear_tile_n(ny);
+    if (!encode_map_rows(&p.tmX, x, M, K, kLinRows) || !encode_map_rows(&p.tmW, w, Nout, K, p.BN)) return BRA_ERR_CUDA;
+    p.bias = static_cast<const __nv_bfloat16 *>(b);
+    for (int i = 0; i < 3; ++i) p.y[i] = static_cast<__nv_bfloat16 *>(y[i < nsplit ? i : 0]);
+    p.M = M;
+    p.K = K;
+    p.Nout = Nout;
+    p.Ny = ny;
+    p.tiles_n = Nout / p.BN;
+    p.tiles = (M + kLinRows - 1) / kLinRows * p.tiles_n;
+    p.tmem_cols = 32;
+    while (p.tmem_cols < (uint32_t)(2 * p.BN)) p.tmem_cols <<= 1;
+    p.wait_limit = kWaitLimit;
+    // CTAs per SM are held to what the tensor memory takes (an allocation beyond its 512
+    // columns would wait for a resident CTA to finish): each CTA asks for enough shared
+    // memory that one more would not fit.
+    const int max_ctas = 512 / (int)p.tmem_cols;
+    constexpr int kSmPerSmBytes = 228 * 1024, kCtaReserve = 1024;
+    p.stages = 4;
+    int smem = linear_smem_layout(p.BN, p.stages, Nout).total;
+    smem = std::max(smem, kSmPerSmBytes / (max_ctas + 1) - kCtaReserve + 16);
+    if (smem > kMaxSmem) return BRA_ERR_SHAPE;
+    if (allow_smem(linear_umma_kernel, smem) != cudaSuccess) return BRA_ERR_CUDA;
+    int per_sm = 0, sms = 0;
+    if (occupancy(&per_sm, linear_umma_kernel, kLinThreads, smem, 0, nullptr) != cudaSuccess || per_sm < 1 ||
+        per_sm > max_ctas)
+        return BRA_ERR_CUDA;
+    int rc = sm_count(&sms);
+    if (rc) return rc;
+    const int grid = std::min(p.tiles, sms * per_sm);
+    LaunchScope ls(BRA_KERNEL_LINEAR_BF16, st);
+    linear_umma_kernel<<<grid, kLinThreads, smem, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
 // Everything a shape must pass before any CUDA call is made.
 static int check_plan(const Shape &s) {
     int rc = check_shape(s);
@@ -958,6 +1050,8 @@ const char *bra_kernel_name(int kernel_class) {
         case BRA_KERNEL_ATTN_F32: return "attn_f32_kernel";
         case BRA_KERNEL_FUSED_IMAGE: return "bra_image_kernel";
         case BRA_KERNEL_ATTN_UMMA: return "attn_umma_kernel";
+        case BRA_KERNEL_LINEAR_BF16: return "linear_umma_kernel";
+        case BRA_KERNEL_LINEAR_F32: return "linear_f32_kernel";
         default: return "unknown";
     }
 }
@@ -1033,6 +1127,63 @@ int bra_forward(const void *q, const void *k, const void *v, const void *lce_w, 
     const size_t es = dtype == BRA_BF16 ? 2 : 4;
     if (!aligned(lce_w, es) || !aligned(lce_b, es)) return BRA_ERR_ALIGN;
     return forward_device(s, q, k, v, lce_w, lce_b, out, r_idx, r_weight, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bra_linear(const void *x, const void *w, const void *b, int M, int K, int Nout, int dtype, void *y,
+               bra_stream_t stream) {
+    int rc = check_linear(M, K, Nout, 1, dtype);
+    if (rc) return rc;
+    if (M == 0) return BRA_OK;
+    if (!x || !w || !b || !y) return BRA_ERR_NULL;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 16) || !aligned(b, es)) return BRA_ERR_ALIGN;
+    void *ys[1] = {y};
+    return launch_linear(x, w, b, M, K, Nout, 1, ys, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bra_qkv(const void *x, const void *w_qkv, const void *b_qkv, int M, int C, int dtype, void *q, void *k,
+            void *v, bra_stream_t stream) {
+    if (C <= 0 || C > 4096 / 3) return dtype == BRA_F32 || dtype == BRA_BF16 ? BRA_ERR_SHAPE : BRA_ERR_DTYPE;
+    int rc = check_linear(M, C, 3 * C, 3, dtype);
+    if (rc) return rc;
+    if (M == 0) return BRA_OK;
+    if (!x || !w_qkv || !b_qkv || !q || !k || !v) return BRA_ERR_NULL;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(b_qkv, es))
+        return BRA_ERR_ALIGN;
+    void *ys[3] = {q, k, v};
+    return launch_linear(x, w_qkv, b_qkv, M, C, 3 * C, 3, ys, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, const void *w_o, const void *b_o,
+                        const void *lce_w, const void *lce_b, int N, int H, int W, int C, int heads, int S,
+                        int topk, int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream) {
+    const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
+    int rc = check_plan(s);
+    if (rc) return rc;
+    const long long T = (long long)N * H * W;
+    if (T > INT_MAX) return BRA_ERR_SHAPE;
+    if ((rc = check_linear((int)T, C, 3 * C, 3, dtype)) || (rc = check_linear((int)T, C, C, 1, dtype))) return rc;
+    if (N == 0) return BRA_OK;
+    if (!x || !w_qkv || !b_qkv || !w_o || !b_o || !lce_w || !lce_b || !out || !r_idx || !r_weight)
+        return BRA_ERR_NULL;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(w_o, 16) || !aligned(out, 16) || !aligned(b_qkv, es) ||
+        !aligned(b_o, es) || !aligned(lce_w, es) || !aligned(lce_b, es) || !aligned(r_idx, 4) ||
+        !aligned(r_weight, 4))
+        return BRA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t plane = ((size_t)T * C * es + 255) / 256 * 256;  // one (N,H,W,C) tensor
+    unsigned char *buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&buf), 4 * plane, st) != cudaSuccess) return BRA_ERR_CUDA;
+    void *qkv[3] = {buf, buf + plane, buf + 2 * plane};
+    void *o = buf + 3 * plane;
+    rc = launch_linear(x, w_qkv, b_qkv, (int)T, C, 3 * C, 3, qkv, dtype, st);
+    if (rc == BRA_OK) rc = forward_device(s, qkv[0], qkv[1], qkv[2], lce_w, lce_b, o, r_idx, r_weight, st);
+    if (rc == BRA_OK) rc = launch_linear(o, w_o, b_o, (int)T, C, C, 1, &out, dtype, st);
+    if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    return rc;
 }
 
 int bra_attend(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b, int N,
