@@ -171,10 +171,12 @@ int bra_qkv(const void *x, const void *w_qkv, const void *b_qkv, int M, int C, i
             void *v, bra_stream_t stream);
 
 /* The whole layer: out = wo(BRA(qkv(x))) with x, out (N,H,W,C); q, k, v and the
- * attention output are stored in `dtype` between the steps (scratch of 4*N*H*W*C
- * elements taken stream-ordered from the default memory pool, besides the routing
- * scratch of bra_forward). r_idx and r_weight as in bra_forward. BRA's shape rules
- * apply, plus those of the projections with K = C. */
+ * attention output are stored in `dtype` between the steps. Scratch (4*N*H*W*C
+ * elements plus the routing's 2*N*S*S*C floats) is taken stream-ordered: outside a
+ * stream capture from the library's per-device pool that keeps its memory between
+ * calls (the pool of bra_forward_host), inside a capture from the device's default
+ * pool (a memory node of the graph). r_idx and r_weight as in bra_forward. BRA's
+ * shape rules apply, plus those of the projections with K = C. */
 int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, const void *w_o, const void *b_o,
                         const void *lce_w, const void *lce_b, int N, int H, int W, int C, int heads, int S,
                         int topk, int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream);

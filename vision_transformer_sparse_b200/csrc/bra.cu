@@ -20,6 +20,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <set>
 #include <tuple>
 #include <type_traits>
 #include <utility>
@@ -186,6 +187,21 @@ template <typename K> static cudaError_t allow_smem(K kern, int bytes) {
     if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess) g_smem_set[key] = bytes;
+    return e;
+}
+
+// Ask for the largest shared-memory carveout for `kern` on the current device, so that
+// the occupancy reported (and reached) counts every CTA the shared memory can hold.
+static std::set<std::pair<int, const void *>> g_carveout;
+template <typename K> static cudaError_t prefer_shared(K kern) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_pair(dev, reinterpret_cast<const void *>(kern));
+    std::lock_guard<std::mutex> g(g_facts_mu);
+    if (g_carveout.count(key)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess) g_carveout.insert(key);
     return e;
 }
 
@@ -861,18 +877,19 @@ static int launch_fused_image(const Shape &s, bool routed, const void *q, const 
 
 // ----------------------------------------------------------------------------- projections
 
-// 2-D bfloat16 map of a row-major (rows x cols) matrix: boxes of 32 columns x box_rows
-// rows, 64-byte swizzle (the MMA operand layout), zero fill past the last row.
-static bool encode_map_rows(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
+// 2-D bfloat16 map of a row-major (rows x cols) matrix: boxes of box_cols (32 or 64)
+// columns x box_rows rows with the matching 64- or 128-byte swizzle (the MMA operand and
+// output staging layouts); loads fill zeros past the last row, stores clip there.
+static bool encode_map_rows(CUtensorMap *m, const void *base, int rows, int cols, int box_rows, int box_cols = 32) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {32u, (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1u, 1u};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               CU_TENSOR_MAP_INTERLEAVE_NONE, box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Output columns per tile: the largest power of two in [32, 256] dividing ny (so that a
@@ -916,35 +933,50 @@ static int launch_linear(const void *x, const void *w, const void *b, int M, int
     LinearParams p;
     memset(&p, 0, sizeof(p));
     p.BN = linear_tile_n(ny);
-    if (!encode_map_rows(&p.tmX, x, M, K, kLinRows) || !encode_map_rows(&p.tmW, w, Nout, K, p.BN)) return BRA_ERR_CUDA;
+    p.kc_elems = K % 64 == 0 ? 64 : 32;
+    if (!encode_map_rows(&p.tmX, x, M, K, kLinRows, p.kc_elems) || !encode_map_rows(&p.tmW, w, Nout, K, p.BN, p.kc_elems))
+        return BRA_ERR_CUDA;
+    for (int i = 0; i < nsplit; ++i)
+        if (!encode_map_rows(&p.tmY[i], y[i], M, ny, 32)) return BRA_ERR_CUDA;
     p.bias = static_cast<const __nv_bfloat16 *>(b);
-    for (int i = 0; i < 3; ++i) p.y[i] = static_cast<__nv_bfloat16 *>(y[i < nsplit ? i : 0]);
     p.M = M;
     p.K = K;
     p.Nout = Nout;
     p.Ny = ny;
     p.tiles_n = Nout / p.BN;
-    p.tiles = (M + kLinRows - 1) / kLinRows * p.tiles_n;
+    p.tiles_m = (M + kLinRows - 1) / kLinRows;
     p.tmem_cols = 32;
     while (p.tmem_cols < (uint32_t)(2 * p.BN)) p.tmem_cols <<= 1;
     p.wait_limit = kWaitLimit;
-    // CTAs per SM are held to what the tensor memory takes (an allocation beyond its 512
-    // columns would wait for a resident CTA to finish): each CTA asks for enough shared
-    // memory that one more would not fit.
-    const int max_ctas = 512 / (int)p.tmem_cols;
-    constexpr int kSmPerSmBytes = 228 * 1024, kCtaReserve = 1024;
-    p.stages = 4;
-    int smem = linear_smem_layout(p.BN, p.stages, Nout).total;
-    smem = std::max(smem, kSmPerSmBytes / (max_ctas + 1) - kCtaReserve + 16);
-    if (smem > kMaxSmem) return BRA_ERR_SHAPE;
-    if (allow_smem(linear_umma_kernel, smem) != cudaSuccess) return BRA_ERR_CUDA;
-    int per_sm = 0, sms = 0;
-    if (occupancy(&per_sm, linear_umma_kernel, kLinThreads, smem, 0, nullptr) != cudaSuccess || per_sm < 1 ||
-        per_sm > max_ctas)
-        return BRA_ERR_CUDA;
+    const int kch = K / p.kc_elems, a_bytes = kLinRows * p.kc_elems * 2;
+    int sms = 0;
     int rc = sm_count(&sms);
     if (rc) return rc;
-    const int grid = std::min(p.tiles, sms * per_sm);
+    constexpr int kSmPerSmBytes = 228 * 1024, kCtaReserve = 1024;
+    // One CTA per SM (its 320 threads take most of the register file). W resident when
+    // W and two row tiles' worth of X chunks fit: X is then read once and W once per
+    // CTA. Otherwise streaming, with 2 to 8 stages. Each CTA asks for enough shared
+    // memory that a second one would not fit: the tensor memory would not hold it (an
+    // allocation beyond its 512 columns would wait for a resident CTA to finish).
+    int smem = 0;
+    const int res_fixed = linear_smem_layout(p.BN, 0, Nout, K, true, p.kc_elems).total;
+    if (res_fixed + 2 * kch * (a_bytes + 16) <= kMaxSmem) {
+        p.w_resident = 1;
+        p.stages = std::min(4 * kch, (kMaxSmem - res_fixed) / (a_bytes + 16));
+        smem = linear_smem_layout(p.BN, p.stages, Nout, K, true, p.kc_elems).total;
+        smem = std::max(smem, kSmPerSmBytes / 2 - kCtaReserve + 16);  // one CTA per SM
+    } else {
+        p.stages = 2;
+        while (p.stages < 8 && linear_smem_layout(p.BN, p.stages + 1, Nout, K, false, p.kc_elems).total <= kMaxSmem)
+            ++p.stages;
+        smem = linear_smem_layout(p.BN, p.stages, Nout, K, false, p.kc_elems).total;
+        smem = std::max(smem, kSmPerSmBytes / 2 - kCtaReserve + 16);
+    }
+    if (smem > kMaxSmem) return BRA_ERR_SHAPE;
+    if (allow_smem(linear_umma_kernel, smem) != cudaSuccess || prefer_shared(linear_umma_kernel) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    const int work = p.w_resident ? p.tiles_m : p.tiles_m * p.tiles_n;
+    const int grid = std::min(work, sms);
     LaunchScope ls(BRA_KERNEL_LINEAR_BF16, st);
     linear_umma_kernel<<<grid, kLinThreads, smem, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
@@ -1175,12 +1207,27 @@ int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, con
         return BRA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t plane = ((size_t)T * C * es + 255) / 256 * 256;  // one (N,H,W,C) tensor
+    const size_t route = 2 * (size_t)N * s.P * C * sizeof(float);
+    // outside a stream capture the scratch comes from the library's pool that keeps its
+    // memory between calls (mapping tens of MB again on every call costs milliseconds);
+    // inside one, from the default pool (a memory node of the graph)
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return BRA_ERR_CUDA;
     unsigned char *buf = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&buf), 4 * plane, st) != cudaSuccess) return BRA_ERR_CUDA;
+    if (cs == cudaStreamCaptureStatusNone) {
+        cudaMemPool_t pool = nullptr;
+        cudaStream_t up = nullptr, back = nullptr;
+        if ((rc = host_call_pool(&pool, &up, &back))) return rc;
+        if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&buf), 4 * plane + route, pool, st) != cudaSuccess)
+            return BRA_ERR_CUDA;
+    } else if (cudaMallocAsync(reinterpret_cast<void **>(&buf), 4 * plane + route, st) != cudaSuccess) {
+        return BRA_ERR_CUDA;
+    }
     void *qkv[3] = {buf, buf + plane, buf + 2 * plane};
     void *o = buf + 3 * plane;
+    float *ws = reinterpret_cast<float *>(buf + 4 * plane);
     rc = launch_linear(x, w_qkv, b_qkv, (int)T, C, 3 * C, 3, qkv, dtype, st);
-    if (rc == BRA_OK) rc = forward_device(s, qkv[0], qkv[1], qkv[2], lce_w, lce_b, o, r_idx, r_weight, st);
+    if (rc == BRA_OK) rc = forward_device(s, qkv[0], qkv[1], qkv[2], lce_w, lce_b, o, r_idx, r_weight, st, ws);
     if (rc == BRA_OK) rc = launch_linear(o, w_o, b_o, (int)T, C, C, 1, &out, dtype, st);
     if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     return rc;

@@ -11,10 +11,14 @@
 // n / Ny, column n % Ny): the qkv projection writes q, k and v directly.
 //
 // bfloat16: linear_umma_kernel, a persistent tcgen05 GEMM. One warp issues tensor
-// copies of 128-row X chunks and BN-row W chunks (32 K-elements, 64-byte swizzle) into
+// copies of 128-row X chunks and BN-row W chunks (KC = 64 K-elements with a 128-byte
+// swizzle when K allows, else 32 with a 64-byte swizzle: wider rows stream faster) into
 // a ring of shared-memory stages; one thread issues the 128 x BN x 16 MMAs into a
-// double-buffered float32 accumulator in tensor memory; four warps drain it (one TMEM
-// lane quarter each), add the bias, round to bfloat16 and store. Every wait is bounded.
+// double-buffered float32 accumulator in tensor memory; eight warps drain it (two per
+// TMEM lane quarter, alternate 32-column blocks, the next block's tensor-memory load in
+// flight while the current one is processed), add the bias, round to bfloat16 and stage
+// each 32 x 32 block in shared memory (64-byte swizzle), from where a tensor store
+// writes it out (rows past M are clipped by the store). Every wait is bounded.
 // float32: linear_f32_kernel, shared-memory tiles and FMA.
 #pragma once
 
@@ -27,31 +31,44 @@
 namespace bra {
 
 struct LinearParams {
-    CUtensorMap tmX;  // X (M, K): box (32, 128), 64-byte swizzle, zero fill past row M
-    CUtensorMap tmW;  // W (Nout, K): box (32, BN), 64-byte swizzle
+    CUtensorMap tmX;     // X (M, K): box (32, 128), 64-byte swizzle, zero fill past row M
+    CUtensorMap tmW;     // W (Nout, K): box (32, BN), 64-byte swizzle
+    CUtensorMap tmY[3];  // Y_i (M, Ny): box (32, 32), 64-byte swizzle
     const __nv_bfloat16 *bias;
-    __nv_bfloat16 *y[3];
-    int M, K, Nout, Ny, BN, tiles_n, tiles, stages;
+    int M, K, Nout, Ny, BN, tiles_n, tiles_m, stages;
+    int kc_elems;    // K-elements per chunk: 64 (128-byte rows) or 32 (64-byte rows)
+    int w_resident;  // 1: all of W stays in shared memory, the stages carry X chunks only
     uint32_t tmem_cols;
     unsigned wait_limit;
 };
 
-constexpr int kLinThreads = 192;  // warp 0 copies, warp 1 MMA, warps 2-5 epilogue
-constexpr int kLinRows = 128;     // rows of X per tile (the MMA's M)
+constexpr int kLinEpiWarps = 8;                     // two per tensor-memory lane quarter
+constexpr int kLinThreads = 64 + 32 * kLinEpiWarps;  // warp 0 copies, warp 1 MMA, then the epilogue
+constexpr int kLinRows = 128;                        // rows of X per tile (the MMA's M)
+constexpr int kLinOutSlots = 4;                      // 32 x 32 output blocks in flight per epilogue warp
 
 struct LinearSmem {
-    int stage_bytes, a_bytes, bias, bars, tslot, total;
+    int stage_bytes, a_bytes, w, out, bias, bars, tslot, total;
 };
 
-__host__ __device__ inline LinearSmem linear_smem_layout(int BN, int stages, int Nout) {
+// Two modes. W resident (Nout * K * 2 bytes of W held for the whole kernel, loaded once
+// per CTA): a stage is one 32-wide K chunk of a 128-row X tile, and each X tile is used
+// for all tiles_n column tiles before its stages are released. Streaming: a stage is an
+// X chunk and the matching BN-row W chunk of one (row tile, column tile) unit.
+__host__ __device__ inline LinearSmem linear_smem_layout(int BN, int stages, int Nout, int K, bool w_resident,
+                                                        int kc_elems) {
     LinearSmem s;
-    s.a_bytes = kLinRows * 64;  // 128 rows x 32 bf16
-    s.stage_bytes = s.a_bytes + BN * 64;
+    s.a_bytes = kLinRows * kc_elems * 2;  // 128 rows x one K chunk
+    s.stage_bytes = w_resident ? s.a_bytes : s.a_bytes + BN * kc_elems * 2;
     int end = stages * s.stage_bytes;
+    s.w = end;  // W resident: [tiles_n][K / KC][BN rows x one K chunk]
+    end += w_resident ? Nout * K * 2 : 0;
+    s.out = end;  // [kLinEpiWarps][kLinOutSlots][32 rows x 64 B] output staging
+    end += kLinEpiWarps * kLinOutSlots * 2048;
     s.bias = end;  // float32 [Nout]
     end += ((Nout * 4 + 15) / 16) * 16;
-    s.bars = end;  // full[stages], empty[stages], tfull[2], tempty[2], drain
-    end += 8 * (2 * stages + 5);
+    s.bars = end;  // full[stages], empty[stages], tfull[2], tempty[2], drain, wfull
+    end += 8 * (2 * stages + 6);
     s.tslot = end;
     end += 16;
     s.total = end + 1024;  // 1024-byte alignment of the base
@@ -68,19 +85,63 @@ __device__ inline void lin_tma_load_2d(uint32_t dst, const void *tmap, int c0, i
 __device__ inline void lin_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
+__device__ inline void lin_tma_store_2d(const void *tmap, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];\n" ::"l"(tmap),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ inline void lin_bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// Wait until at most N of this thread's committed store groups still read shared memory.
+template <int N> __device__ inline void lin_bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;\n" ::"n"(N) : "memory");
+}
+// Wait until at most N of this thread's committed store groups are still incomplete.
+template <int N> __device__ inline void lin_bulk_wait() {
+    asm volatile("cp.async.bulk.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// The work of a CTA is a sequence of units (row tile, column tile): W resident, its
+// row tiles blockIdx.x, blockIdx.x + gridDim.x, ... each with column tiles 0 .. tiles_n-1
+// in order; streaming, the units blockIdx.x, blockIdx.x + gridDim.x, ... of the
+// row-major unit grid.
+__device__ inline int lin_units(const LinearParams &p) {
+    if (p.w_resident) {
+        const int mt = (int)blockIdx.x < p.tiles_m ? (p.tiles_m - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+        return mt * p.tiles_n;
+    }
+    const int tiles = p.tiles_m * p.tiles_n;
+    return (int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+}
+__device__ inline void lin_unit(const LinearParams &p, int i, int &mt, int &nt) {
+    if (p.w_resident) {
+        mt = (int)blockIdx.x + (i / p.tiles_n) * (int)gridDim.x;
+        nt = i % p.tiles_n;
+    } else {
+        const int t = (int)blockIdx.x + i * (int)gridDim.x;
+        mt = t / p.tiles_n;
+        nt = t % p.tiles_n;
+    }
+}
 
 __global__ void __launch_bounds__(kLinThreads, 1) linear_umma_kernel(const __grid_constant__ LinearParams prm) {
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *sm = smem_raw + (base - raw);
-    const int BN = prm.BN, NS = prm.stages, kch = prm.K >> 5;
-    const LinearSmem L = linear_smem_layout(BN, NS, prm.Nout);
+    const int BN = prm.BN, NS = prm.stages, KC = prm.kc_elems, kch = prm.K / KC;
+    const bool wres = prm.w_resident != 0;
+    const LinearSmem L = linear_smem_layout(BN, NS, prm.Nout, prm.K, wres, KC);
+    // K-major operands: rows of KC bf16 (2 * KC bytes), 8-row groups 16 * KC bytes apart,
+    // the k-th 16-element step 32 bytes into the row
+    const uint32_t sbo = (uint32_t)(16 * KC);
+    const uint64_t swz = KC == 64 ? kDescSwizzle128B : kDescSwizzle64B;
+    const int wchunk = BN * KC * 2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t bars = base + L.bars;
     const uint32_t full0 = bars, empty0 = bars + 8 * NS, tfull0 = bars + 16 * NS, tempty0 = tfull0 + 16,
-                   drain = tfull0 + 32;
+                   drain = tfull0 + 32, wfull = tfull0 + 40;
     const uint32_t lim = prm.wait_limit;
+    const int units = lin_units(prm);
     float *sBias = reinterpret_cast<float *>(sm + L.bias);
 
     if (warp == 1) {
@@ -94,9 +155,10 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_umma_kernel(const __gri
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
-            mbar_init(tempty0 + 8 * b, 128);
+            mbar_init(tempty0 + 8 * b, 32 * kLinEpiWarps);
         }
         mbar_init(drain, 1);
+        mbar_init(wfull, 1);
         fence_mbar_init();
     }
     for (int i = tid; i < prm.Nout; i += kLinThreads) sBias[i] = __bfloat162float(prm.bias[i]);
@@ -108,11 +170,20 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_umma_kernel(const __gri
     if (warp == 0) {
         // ---------------------------------------------------------------- tensor copies
         if (lane == 0) {
+            if (wres && units > 0) {
+                // all of W once, chunk (nt, kc) at ((nt * kch) + kc) * wchunk
+                mbar_arrive_expect_tx(wfull, (uint32_t)(prm.Nout * prm.K * 2));
+                for (int nt = 0; nt < prm.tiles_n; ++nt)
+                    for (int kc = 0; kc < kch; ++kc)
+                        lin_tma_load_2d(base + L.w + (nt * kch + kc) * wchunk, &prm.tmW, kc * KC, nt * BN, wfull);
+            }
             const uint32_t bytes = (uint32_t)L.stage_bytes;
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < prm.tiles && ok; t += gridDim.x) {
-                const int m0 = (t / prm.tiles_n) * kLinRows, n0 = (t % prm.tiles_n) * BN;
+            for (int i = 0; i < units && ok; ++i) {
+                int mt, nt;
+                lin_unit(prm, i, mt, nt);
+                if (wres && nt > 0) continue;  // the row tile's chunks serve all its column tiles
                 for (int kc = 0; kc < kch; ++kc, ++it) {
                     const int s = it % NS, use = it / NS;
                     if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1, lim)) {
@@ -121,46 +192,55 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_umma_kernel(const __gri
                     }
                     const uint32_t st = base + s * L.stage_bytes;
                     mbar_arrive_expect_tx(full0 + 8 * s, bytes);
-                    lin_tma_load_2d(st, &prm.tmX, kc * 32, m0, full0 + 8 * s);
-                    lin_tma_load_2d(st + L.a_bytes, &prm.tmW, kc * 32, n0, full0 + 8 * s);
+                    lin_tma_load_2d(st, &prm.tmX, kc * KC, mt * kLinRows, full0 + 8 * s);
+                    if (!wres) lin_tma_load_2d(st + L.a_bytes, &prm.tmW, kc * KC, nt * BN, full0 + 8 * s);
                 }
             }
             if (!ok) atomicExch(&g_bra_timeout_flag, 1);
             // every copy issued has landed before the CTA may exit (immediate when the
             // MMA thread consumed them all)
             for (int s = 0; s < NS && s < it; ++s) mbar_wait_bounded(full0 + 8 * s, ((it - 1 - s) / NS) & 1, lim);
+            if (wres && units > 0) mbar_wait_bounded(wfull, 0, lim);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issue
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(kLinRows, BN, 0, 0);
-            int it = 0, k = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < prm.tiles && ok; t += gridDim.x, ++k) {
-                const int b = k & 1, ub = k >> 1;
+            bool ok = !(wres && units > 0) || mbar_wait_bounded(wfull, 0, lim);
+            int it = 0;  // first stage index of the current row tile (W resident) / unit
+            for (int i = 0; i < units && ok; ++i) {
+                int mt, nt;
+                lin_unit(prm, i, mt, nt);
+                const int b = i & 1, ub = i >> 1;
                 if (ub > 0 && !mbar_wait_bounded(tempty0 + 8 * b, (ub - 1) & 1, lim)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d = tbase + (uint32_t)(b * BN);
-                for (int kc = 0; kc < kch; ++kc, ++it) {
-                    const int s = it % NS, use = it / NS;
-                    if (!mbar_wait_bounded(full0 + 8 * s, use & 1, lim)) {
+                for (int kc = 0; kc < kch; ++kc) {
+                    const int s = (it + kc) % NS, use = (it + kc) / NS;
+                    if ((!wres || nt == 0) && !mbar_wait_bounded(full0 + 8 * s, use & 1, lim)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t st = base + s * L.stage_bytes;
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk)
-                        umma_ss(d, smem_desc(st + 32 * kk, 16, 512, kDescSwizzle64B),
-                                smem_desc(st + L.a_bytes + 32 * kk, 16, 512, kDescSwizzle64B), idesc,
+                    const uint32_t a = base + s * L.stage_bytes;
+                    const uint32_t w = wres ? base + L.w + (nt * kch + kc) * wchunk : a + L.a_bytes;
+                    for (int kk = 0; kk < KC / 16; ++kk)
+                        umma_ss(d, smem_desc(a + 32 * kk, 16, sbo, swz), smem_desc(w + 32 * kk, 16, sbo, swz), idesc,
                                 (uint32_t)((kc | kk) != 0));
-                    umma_commit(empty0 + 8 * s);  // the stage is free once these MMAs have read it
+                    if (!wres) umma_commit(empty0 + 8 * s);  // streaming: the stage is free once read
                 }
                 if (!ok) break;
                 umma_commit(tfull0 + 8 * b);  // the accumulator is complete
+                if (!wres) {
+                    it += kch;
+                } else if (nt == prm.tiles_n - 1) {
+                    // the row tile's stages are free once its last column tile has read them
+                    for (int kc = 0; kc < kch; ++kc) umma_commit(empty0 + 8 * ((it + kc) % NS));
+                    it += kch;
+                }
             }
             if (!ok) atomicExch(&g_bra_timeout_flag, 1);
             // every MMA must have completed before the tensor memory is released
@@ -169,41 +249,78 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_umma_kernel(const __gri
         }
     } else {
         // ---------------------------------------------------------------- epilogue
-        const int q = warp & 3;  // tensor-memory lane quarter of this warp
-        int k = 0;
+        // warp (q, h): rows 32q .. 32q + 31 (its tensor-memory lane quarter), column
+        // blocks 32h, 32h + 64, ... of each unit
+        const int q = warp & 3, h = (warp - 2) >> 2;
+        const uint32_t stg = base + L.out + (warp - 2) * (kLinOutSlots * 2048);
+        int g = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < prm.tiles; t += gridDim.x, ++k) {
-            const int b = k & 1, ub = k >> 1;
+        for (int i = 0; i < units; ++i) {
+            const int b = i & 1, ub = i >> 1;
             if (!mbar_wait_bounded(tfull0 + 8 * b, ub & 1, lim)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int m0 = (t / prm.tiles_n) * kLinRows, n0 = (t % prm.tiles_n) * BN;
-            const int row = m0 + 32 * q + lane;
+            int mt, nt;
+            lin_unit(prm, i, mt, nt);
+            const int m0 = mt * kLinRows, n0 = nt * BN;
             const int which = n0 / prm.Ny, col0 = n0 - which * prm.Ny;
-            __nv_bfloat16 *dst = prm.y[which] + (size_t)row * prm.Ny + col0;
             const uint32_t taddr = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN);
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(taddr + (uint32_t)c, r);
-                uint32_t pk[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float2 bb = *reinterpret_cast<const float2 *>(sBias + n0 + c + 2 * j);
-                    const __nv_bfloat162 h =
-                        __floats2bfloat162_rn(__uint_as_float(r[2 * j]) + bb.x, __uint_as_float(r[2 * j + 1]) + bb.y);
-                    pk[j] = *reinterpret_cast<const uint32_t *>(&h);
+            // bias, round, stage and store the 32 x 32 block at column c of the unit
+            auto emit = [&](const uint32_t (&r)[32], int c) {
+                const uint32_t sb = stg + (g % kLinOutSlots) * 2048;
+                if (g >= kLinOutSlots) {
+                    // the store that used this slot has finished reading it
+                    if (lane == 0) lin_bulk_wait_read<kLinOutSlots - 1>();
+                    __syncwarp();
                 }
-                if (row < prm.M) {
-                    uint4 *o = reinterpret_cast<uint4 *>(dst + c);
+                // row `lane` of the block: four 16-byte chunks, 64-byte swizzle
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) o[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = 8 * j + 2 * e;
+                        const float2 bb = *reinterpret_cast<const float2 *>(sBias + n0 + c + col);
+                        const __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(r[col]) + bb.x,
+                                                                        __uint_as_float(r[col + 1]) + bb.y);
+                        pk[e] = *reinterpret_cast<const uint32_t *>(&hv);
+                    }
+                    const uint32_t dst = sb + lane * 64 + (((j ^ (lane >> 1)) & 3) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
+                                 "r"(pk[2]), "r"(pk[3])
+                                 : "memory");
                 }
+                fence_proxy_async();  // the tensor store reads what the generic stores wrote
+                __syncwarp();
+                if (lane == 0) {
+                    // a block wholly past row M is not stored (its group is empty), so that
+                    // every block still commits one group for the slot bookkeeping
+                    if (m0 + 32 * q < prm.M) lin_tma_store_2d(&prm.tmY[which], sb, col0 + c, m0 + 32 * q);
+                    lin_bulk_commit();
+                }
+                ++g;
+            };
+            uint32_t ra[32], rb[32];
+            int c = 32 * h;
+            if (c < BN) tmem_ld32_nowait(taddr + (uint32_t)c, ra);
+            while (c < BN) {
+                tmem_wait_ld(ra);
+                const int c1 = c + 64;
+                if (c1 < BN) tmem_ld32_nowait(taddr + (uint32_t)c1, rb);
+                emit(ra, c);
+                if (c1 >= BN) break;
+                tmem_wait_ld(rb);
+                const int c2 = c1 + 64;
+                if (c2 < BN) tmem_ld32_nowait(taddr + (uint32_t)c2, ra);
+                emit(rb, c1);
+                c = c2;
             }
             tc_fence_before();
-            lin_arrive(tempty0 + 8 * b);  // this thread's lane of the accumulator is read
+            lin_arrive(tempty0 + 8 * b);  // this thread's share of the accumulator is read
         }
+        if (lane == 0) lin_bulk_wait<0>();  // the stores are complete before the CTA exits
         if (!ok && lane == 0) atomicExch(&g_bra_timeout_flag, 1);
     }
 
