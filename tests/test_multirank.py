@@ -1,7 +1,7 @@
 """Multi-process (gloo, world size 2, CPU) checks of the batch-sharded path.
 
 BRA never crosses images: region means, routing, the routed attention and the LCE
-all stay inside one image. So N images split over ranks, each rank running its own
+all stay inside one image (and the projections of the attention layer act per token). So N images split over ranks, each rank running its own
 share with no exchange, must give exactly the full-batch result, and the benchmark
 only needs a max-over-ranks reduction of its timings. The ranks here run the oracle
 (there is no GPU in this test); the property checked is the partition itself.
@@ -36,22 +36,33 @@ def _free_port():
     return port
 
 
-def _rank_main(rank, world, port, result_path):
+LAYER_KEYS = ("x", "w_qkv", "b_qkv", "w_o", "b_o", "lce_w", "lce_b")
+
+
+def _run(inp, a, b, layer):
+    """The forward (or the whole layer) of images a .. b-1."""
+    if layer:
+        args = [inp[k] for k in LAYER_KEYS]
+        args[0] = args[0][a:b]
+        return oracle.layer_forward(*args, W.heads, W.S, W.topk, W.dtype)
+    return oracle.forward(*(inp[k][a:b] for k in ("q", "k", "v")), inp["lce_w"], inp["lce_b"], W.heads, W.S,
+                          W.topk)
+
+
+def _rank_main(rank, world, port, result_path, layer=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        inp = synth.make_inputs(W)
+        inp = synth.make_layer_inputs(W) if layer else synth.make_inputs(W)
         a, b = shard(W.N, world, rank)
-        out, r_idx, r_w = oracle.forward(*(inp[k][a:b] for k in ("q", "k", "v")), inp["lce_w"], inp["lce_b"],
-                                         W.heads, W.S, W.topk)
+        out, r_idx, r_w = _run(inp, a, b, layer)
         parts = [None] * world
         dist.all_gather_object(parts, (a, b, out, r_idx, r_w))
         t = torch.tensor([1.0 + rank], dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         if rank == 0:
-            full_out, full_idx, full_w = oracle.forward(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"],
-                                                        W.heads, W.S, W.topk)
+            full_out, full_idx, full_w = _run(inp, 0, W.N, layer)
             cat_out = np.concatenate([p[2] for p in parts])
             cat_idx = np.concatenate([p[3] for p in parts])
             cat_w = np.concatenate([p[4] for p in parts])
@@ -79,3 +90,12 @@ def test_two_rank_batch_split_equals_full_batch(tmp_path):
     result = str(tmp_path / "result.txt")
     mp.spawn(_rank_main, args=(2, _free_port(), result), nprocs=2, join=True)
     assert open(result).read() == "ok"
+
+
+@pytest.mark.timeout(300)
+def test_two_rank_layer_split_equals_full_batch(tmp_path):
+    """The same partition for the attention layer (qkv projection, BRA, output projection)."""
+    result = str(tmp_path / "result.txt")
+    mp.spawn(_rank_main, args=(2, _free_port(), result, True), nprocs=2, join=True)
+    with open(result) as f:
+        assert f.read() == "ok"
