@@ -4,9 +4,11 @@ Only `tests/`, `__graft_entry__.smoke()` and the benchmark's CPU-baseline leg ma
 import this package. The CUDA library never calls it, and it imports nothing from
 the CUDA package.
 
-The arithmetic lives in `bra_oracle.c` (plain C, float64, OpenMP over regions),
-compiled with gcc into `liboracle_bra.so` next to it. This module only marshals
-numpy arrays through ctypes.
+The forward's arithmetic lives in `bra_oracle.c` (plain C, float64, OpenMP over
+regions), compiled with gcc into `liboracle_bra.so` next to it; this module marshals
+numpy arrays through ctypes and adds the attention layer's projections (numpy, float64,
+below). The backward pass with the routing detached is `oracle/backward.py` (numpy,
+float64).
 
 Every function follows the official BRA code as walked through on
 "BiFormer ... 前向传播过程" (niftyadmin), section "BRA模块", eqs. 4-7, and
