@@ -141,12 +141,38 @@ def kernel_sources(kernel: str):
     return sorted(seen)
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without its comments, trailing blanks and empty lines (string and
+    character literals kept as they are), so that a comment edit leaves the hash alone."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).split("\n"))
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_hash(kernel: str) -> str:
+    """Hash of the kernel's header closure with comments and blank lines removed."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "vision_transformer_sparse_b200", "csrc")
     for name in kernel_sources(kernel):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -31,8 +31,8 @@
 namespace bra {
 
 struct LinearParams {
-    CUtensorMap tmX;     // X (M, K): box (32, 128), 64-byte swizzle, zero fill past row M
-    CUtensorMap tmW;     // W (Nout, K): box (32, BN), 64-byte swizzle
+    CUtensorMap tmX;     // X (M, K): box (KC, 128), KC-matched swizzle, zero fill past row M
+    CUtensorMap tmW;     // W (Nout, K): box (KC, BN), KC-matched swizzle
     CUtensorMap tmY[3];  // Y_i (M, Ny): box (32, 32), 64-byte swizzle
     const __nv_bfloat16 *bias;
     int M, K, Nout, Ny, BN, tiles_n, tiles_m, stages;
@@ -52,7 +52,7 @@ struct LinearSmem {
 };
 
 // Two modes. W resident (Nout * K * 2 bytes of W held for the whole kernel, loaded once
-// per CTA): a stage is one 32-wide K chunk of a 128-row X tile, and each X tile is used
+// per CTA): a stage is one KC-wide K chunk of a 128-row X tile, and each X tile is used
 // for all tiles_n column tiles before its stages are released. Streaming: a stage is an
 // X chunk and the matching BN-row W chunk of one (row tile, column tile) unit.
 __host__ __device__ inline LinearSmem linear_smem_layout(int BN, int stages, int Nout, int K, bool w_resident,
