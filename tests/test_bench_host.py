@@ -64,7 +64,7 @@ def test_algorithmic_figures_of_the_detection_stage(bench):
     assert acc["gathered_bytes"] == w.N * w.S * w.S * L * 2 * w.C * 2
 
 
-def test_source_hash_ignores_comments_only():
+def test_source_hash_ignores_comments_only(bench):
     """A profile stays matched across comment edits, and not across code edits."""
     src = 'int a = 1; // note\n/* block\n comment */ const char *s = "x // kept"; char q = \'/\';\n\n  int b;\n'
     assert bench.strip_comments(src) == 'int a = 1;\n const char *s = "x // kept"; char q = \'/\';\n  int b;'
