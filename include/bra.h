@@ -182,6 +182,24 @@ int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, con
                         int topk, int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * The backward pass of steps 4-5 with the routing detached: the walk-through's router
+ * ("BiFormer ... 前向传播过程", section "BRA模块", TopkRouting) detaches the region
+ * query and key when diff_routing is off (its default); the top-k index is discrete and
+ * r_weight does not scale K or V, so gradients flow through the token attention and the
+ * LCE only. Given dout = dL/dout (N,H,W,C) in `dtype` and the forward's r_idx, writes
+ *   dq, dk, dv: (N,H,W,C) float32;  dlce_w: (C,5,5) float32;  dlce_b: (C) float32.
+ * Arithmetic in float32; dk and dv are accumulated with atomics (the summation order,
+ * and so the last bits, can differ between calls). The attention softmax is recomputed
+ * from q and k. Every r_idx entry must lie in [0, S*S): an entry outside is skipped and
+ * the call returns BRA_ERR_INDEX; like bra_attend, this call synchronises `stream` to
+ * read that flag. Shapes as bra_forward; q, k, v, dout, lce_w aligned to their element,
+ * the float32 outputs and r_idx to 4 bytes. N = 0 zeroes dlce_w and dlce_b only.
+ * Plain SIMT kernels: a first, correct form of this step, not yet tuned. */
+int bra_backward(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
+                 const void *dout, int N, int H, int W, int C, int heads, int S, int topk, int dtype, float *dq,
+                 float *dk, float *dv, float *dlce_w, float *dlce_b, bra_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Tracing (measurement support; no part of the computation).
  *
  * Kernel classes the library launches, for bra_trace_end and bra_kernel_name. */
@@ -194,7 +212,8 @@ enum {
     BRA_KERNEL_ATTN_UMMA = 5,   /* steps 4-5, tcgen05 kernel (large regions)       */
     BRA_KERNEL_LINEAR_BF16 = 6, /* qkv / output projection, tcgen05 GEMM          */
     BRA_KERNEL_LINEAR_F32 = 7,  /* qkv / output projection, float32 SIMT          */
-    BRA_KERNEL_CLASSES = 8
+    BRA_KERNEL_BACKWARD = 8,    /* bra_backward's kernels, timed together          */
+    BRA_KERNEL_CLASSES = 9
 };
 
 /* Number of kernels this library has launched since it was loaded (all threads,

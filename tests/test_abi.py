@@ -149,3 +149,22 @@ def test_layer_nulls_and_alignment(bra_lib):
         ptrs[i] = ODD
         assert bra.raw_call("bra_attention_layer", *ptrs[:7], *shape, *ptrs[7:], None) == 3
     assert bra.raw_call("bra_attention_layer", *[None] * 7, 0, 56, 56, 64, 2, 7, 1, 1, *[None] * 3, None) == 0
+
+
+def test_backward_rejects_before_cuda(bra_lib):
+    shape = (1, 56, 56, 64, 2, 7, 1, 1)
+    call = lambda ptrs, shp=shape: bra.raw_call("bra_backward", *ptrs[:6], *shp, *ptrs[6:], None)
+    assert call([FAKE] * 11, (1, 57, 56, 64, 2, 7, 1, 1)) == 2      # H % S
+    assert call([FAKE] * 11, (1, 56, 56, 64, 2, 7, 1, 7)) == 4      # dtype
+    for i in range(11):
+        ptrs = [FAKE] * 11
+        ptrs[i] = None
+        assert call(ptrs) == 1
+    for i in (0, 1, 2, 3, 5):   # bf16 maps and weight: 2-byte alignment
+        ptrs = [FAKE] * 11
+        ptrs[i] = ctypes.c_void_p(0x10001)
+        assert call(ptrs) == 3
+    for i in (4, 6, 7, 8, 9, 10):   # r_idx and the float32 outputs: 4 bytes
+        ptrs = [FAKE] * 11
+        ptrs[i] = ctypes.c_void_p(0x10002)
+        assert call(ptrs) == 3

@@ -27,8 +27,8 @@ SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_fo
            "bra_status_string",
            "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name",
            "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout", "bra_trace_read",
-           "bra_linear", "bra_qkv", "bra_attention_layer")
-KERNEL_CLASSES = 8
+           "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward")
+KERNEL_CLASSES = 9
 
 
 class BraError(RuntimeError):
@@ -54,8 +54,9 @@ def lib() -> ctypes.CDLL:
         L.bra_linear.argtypes = [vp] * 3 + [i] * 4 + [vp, vp]
         L.bra_qkv.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
         L.bra_attention_layer.argtypes = [vp] * 7 + shape + [vp, vp, vp, vp]
+        L.bra_backward.argtypes = [vp] * 6 + shape + [vp] * 6
         for f in ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
-                  "bra_version", "bra_linear", "bra_qkv", "bra_attention_layer"):
+                  "bra_version", "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward"):
             getattr(L, f).restype = i
         L.bra_status_string.argtypes = [i]
         L.bra_status_string.restype = ctypes.c_char_p
@@ -162,6 +163,23 @@ def attention_layer(x, w_qkv, b_qkv, w_o, b_o, lce_w, lce_b, heads: int, S: int,
                                    _ptr(r_idx), _ptr(r_weight), _stream(stream))
     _raise(rc, "bra_attention_layer")
     return out, r_idx, r_weight
+
+
+def backward(q, k, v, lce_w, r_idx, dout, heads: int, S: int, stream=None) -> dict:
+    """bra_backward: gradients (float32) of sum(dout * forward output) for the routing
+    r_idx (N, S*S, topk), routing detached -> {dq, dk, dv, dlce_w, dlce_b}."""
+    N, H, W, C = q.shape
+    topk = r_idx.shape[-1]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"dq": torch.empty((N, H, W, C), **f32), "dk": torch.empty((N, H, W, C), **f32),
+         "dv": torch.empty((N, H, W, C), **f32), "dlce_w": torch.empty((C, 5, 5), **f32),
+         "dlce_b": torch.empty((C,), **f32)}
+    _check_dev(q, k, v, lce_w, r_idx, dout, *g.values())
+    rc = lib().bra_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(r_idx), _ptr(dout), N, H, W, C, heads, S,
+                            topk, _dtype_code(q), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlce_w"]),
+                            _ptr(g["dlce_b"]), _stream(stream))
+    _raise(rc, "bra_backward")
+    return g
 
 
 def forward_noalloc(q, k, v, lce_w, lce_b, heads: int, S: int, topk: int, out=None, r_idx=None,

@@ -33,6 +33,7 @@
 #include "attn_pipe.cuh"
 #include "attn_tma.cuh"
 #include "attn_umma.cuh"
+#include "backward.cuh"
 #include "fused_image.cuh"
 #include "linear.cuh"
 #include "route.cuh"
@@ -1084,6 +1085,7 @@ const char *bra_kernel_name(int kernel_class) {
         case BRA_KERNEL_ATTN_UMMA: return "attn_umma_kernel";
         case BRA_KERNEL_LINEAR_BF16: return "linear_umma_kernel";
         case BRA_KERNEL_LINEAR_F32: return "linear_f32_kernel";
+        case BRA_KERNEL_BACKWARD: return "bwd_kernels";
         default: return "unknown";
     }
 }
@@ -1230,6 +1232,62 @@ int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, con
     if (rc == BRA_OK) rc = forward_device(s, qkv[0], qkv[1], qkv[2], lce_w, lce_b, o, r_idx, r_weight, st, ws);
     if (rc == BRA_OK) rc = launch_linear(o, w_o, b_o, (int)T, C, C, 1, &out, dtype, st);
     if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    return rc;
+}
+
+int bra_backward(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
+                 const void *dout, int N, int H, int W, int C, int heads, int S, int topk, int dtype, float *dq,
+                 float *dk, float *dv, float *dlce_w, float *dlce_b, bra_stream_t stream) {
+    const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!lce_w || !dlce_w || !dlce_b) return BRA_ERR_NULL;
+    if (!aligned(dlce_w, 4) || !aligned(dlce_b, 4)) return BRA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {  // the parameter gradients of an empty batch are zero
+        if (cudaMemsetAsync(dlce_w, 0, (size_t)C * 25 * sizeof(float), st) != cudaSuccess ||
+            cudaMemsetAsync(dlce_b, 0, (size_t)C * sizeof(float), st) != cudaSuccess)
+            return BRA_ERR_CUDA;
+        return BRA_OK;
+    }
+    if (!q || !k || !v || !r_idx || !dout || !dq || !dk || !dv) return BRA_ERR_NULL;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    if (!aligned(q, es) || !aligned(k, es) || !aligned(v, es) || !aligned(dout, es) || !aligned(lce_w, es) ||
+        !aligned(r_idx, 4) || !aligned(dq, 4) || !aligned(dk, 4) || !aligned(dv, 4))
+        return BRA_ERR_ALIGN;
+    int sms = 0;
+    if ((rc = sm_count(&sms))) return rc;
+    int *flag = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&flag), sizeof(int), st) != cudaSuccess) return BRA_ERR_CUDA;
+    const BwdParams p = make_bwd_params(q, k, v, dout, lce_w, r_idx, N, H, W, C, heads, S, topk, dtype == BRA_BF16,
+                                        dq, dk, dv, dlce_w, dlce_b, flag);
+    const size_t elems = bwd_elems(p), items = bwd_attn_items(p);
+    rc = cudaMemsetAsync(flag, 0, sizeof(int), st) == cudaSuccess &&
+                 cudaMemsetAsync(dk, 0, elems * sizeof(float), st) == cudaSuccess
+             ? BRA_OK
+             : BRA_ERR_CUDA;
+    if (rc == BRA_OK) {
+        {
+            LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+            bwd_lce_dv_kernel<<<(unsigned)std::min<size_t>((elems + 255) / 256, (size_t)sms * 8), 256, 0, st>>>(p);
+        }
+        {
+            LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+            bwd_attn_kernel<<<(unsigned)std::min<size_t>((items + 127) / 128, (size_t)sms * 16), 128, 0, st>>>(p);
+        }
+        {
+            LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+            bwd_lce_param_kernel<<<C * 26, 256, 0, st>>>(p);
+        }
+        if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
+    }
+    int host_flag = 0;
+    if (rc == BRA_OK &&
+        cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        rc = BRA_ERR_CUDA;
+    if (cudaFreeAsync(flag, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    if (rc == BRA_OK && host_flag) rc = BRA_ERR_INDEX;
     return rc;
 }
 
