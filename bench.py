@@ -48,6 +48,7 @@ from vision_transformer_sparse_b200 import synth  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "BRA fwd tokens/s and TFLOP/s at 1 B200; % of bf16 tensor/HBM roofline"
 METRIC_LAYER = "BRA attention layer fwd (qkv projection + BRA + output projection) tokens/s at 1 B200"
+METRIC_BWD = "BRA backward (routing detached) tokens/s at 1 B200"
 
 
 def parse():
@@ -62,6 +63,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch each step directly")
     ap.add_argument("--layer", action="store_true",
                     help="time the whole attention layer (bra_attention_layer) instead of the BRA forward")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (bra_backward, routing detached) instead of the forward")
     ap.add_argument("--variant", default="auto", choices=["auto", "generic", "tma", "split", "pipe"],
                     help="attention kernel (auto: persistent TMA pipeline where the shape allows)")
     ap.add_argument("--source-hash", metavar="KERNEL",
@@ -91,9 +94,12 @@ def algorithmic(w: synth.Workload):
     # over the two launches of a layer forward.
     lin_bytes = (4.0 * T * w.C * b + 3 * w.C * w.C * b + 2.0 * T * w.C * b + w.C * w.C * b) / 2
     lin_flops = 8.0 * T * w.C * w.C
+    # the backward: q, k, v and dout read, dq, dk, dv written in float32, the routing and
+    # the LCE weight read, its float32 gradients written (per call, all its kernels)
+    bwd_bytes = 4.0 * T * w.C * b + 3.0 * T * w.C * 4 + w.N * w.regions * w.topk * 4 + w.C * 25 * (b + 4) + w.C * 4
     return {"tokens": T, "flops": flops, "gathered_bytes": gathered, "attn_bytes": attn_unique,
             "pool_bytes": pool_bytes, "route_bytes": route_bytes, "fused_bytes": fused_bytes,
-            "linear_bytes": lin_bytes, "linear_flops": lin_flops, "elem_bytes": b}
+            "linear_bytes": lin_bytes, "linear_flops": lin_flops, "bwd_bytes": bwd_bytes, "elem_bytes": b}
 
 
 def load_peaks():
@@ -119,6 +125,7 @@ KERNEL_HEADERS = {
     "route_kernel": ["route.cuh"],
     "linear_umma_kernel": ["linear.cuh"],
     "linear_f32_kernel": ["linear.cuh"],
+    "bwd_kernels": ["backward.cuh"],
 }
 
 
@@ -271,9 +278,16 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- reference arm
 
-def oracle_step(w: synth.Workload, sample: synth.Workload, layer: bool):
-    """One call of the oracle on `sample` (the BRA forward, or the whole layer)."""
+def oracle_step(w: synth.Workload, sample: synth.Workload, layer: bool, backward: bool = False):
+    """One call of the oracle on `sample` (the BRA forward, the whole layer, or the backward
+    for the forward's routing)."""
     import oracle
+    if backward:
+        from oracle import backward as ob
+        inp = {k: v.astype(np.float64) for k, v in synth.make_inputs(sample).items()}
+        dout = synth.make_inputs(sample, seed_base=0xB0D0 + sample.index)["q"].astype(np.float64)
+        r_idx, _ = oracle.route(inp["q"], inp["k"], w.heads, w.S, w.topk)
+        return lambda: ob.backward(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], w.heads, w.S, r_idx, dout)
     if layer:
         inp = {k: v.astype(np.float64) for k, v in synth.make_layer_inputs(sample).items()}
         keys = ("x", "w_qkv", "b_qkv", "w_o", "b_o", "lce_w", "lce_b")
@@ -288,7 +302,7 @@ def bench_reference(args, w: synth.Workload, rank: int):
     if rank != 0:
         return None
     sample = w.with_(N=1)
-    step = oracle_step(w, sample, args.layer)
+    step = oracle_step(w, sample, args.layer, args.backward)
 
     for _ in range(args.warmup):
         step()
@@ -299,7 +313,8 @@ def bench_reference(args, w: synth.Workload, rank: int):
     value = sample.tokens * args.steps / dt
     cores = oracle.threads()
     line = {
-        "impl": "reference", "metric": METRIC_LAYER if args.layer else METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
+        "impl": "reference", "metric": METRIC_BWD if args.backward else (METRIC_LAYER if args.layer else METRIC),
+        "value": value, "unit": "tokens/s", "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1), BiFormer stage shape)",
@@ -312,12 +327,12 @@ def bench_reference(args, w: synth.Workload, rank: int):
     return line
 
 
-def cpu_baseline(w: synth.Workload, budget_s: float = 12.0, layer: bool = False):
+def cpu_baseline(w: synth.Workload, budget_s: float = 12.0, layer: bool = False, backward: bool = False):
     """The oracle as it stands on a bounded sample: whole images (at most 8), repeated
     until about `budget_s` seconds of host time are used (at least once)."""
     import oracle
     sample = w.with_(N=max(1, min(w.N, 8)))
-    step = oracle_step(w, sample, layer)
+    step = oracle_step(w, sample, layer, backward)
     reps, t0 = 0, time.perf_counter()
     while True:
         step()
@@ -326,7 +341,8 @@ def cpu_baseline(w: synth.Workload, budget_s: float = 12.0, layer: bool = False)
         if dt > budget_s:
             break
     return {"value": sample.tokens * reps / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": "%d x %s of %d images (%d tokens), %.1f s" % (reps, "layer" if layer else "forward",
+            "sample": "%d x %s of %d images (%d tokens), %.1f s" % (reps, "backward" if backward else
+                                                                   ("layer" if layer else "forward"),
                                                                    sample.N, sample.tokens, dt)}
 
 
@@ -372,27 +388,39 @@ def main():
 
     # inputs: this rank's own batch (weak scaling); seeded per rank
     seed = None if rank == 0 else 0xB1F0 + 16 * w.index + 1000 * rank
-    layer = args.layer
+    layer, backward = args.layer, args.backward
     inp = synth.make_layer_inputs(w, seed_base=seed) if layer else synth.make_inputs(w, seed_base=seed)
+    if backward:  # dL/dout: another seeded map of the same shape, stored in the dtype
+        inp["dout"] = synth.make_inputs(w, seed_base=0xB0D0 + w.index + 1000 * rank)["q"]
     base = {k: torch.from_numpy(v).to(dev).to(tdt).contiguous() for k, v in inp.items()}
     lead = "x" if layer else "q"  # the (N,H,W,C) input whose shape the output takes
+    if backward:  # the forward's routing, computed once on the device
+        _, r0, _ = bra.forward(base["q"], base["k"], base["v"], base["lce_w"], base["lce_b"], w.heads, w.S, w.topk)
+        base["r_idx"] = r0
+        torch.cuda.synchronize(dev)
     # bytes of one input set plus its output (the layer's q, k, v and attention output
     # are the library's scratch, produced and consumed inside the step)
     set_bytes = (2 if layer else 4) * w.tokens * w.C * acc["elem_bytes"]
+    if backward:
+        set_bytes = 5 * w.tokens * w.C * acc["elem_bytes"] + 3 * w.tokens * w.C * 4
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     n_sets = max(2, math.ceil(3 * l2 / set_bytes))
     sets = []
     for _ in range(n_sets):
         s = {k: v.clone() for k, v in base.items()}
         s["out"] = torch.empty_like(base[lead])
-        s["r_idx"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.int32, device=dev)
+        if not backward:  # the backward reads the forward's routing (copied with the set)
+            s["r_idx"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.int32, device=dev)
         s["r_w"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.float32, device=dev)
         sets.append(s)
 
     stream = torch.cuda.Stream(device=dev)
 
     def fwd(s):
-        if layer:
+        if backward:
+            s["grads"] = bra.backward(s["q"], s["k"], s["v"], s["lce_w"], s["r_idx"], s["dout"], w.heads, w.S,
+                                      stream=stream)
+        elif layer:
             bra.attention_layer(s["x"], s["w_qkv"], s["b_qkv"], s["w_o"], s["b_o"], s["lce_w"], s["lce_b"],
                                 w.heads, w.S, w.topk, out=s["out"], r_idx=s["r_idx"], r_weight=s["r_w"],
                                 stream=stream)
@@ -406,7 +434,7 @@ def main():
     with torch.cuda.stream(stream):
         fwd(sets[0])  # first call outside capture: lazy module load, pool init
     stream.synchronize()
-    if not args.no_graph:
+    if not args.no_graph and not backward:  # bra_backward synchronises: direct launches
         for s in sets:
             g = torch.cuda.CUDAGraph()
             c0 = bra.launch_count()
@@ -457,27 +485,35 @@ def main():
     # replayed for at least K steps, and the pairs are read after every round.
     torch.cuda.synchronize(dev)
     bra.trace_begin()
-    traced = []
-    with torch.cuda.stream(stream):
-        for s_ in sets:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                fwd(s_)
-            traced.append(g)
     trace = {}
-    rounds = max(1, math.ceil(args.steps / n_sets))
-    for _ in range(rounds):
+    if backward:
         with torch.cuda.stream(stream):
-            for g in traced:
-                g.replay()
+            for i in range(args.steps):
+                fwd(sets[i % n_sets])
         torch.cuda.synchronize(dev)
-        for k_, (t_ms, t_n) in bra.trace_read().items():
-            a_ = trace.setdefault(k_, [0.0, 0])
-            a_[0] += t_ms
-            a_[1] += t_n
+        trace = {k_: [t_ms, t_n] for k_, (t_ms, t_n) in bra.trace_read().items()}
+        traced_steps = args.steps
+    else:
+        traced = []
+        with torch.cuda.stream(stream):
+            for s_ in sets:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    fwd(s_)
+                traced.append(g)
+        rounds = max(1, math.ceil(args.steps / n_sets))
+        for _ in range(rounds):
+            with torch.cuda.stream(stream):
+                for g in traced:
+                    g.replay()
+            torch.cuda.synchronize(dev)
+            for k_, (t_ms, t_n) in bra.trace_read().items():
+                a_ = trace.setdefault(k_, [0.0, 0])
+                a_[0] += t_ms
+                a_[1] += t_n
+        del traced
+        traced_steps = rounds * n_sets
     bra.trace_end()
-    del traced
-    traced_steps = rounds * n_sets
     clocks.stop()
 
     # ---- end to end through the public API from pinned host memory: the host-buffer
@@ -488,9 +524,20 @@ def main():
     h_idx = torch.empty((w.N, w.regions, w.topk), dtype=torch.int32).pin_memory()
     h_w = torch.empty((w.N, w.regions, w.topk), dtype=torch.float32).pin_memory()
     d_in = sets[0]
+    if backward:
+        host = {k: v.cpu().pin_memory() for k, v in base.items()}
+        h_grads = {k: torch.empty(v.shape, dtype=torch.float32).pin_memory() for k, v in sets[0]["grads"].items()}
 
     def e2e_step():
-        if layer:
+        if backward:
+            with torch.cuda.stream(stream):
+                for k_, v_ in host.items():
+                    d_in[k_].copy_(v_, non_blocking=True)
+                fwd(d_in)
+                for k_, t_ in d_in["grads"].items():
+                    h_grads[k_].copy_(t_, non_blocking=True)
+            stream.synchronize()
+        elif layer:
             with torch.cuda.stream(stream):
                 for k_, v_ in host.items():
                     d_in[k_].copy_(v_, non_blocking=True)
@@ -520,6 +567,8 @@ def main():
         e2e_ms = float(t.item())
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = h_out.numel() * h_out.element_size() + h_idx.numel() * 4 + h_w.numel() * 4
+    if backward:
+        d2h = sum(t.numel() * 4 for t in h_grads.values())
 
     if rank != 0:
         if world > 1:
@@ -540,6 +589,9 @@ def main():
     alg_bytes = {"bra_image_kernel": acc["fused_bytes"], "region_mean_kernel": acc["pool_bytes"],
                  "route_kernel": acc["route_bytes"], "linear_umma_kernel": acc["linear_bytes"],
                  "linear_f32_kernel": acc["linear_bytes"]}.get(attn_name, acc["attn_bytes"])
+    if backward:  # the backward's three kernels form one traced class: time per call
+        attn_s = t_ms / max(traced_steps, 1) / 1e3
+        alg_bytes = acc["bwd_bytes"]
     step_traced_ms = sum(v[0] for v in trace.values()) / traced_steps
     share = {k: round(v[0] / max(1e-12, sum(x[0] for x in trace.values())), 4) for k, v in trace.items() if v[1]}
     achieved = alg_bytes / attn_s / 1e9
@@ -550,7 +602,8 @@ def main():
     t_gath = acc["gathered_bytes"] / (peaks["hbm_gbs"] * 1e9)
     ns_bound = "tensor" if t_flop > t_gath else "hbm"
     line = {
-        "metric": METRIC_LAYER if layer else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC_BWD if backward else (METRIC_LAYER if layer else METRIC), "value": value,
+        "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
@@ -561,8 +614,9 @@ def main():
                          % (n_sets, set_bytes / 1e6, n_sets * set_bytes / 1e6, l2 / 1e6),
                    "launch": "CUDA graph per step" if graphs else "direct launches",
                    "attention_kernel": args.variant,
-                   "step": "bra_attention_layer (qkv projection, BRA, output projection)" if layer
-                           else "bra_forward",
+                   "step": "bra_backward (routing detached, the forward's r_idx)" if backward else
+                           ("bra_attention_layer (qkv projection, BRA, output projection)" if layer
+                            else "bra_forward"),
                    "parallelism": "dp%d (independent images, no collective)" % world},
         "tflops": tflops,
         "gpu_launches": gpu_launches,
@@ -581,11 +635,15 @@ def main():
         "clocks": clocks.summary(),
         "e2e": {"value": tokens_all * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-                "entry": "bra_attention_layer with stream copies (pinned host buffers)" if layer
-                         else "bra_forward_host (pinned host buffers)"},
+                "entry": "bra_backward with stream copies (pinned host buffers)" if backward else
+                         ("bra_attention_layer with stream copies (pinned host buffers)" if layer
+                          else "bra_forward_host (pinned host buffers)")},
     }
+    if backward:  # the forward's FLOP accounting does not describe this step
+        line.pop("tflops")
+        line.pop("roofline_gathered")
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, layer=layer)
+        line["cpu_baseline"] = cpu_baseline(w, layer=layer, backward=backward)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
