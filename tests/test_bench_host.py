@@ -72,3 +72,21 @@ def test_source_hash_ignores_comments_only(bench):
     assert bench.strip_comments(src) == 'int a = 1;\n const char *s = "x // kept"; char q = \'/\';\n  int b;'
     assert bench.strip_comments(src.replace("// note", "// other note")) == bench.strip_comments(src)
     assert bench.strip_comments(src.replace("int b;", "int c;")) != bench.strip_comments(src)
+
+
+def test_algorithmic_figures_of_the_layer_and_the_backward(bench):
+    """Bytes per launch of the projections (the mean of the qkv and output launches) and
+    per call of the backward, written out from their tensors' sizes."""
+    from vision_transformer_sparse_b200 import synth
+    w = synth.WORKLOADS["cls_stage2_224"]
+    acc = bench.algorithmic(w)
+    T, C, b = w.tokens, w.C, 2
+    qkv = T * C * b + 3 * C * C * b + 3 * T * C * b      # x, w_qkv read; q, k, v written
+    wo = T * C * b + C * C * b + T * C * b               # o, w_o read; out written
+    assert acc["linear_bytes"] == (qkv + wo) / 2
+    assert acc["linear_flops"] == 2 * T * C * 3 * C + 2 * T * C * C
+    bwd = (4 * T * C * b                                 # q, k, v, dout read
+           + 3 * T * C * 4                               # dq, dk, dv written (float32)
+           + w.N * w.regions * w.topk * 4                # r_idx
+           + C * 25 * b + C * 25 * 4 + C * 4)            # lce_w read; dlce_w, dlce_b written
+    assert acc["bwd_bytes"] == bwd
