@@ -99,3 +99,43 @@ def test_two_rank_layer_split_equals_full_batch(tmp_path):
     mp.spawn(_rank_main, args=(2, _free_port(), result, True), nprocs=2, join=True)
     with open(result) as f:
         assert f.read() == "ok"
+
+
+def _rank_backward(rank, world, port, result_path):
+    """Data-parallel backward: each rank takes its images; the per-image gradients (dq, dk,
+    dv) are concatenated, the LCE parameter gradients (sums over the batch) all-reduced."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from oracle import backward as ob
+        inp = synth.make_inputs(W)
+        dout = synth.make_inputs(W, seed_base=0xB0D0)["q"]
+        r_idx, _ = oracle.route(inp["q"], inp["k"], W.heads, W.S, W.topk)
+        a, b = shard(W.N, world, rank)
+        g = ob.backward(*(inp[k][a:b] for k in ("q", "k", "v")), inp["lce_w"], inp["lce_b"], W.heads, W.S,
+                        r_idx[a:b], dout[a:b])
+        for name in ("dlce_w", "dlce_b"):
+            t = torch.from_numpy(g[name].copy())
+            dist.all_reduce(t, op=dist.ReduceOp.SUM)
+            g[name] = t.numpy()
+        parts = [None] * world
+        dist.all_gather_object(parts, {k: g[k] for k in ("dq", "dk", "dv")})
+        if rank == 0:
+            full = ob.backward(inp["q"], inp["k"], inp["v"], inp["lce_w"], inp["lce_b"], W.heads, W.S, r_idx, dout)
+            ok = all(np.allclose(np.concatenate([p[k] for p in parts]), full[k], rtol=1e-12, atol=1e-12)
+                     for k in ("dq", "dk", "dv"))
+            ok = ok and all(np.allclose(g[k], full[k], rtol=1e-12, atol=1e-12) for k in ("dlce_w", "dlce_b"))
+            with open(result_path, "w") as f:
+                f.write("ok" if ok else "mismatch")
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_two_rank_backward_shards_and_all_reduces_parameter_gradients(tmp_path):
+    result = str(tmp_path / "result.txt")
+    mp.spawn(_rank_backward, args=(2, _free_port(), result), nprocs=2, join=True)
+    with open(result) as f:
+        assert f.read() == "ok"
