@@ -42,7 +42,7 @@ struct BwdParams {
     float scale;
 };
 
-#ifdef BRA_BWD_HOST_CHECK
+#if defined(BRA_BWD_HOST_CHECK) && !defined(__CUDA_ARCH__)  // the host pass of a host-check build
 void bra_bwd_host_bounds_failure(const char *what, long long i, long long n);
 #define BRA_BWD_CHECK(what, i, n) \
     do { if ((long long)(i) < 0 || (long long)(i) >= (long long)(n)) bra_bwd_host_bounds_failure(what, (i), (n)); } while (0)
