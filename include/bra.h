@@ -126,13 +126,16 @@ int bra_forward_host(const void *q, const void *k, const void *v, const void *lc
  * library: BRA_STATIC_SCRATCH_FLOATS floats (16 MiB), present on every GPU that
  * loads the library and held until the process exits. It calls no allocator.
  *
- *   - Same arguments, layouts, results and error codes as bra_forward; the
- *     caller still passes (and owns) every input and output buffer.
- *   - Limit: 2*N*S*S*C must not exceed BRA_STATIC_SCRATCH_FLOATS; a larger
- *     problem returns BRA_ERR_SCRATCH before anything is launched.
- *   - The first call on each device looks up the array's device address on that
- *     device (it must be the current device, as for every call); make that first
- *     call before any CUDA graph capture starts on the device.
+ *   - Same arguments, layouts and error codes as bra_forward, and the same
+ *     kernels: the results are bit for bit those of bra_forward on the same
+ *     inputs. The caller still passes (and owns) every input and output buffer.
+ *   - Limit: 2*N*S*S*C must not exceed BRA_STATIC_SCRATCH_FLOATS, even for shapes
+ *     whose one-kernel form needs no scratch; a larger problem returns
+ *     BRA_ERR_SCRATCH before anything is launched.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, no allocation). The first call on a device may load
+ *     the library's kernels onto it, so make that first call before any CUDA
+ *     graph capture starts on the device.
  *   - All calls share the one array, which keeps the last call's contents. No
  *     part of it needs to start at zero: a call writes every element it reads.
  *     Two calls whose kernels overlap on the GPU (different streams, or

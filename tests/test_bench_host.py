@@ -90,3 +90,20 @@ def test_algorithmic_figures_of_the_layer_and_the_backward(bench):
            + w.N * w.regions * w.topk * 4                # r_idx
            + C * 25 * b + C * 25 * 4 + C * 4)            # lce_w read; dlce_w, dlce_b written
     assert acc["bwd_bytes"] == bwd
+
+
+def test_method_roofline_picks_the_slower_term(bench):
+    """The detection stage is bound by its FLOPs at the burst bf16 peak, the classification
+    stage by its gathered K/V bytes at HBM bandwidth; frac = roofline time / kernel time."""
+    from vision_transformer_sparse_b200 import synth
+    peaks = {"hbm_gbs": 6540.8, "bf16_tflops": 1645.8, "bf16_tflops_sustained": 1369.4}
+    det = bench.algorithmic(synth.WORKLOADS["det_stage1_1024"])
+    r = bench.method_roofline(det, peaks, 20e-6)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == 1645.8
+    t_flop = det["flops"] / 1645.8e12
+    assert abs(r["frac"] - t_flop / 20e-6) < 1e-12
+    assert abs(r["roofline_us"] - t_flop * 1e6) < 1e-9
+    cls = bench.algorithmic(synth.WORKLOADS["cls_stage2_224"])
+    r = bench.method_roofline(cls, peaks, 50e-6)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["frac"] - cls["gathered_bytes"] / 6540.8e9 / 50e-6) < 1e-12

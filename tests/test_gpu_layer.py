@@ -5,7 +5,8 @@ Tolerances: a projection result rounded to bfloat16 is within half an ulp of its
 float32-accumulated value (2^-8 relative) plus the accumulation error, bounded here by
 1e-4 times sum |x||w| + |b| (float32: 1e-5 times the same sum). The layer is checked by
 oracle.compare.check_layer (routing set-exact off near ties, output within the forward's
-tolerance)."""
+tolerance); its r_weight is also checked within the forward's 1e-5 against the oracle's
+routing of the q and k the GPU stored (read back through bra_qkv)."""
 import numpy as np
 import pytest
 import torch
@@ -111,6 +112,19 @@ LAYER = [
 ]
 
 
+def check_routing_of_stored_qk(inp, heads, S, topk, dtype, r_idx, r_w):
+    """The layer's routing is the routing of the q and k it stored: the oracle's float64
+    routing of the GPU's own q and k (from bra_qkv, the same projection kernel) must give
+    the layer's r_idx (set-exact off near ties) and r_weight within the forward's 1e-5."""
+    q, k, _ = bra.qkv(dev(inp["x"], dtype), dev(inp["w_qkv"], dtype), dev(inp["b_qkv"], dtype))
+    torch.cuda.synchronize()
+    qh, kh = host(q), host(k)
+    ref_idx, ref_w, logits = oracle.route(qh, kh, heads, S, topk, with_logits=True)
+    rep = compare.Report()
+    compare.check_routing(logits, ref_idx, ref_w, r_idx, r_w, rep, tol_weight=compare.TOL_WEIGHT)
+    assert rep.ok, rep.notes[:2000]
+
+
 @pytest.mark.parametrize("N,H,W,C,heads,S,topk,dtype", LAYER)
 def test_layer_matches_oracle(N, H, W, C, heads, S, topk, dtype):
     w = synth.Workload("layer_case", 40 + C + topk, N, H, W, C, heads, S, topk, dtype, lce_b_std=0.01)
@@ -118,6 +132,7 @@ def test_layer_matches_oracle(N, H, W, C, heads, S, topk, dtype):
     out, r_idx, r_w = run_layer(inp, heads, S, topk, dtype)
     rep = compare.check_layer(inp, heads, S, topk, dtype, out, r_idx, r_w)
     assert rep.ok, rep.notes
+    check_routing_of_stored_qk(inp, heads, S, topk, dtype, r_idx, r_w)
 
 
 @pytest.mark.parametrize("name", ["cls_stage2_224", "det_stage1_1024", "stage1_tiny_224"])
@@ -128,3 +143,4 @@ def test_layer_full_workload(name):
     out, r_idx, r_w = run_layer(inp, w.heads, w.S, w.topk, w.dtype)
     rep = compare.check_layer(inp, w.heads, w.S, w.topk, w.dtype, out, r_idx, r_w)
     assert rep.ok, rep.notes
+    check_routing_of_stored_qk(inp, w.heads, w.S, w.topk, w.dtype, r_idx, r_w)

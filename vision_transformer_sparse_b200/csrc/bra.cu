@@ -1401,25 +1401,18 @@ int bra_forward_host(const void *q, const void *k, const void *v, const void *lc
 // bra_forward_noalloc keeps its scratch (the pooled region means of q and k) in
 // this file-scope device array instead of the memory pool. Host code must not
 // pass the symbol itself to a kernel: on the host it names a host-side shadow,
-// so the device address is looked up once per device with cudaGetSymbolAddress.
+// so the device address is looked up with cudaGetSymbolAddress on the current
+// device. The lookup is repeated on every call (it is cheap once the module is
+// loaded) rather than cached, so that a context created anew on the device (after
+// cudaDeviceReset) never receives an address from the old one.
 
 static __device__ __align__(256) float g_static_scratch[BRA_STATIC_SCRATCH_FLOATS];
 
-static constexpr int kMaxDevices = 64;
-static std::mutex g_static_mu;
-static float *g_static_ptr[kMaxDevices] = {};
-
-// Device address of g_static_scratch on the current device (looked up on first use).
+// Device address of g_static_scratch on the current device.
 static int static_scratch(float **out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BRA_ERR_CUDA;
-    std::lock_guard<std::mutex> g(g_static_mu);
-    if (!g_static_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return BRA_ERR_CUDA;
-        g_static_ptr[dev] = static_cast<float *>(p);
-    }
-    *out = g_static_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return BRA_ERR_CUDA;
+    *out = static_cast<float *>(p);
     return BRA_OK;
 }
 
@@ -1440,10 +1433,9 @@ int bra_forward_noalloc(const void *q, const void *k, const void *v, const void 
     float *ws = nullptr;
     rc = static_scratch(&ws);
     if (rc) return rc;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    rc = launch_route_into(s, q, k, r_idx, r_weight, ws, st);
-    if (rc) return rc;
-    return launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, nullptr, st);
+    // the same kernels as bra_forward (the one-kernel fused forms use no scratch at all),
+    // with the static array standing in for the pool's scratch
+    return forward_device(s, q, k, v, lce_w, lce_b, out, r_idx, r_weight, reinterpret_cast<cudaStream_t>(stream), ws);
 }
 
 }  // extern "C"

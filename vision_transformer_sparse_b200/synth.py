@@ -95,7 +95,8 @@ WORKLOADS: Dict[str, Workload] = {
     ]
 }
 
-BENCH_WORKLOAD = "cls_stage2_224"
+# the benchmark default: the largest single-GPU workload (most tokens and attention FLOPs)
+BENCH_WORKLOAD = "det_stage1_1024"
 
 
 def round_bf16(x: np.ndarray) -> np.ndarray:
