@@ -33,6 +33,17 @@
  * all heads; r_weight is returned only and does not weight K/V; ties in the
  * top-k go to the lower region index.
  *
+ * H or W not divisible by S: the bernice.tw notes (section "消融實驗") say that
+ * padding the feature map costs compute, which is why S is chosen per task; the
+ * pages define no padding further. Reading taken: q, k and v are zero-padded at
+ * the bottom and the right to Hp = S*ceil(H/S), Wp = S*ceil(W/S); region means
+ * are taken over the whole padded region (hr*wr tokens, the padding included as
+ * zeros); padded tokens take part as keys (k = 0, v = 0, so their score is 0);
+ * outputs are produced for the H x W real pixels only (the padding is cropped).
+ * LCE(V) of a real pixel is unchanged by the padding, since the padded values
+ * are the same zeros as the convolution's own border. When S divides H and W
+ * every formula below reduces to the unpadded one.
+ *
  * Layouts: q, k, v, out are (N,H,W,C) channels-last float64; lce_w is (C,5,5);
  * lce_b is (C); r_idx is int32 (N,S*S,topk); r_weight is (N,S*S,topk);
  * logits is (N,S*S,S*S). Channel of head m, component c is m*d + c.
@@ -65,22 +76,25 @@ void oracle_set_threads(int t)
 #endif
 }
 
-/* 0 if the shape is one BRA defines: H and W divisible by S (the assert of the
- * walk-through), C divisible by heads, 1 <= topk <= S*S. */
+/* 0 if the shape is one BRA defines: C divisible by heads, 1 <= topk <= S*S
+ * (H and W need not be multiples of S: see the padding reading above). */
 int oracle_check_shape(int N, int H, int W, int C, int heads, int S, int topk)
 {
     if (N < 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0 || S <= 0) return 1;
-    if (H % S != 0 || W % S != 0) return 1;
     if (C % heads != 0) return 1;
     if (topk < 1 || topk > S * S) return 1;
     return 0;
 }
 
-/* Step 2: per-region mean over the region's hr*wr tokens, every channel.
- * x (N,H,W,C) -> xr (N,S*S,C). */
+/* Region height and width of the (padded) grid: ceil(H/S), ceil(W/S). */
+static int region_extent(int H, int S) { return (H + S - 1) / S; }
+
+/* Step 2: per-region mean over the region's hr*wr tokens, every channel; tokens
+ * of the zero padding (row >= H or column >= W) add nothing to the sum but count
+ * in the divisor. x (N,H,W,C) -> xr (N,S*S,C). */
 void oracle_region_mean(const double *x, int N, int H, int W, int C, int S, double *xr)
 {
-    const int hr = H / S, wr = W / S;
+    const int hr = region_extent(H, S), wr = region_extent(W, S);
     for (int n = 0; n < N; ++n)
         for (int j = 0; j < S; ++j)
             for (int i = 0; i < S; ++i) {
@@ -88,8 +102,10 @@ void oracle_region_mean(const double *x, int N, int H, int W, int C, int S, doub
                 for (int c = 0; c < C; ++c) {
                     double sum = 0.0;
                     for (int h = 0; h < hr; ++h)
-                        for (int w = 0; w < wr; ++w)
-                            sum += x[IDX4(n, j * hr + h, i * wr + w, c, H, W, C)];
+                        for (int w = 0; w < wr; ++w) {
+                            const int y = j * hr + h, xx = i * wr + w;
+                            if (y < H && xx < W) sum += x[IDX4(n, y, xx, c, H, W, C)];
+                        }
                     xr[((size_t)n * S * S + p) * C + c] = sum / (double)(hr * wr);
                 }
             }
@@ -182,7 +198,7 @@ int oracle_attend(const double *q, const double *k, const double *v, const doubl
                   const int32_t *r_idx, double *out)
 {
     if (oracle_check_shape(N, H, W, C, heads, S, topk)) return 1;
-    const int P = S * S, hr = H / S, wr = W / S, w2 = hr * wr, d = C / heads;
+    const int P = S * S, hr = region_extent(H, S), wr = region_extent(W, S), w2 = hr * wr, d = C / heads;
     const int L = topk * w2; /* keys per query */
     for (size_t e = 0; e < (size_t)N * P * topk; ++e)
         if (r_idx[e] < 0 || r_idx[e] >= P) return 2;
@@ -211,13 +227,16 @@ int oracle_attend(const double *q, const double *k, const double *v, const doubl
                 const int j = p / S, i = p % S;
                 for (int t = 0; t < w2; ++t) {
                     const int y = j * hr + t / wr, x = i * wr + t % wr;
+                    if (y >= H || x >= W) continue; /* a padded query: cropped */
                     for (int m = 0; m < heads; ++m) {
                         double smax = -INFINITY;
                         for (int l = 0; l < L; ++l) {
+                            /* a padded key has k = 0: its score is 0 */
                             double dot = 0.0;
-                            for (int c = 0; c < d; ++c)
-                                dot += (scale * q[IDX4(n, y, x, m * d + c, H, W, C)]) *
-                                       k[IDX4(n, ky[l], kx[l], m * d + c, H, W, C)];
+                            if (ky[l] < H && kx[l] < W)
+                                for (int c = 0; c < d; ++c)
+                                    dot += (scale * q[IDX4(n, y, x, m * d + c, H, W, C)]) *
+                                           k[IDX4(n, ky[l], kx[l], m * d + c, H, W, C)];
                             s[l] = dot;
                             if (dot > smax) smax = dot;
                         }
@@ -228,8 +247,9 @@ int oracle_attend(const double *q, const double *k, const double *v, const doubl
                         }
                         for (int c = 0; c < d; ++c) {
                             double o = 0.0;
-                            for (int l = 0; l < L; ++l)
-                                o += (s[l] / z) * v[IDX4(n, ky[l], kx[l], m * d + c, H, W, C)];
+                            for (int l = 0; l < L; ++l) /* a padded key has v = 0 */
+                                if (ky[l] < H && kx[l] < W)
+                                    o += (s[l] / z) * v[IDX4(n, ky[l], kx[l], m * d + c, H, W, C)];
                             const size_t oi = IDX4(n, y, x, m * d + c, H, W, C);
                             out[oi] = o + lepe[oi];
                         }
