@@ -8,7 +8,8 @@
  * ("Bi-Level Routing Attention", parts one to three):
  *
  *   1. patchify: the (N,H,W,C) map is cut into S x S regions of
- *      hr x wr = (H/S) x (W/S) tokens; region p = j*S + i is region row j,
+ *      hr x wr = (H/S) x (W/S) tokens (padded grid below when S does not
+ *      divide H or W); region p = j*S + i is region row j,
  *      region column i; tokens inside a region are row-major;
  *   2. region query/key = mean of the region's tokens over all C channels;
  *      affinity A[p][p'] = (scale * q_r[p]) . k_r[p']                     (eq. 4)
@@ -43,9 +44,19 @@
  *     nothing is launched and a BRA_ERR_* code is returned. BRA_ERR_CUDA reports
  *     a failed allocation or launch (the CUDA error is left for the caller to
  *     inspect with cudaGetLastError()). No C++ exception crosses this boundary.
- *   - Supported shapes: H % S == 0, W % S == 0, 1 <= S*S <= 256,
- *     1 <= topk <= S*S, C % heads == 0, d in {32, 64}, C <= 1024,
- *     W/S <= 128. N may be 0 (nothing is launched; pointers may be NULL).
+ *   - Supported shapes: 1 <= S*S <= 256, 1 <= topk <= S*S, C % heads == 0,
+ *     d in {32, 64}, C <= 1024, ceil(W/S) <= 128. N may be 0 (nothing is
+ *     launched; pointers may be NULL).
+ *   - H or W not a multiple of S (the padded grid; the bernice.tw notes, section
+ *     "消融實驗", name padding's cost as the reason S is chosen per task and define
+ *     it no further): q, k and v are zero-padded at the bottom and the right to
+ *     Hp = S*ceil(H/S), Wp = S*ceil(W/S); regions are ceil(H/S) x ceil(W/S)
+ *     tokens; region means are taken over whole padded regions; padded tokens
+ *     take part as keys (k = v = 0); out holds the H x W real pixels only. The
+ *     library makes the padded copies in scratch taken like the pooled means
+ *     (3*N*Hp*Wp*C elements for q, k, v plus N*Hp*Wp*C for the padded output)
+ *     and crops the result into `out`. With H and W multiples of S nothing of
+ *     this happens.
  *   - Alignment: q, k, v, out 16-byte aligned; r_idx, r_weight 4-byte aligned.
  */
 #ifndef BRA_H
@@ -131,7 +142,9 @@ int bra_forward_host(const void *q, const void *k, const void *v, const void *lc
  *     inputs. The caller still passes (and owns) every input and output buffer.
  *   - Limit: 2*N*S*S*C must not exceed BRA_STATIC_SCRATCH_FLOATS, even for shapes
  *     whose one-kernel form needs no scratch; a larger problem returns
- *     BRA_ERR_SCRATCH before anything is launched.
+ *     BRA_ERR_SCRATCH before anything is launched. So does a shape whose H or W
+ *     is not a multiple of S: its padded copies would need more scratch than the
+ *     array holds.
  *   - Every call looks up the array's device address on the current device
  *     (cudaGetSymbolAddress, no allocation). The first call on a device may load
  *     the library's kernels onto it, so make that first call before any CUDA
@@ -185,6 +198,46 @@ int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, con
                         int topk, int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * The BiFormer block around the attention layer, as the walk-through prints and runs it
+ * ("BiFormer ... 前向传播过程", section "2、BiFormer Block": x = x + pos_embed(x), then
+ * x = x + drop_path(attn(norm1(x))); the module printout of section "网络结构":
+ * pos_embed = Conv2d(C, C, 3, padding 1, groups C), norm1 / norm2 = LayerNorm(C,
+ * eps 1e-6), mlp = Linear(C, 3C) -> GELU -> Linear(3C, C), drop_path = Identity). The
+ * walk-through says nothing of the MLP line; it is read as the same pre-norm residual
+ * form, x = x + mlp(norm2(x)), with PyTorch's default (exact erf) GELU. */
+
+/* The MLP's linear layers: y (M x Nout) = act(x w^T + b) with x (M x K), w (Nout, K),
+ * b (Nout), all in `dtype`, float32 accumulation:
+ *   BRA_ACT_NONE:     y = round(x w^T + b)                   (as bra_linear)
+ *   BRA_ACT_GELU:     y = round(GELU(x w^T + b)), GELU(t) = t/2 (1 + erf(t / sqrt 2))
+ *   BRA_ACT_RESIDUAL: y = round(res + round(x w^T + b)), res (M x Nout) in `dtype`
+ * round = the dtype's rounding (nearest even for bf16; none for float32). Shape and
+ * alignment rules of bra_linear; res (when used) 16-byte aligned. */
+enum { BRA_ACT_NONE = 0, BRA_ACT_GELU = 1, BRA_ACT_RESIDUAL = 2 };
+int bra_linear_act(const void *x, const void *w, const void *b, const void *res, int M, int K, int Nout, int act,
+                   int dtype, void *y, bra_stream_t stream);
+
+/* One block: x, out (N,H,W,C) in `dtype`;
+ *   x1 = x + pos_embed(x)        pos_w (C,3,3), pos_b (C): depthwise 3x3 cross-correlation,
+ *                                zero padding 1, plus bias
+ *   h  = norm1(x1)               ln1_g, ln1_b (C): (t - mean) / sqrt(var + 1e-6) * g + b over
+ *                                the C channels of a pixel, var the mean squared deviation
+ *   x2 = x1 + attn(h)            the attention layer (bra_attention_layer's weights)
+ *   out = x2 + mlp(norm2(x2))    ln2_g, ln2_b (C); mlp_w1 (3C, C), mlp_b1 (3C), GELU,
+ *                                mlp_w2 (C, 3C), mlp_b2 (C)
+ * Every stored intermediate (x1, h, the layer's own, x2, norm2's output, the MLP hidden
+ * layer after GELU, the MLP output before the residual) is rounded once to `dtype`.
+ * r_idx, r_weight: the attention's routing, as in bra_forward. Shapes: BRA's rules (the
+ * padded grid included) and the projections', with C <= 256. x, out, w_qkv, w_o, mlp_w1,
+ * mlp_w2 16-byte aligned; the other parameters aligned to their element. Scratch
+ * (7*N*H*W*C elements plus the attention layer's) is taken like bra_attention_layer's. */
+int bra_block(const void *x, const void *pos_w, const void *pos_b, const void *ln1_g, const void *ln1_b,
+              const void *w_qkv, const void *b_qkv, const void *w_o, const void *b_o, const void *lce_w,
+              const void *lce_b, const void *ln2_g, const void *ln2_b, const void *mlp_w1, const void *mlp_b1,
+              const void *mlp_w2, const void *mlp_b2, int N, int H, int W, int C, int heads, int S, int topk,
+              int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * The backward pass of steps 4-5 with the routing detached: the walk-through's router
  * ("BiFormer ... 前向传播过程", section "BRA模块", TopkRouting) detaches the region
  * query and key when diff_routing is off (its default); the top-k index is discrete and
@@ -195,7 +248,8 @@ int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, con
  * and so the last bits, can differ between calls). The attention softmax is recomputed
  * from q and k. Every r_idx entry must lie in [0, S*S): an entry outside is skipped and
  * the call returns BRA_ERR_INDEX; like bra_attend, this call synchronises `stream` to
- * read that flag. Shapes as bra_forward; q, k, v, dout, lce_w aligned to their element,
+ * read that flag. Shapes as bra_forward, with H and W multiples of S (no padded grid:
+ * BRA_ERR_SHAPE otherwise); q, k, v, dout, lce_w aligned to their element,
  * the float32 outputs and r_idx to 4 bytes. N = 0 zeroes dlce_w and dlce_b only.
  * Plain SIMT kernels: a first, correct form of this step, not yet tuned. */
 int bra_backward(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
@@ -216,7 +270,9 @@ enum {
     BRA_KERNEL_LINEAR_BF16 = 6, /* qkv / output projection, tcgen05 GEMM          */
     BRA_KERNEL_LINEAR_F32 = 7,  /* qkv / output projection, float32 SIMT          */
     BRA_KERNEL_BACKWARD = 8,    /* bra_backward's kernels, timed together          */
-    BRA_KERNEL_CLASSES = 9
+    BRA_KERNEL_PAD = 9,         /* padded grid: zero-padded copies and the crop   */
+    BRA_KERNEL_BLOCK = 10,      /* BiFormer block: pos-embed + LN1, residual + LN2 */
+    BRA_KERNEL_CLASSES = 11
 };
 
 /* Number of kernels this library has launched since it was loaded (all threads,

@@ -41,8 +41,6 @@ def fwd(shape, ptrs=None):
 
 
 @pytest.mark.parametrize("shape,code", [
-    ((1, 57, 56, 64, 2, 7, 1, 1), 2),    # H % S
-    ((1, 56, 50, 64, 2, 7, 1, 1), 2),    # W % S
     ((1, 56, 56, 64, 3, 7, 1, 1), 2),    # C % heads
     ((1, 56, 56, 96, 2, 7, 1, 1), 2),    # d = 48
     ((1, 56, 56, 64, 2, 7, 0, 1), 2),    # topk = 0
@@ -52,6 +50,7 @@ def fwd(shape, ptrs=None):
     ((-1, 56, 56, 64, 2, 7, 1, 1), 2),   # N < 0
     ((1, 56, 56, 64, 2, 7, 1, 7), 4),    # dtype
     ((1, 1032, 1032, 64, 2, 4, 1, 1), 2),  # region wider than 128
+    ((1, 64, 1025, 64, 2, 8, 1, 1), 2),    # padded region wider than 128 (ceil(1025/8) = 129)
 ])
 def test_bad_shapes_rejected(bra_lib, shape, code):
     assert fwd(shape) == code
@@ -129,7 +128,6 @@ def test_qkv_rejects_before_cuda(bra_lib):
 
 
 @pytest.mark.parametrize("shape,code", [
-    ((1, 57, 56, 64, 2, 7, 1, 1), 2),    # H % S
     ((1, 56, 56, 96, 2, 7, 1, 1), 2),    # d = 48
     ((1, 56, 56, 64, 2, 7, 50, 1), 2),   # topk > S^2
     ((1, 56, 56, 64, 2, 7, 1, 7), 4),    # dtype
@@ -168,3 +166,23 @@ def test_backward_rejects_before_cuda(bra_lib):
         ptrs = [FAKE] * 11
         ptrs[i] = ctypes.c_void_p(0x10002)
         assert call(ptrs) == 3
+
+
+@pytest.mark.parametrize("shape", [
+    (0, 57, 56, 64, 2, 7, 1, 1),     # H not a multiple of S
+    (0, 56, 50, 64, 2, 7, 1, 1),     # W not a multiple of S
+    (0, 30, 30, 64, 2, 7, 3, 1),     # a whole region row and column of padding
+    (0, 250, 250, 64, 2, 16, 1, 1),  # 250 -> 256: the padded grid of 16 x 16 regions
+])
+def test_padded_grid_shapes_accepted(bra_lib, shape):
+    """H or W not a multiple of S is the padded grid: accepted by every forward entry
+    point (N = 0 launches nothing), refused by the no-allocation entry point (its static
+    array cannot hold the padded copies) and by the backward."""
+    assert fwd(shape, [None] * 8) == 0
+    assert bra.raw_call("bra_route", None, None, *shape, None, None, None) == 0
+    assert bra.raw_call("bra_attend", *[None] * 5, *shape, None, None, None) == 0
+    assert bra.raw_call("bra_forward_host", *[None] * 5, *shape, *[None] * 3, None) == 0
+    assert bra.raw_call("bra_attention_layer", *[None] * 7, *shape, *[None] * 3, None) == 0
+    one = (1,) + shape[1:]
+    assert bra.raw_call("bra_forward_noalloc", *[FAKE] * 5, *one, *[FAKE] * 3, None) == 7
+    assert bra.raw_call("bra_backward", *[FAKE] * 6, *one, *[FAKE] * 5, None) == 2

@@ -27,8 +27,9 @@ SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_fo
            "bra_status_string",
            "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name",
            "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout", "bra_trace_read",
-           "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward")
-KERNEL_CLASSES = 9
+           "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward", "bra_linear_act", "bra_block")
+ACT_NONE, ACT_GELU, ACT_RESIDUAL = 0, 1, 2
+KERNEL_CLASSES = 11
 
 
 class BraError(RuntimeError):
@@ -55,8 +56,11 @@ def lib() -> ctypes.CDLL:
         L.bra_qkv.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
         L.bra_attention_layer.argtypes = [vp] * 7 + shape + [vp, vp, vp, vp]
         L.bra_backward.argtypes = [vp] * 6 + shape + [vp] * 6
+        L.bra_linear_act.argtypes = [vp] * 4 + [i] * 5 + [vp, vp]
+        L.bra_block.argtypes = [vp] * 17 + shape + [vp, vp, vp, vp]
         for f in ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
-                  "bra_version", "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward"):
+                  "bra_version", "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward",
+                  "bra_linear_act", "bra_block"):
             getattr(L, f).restype = i
         L.bra_status_string.argtypes = [i]
         L.bra_status_string.restype = ctypes.c_char_p
@@ -135,6 +139,39 @@ def linear(x, w, b, out=None, stream=None) -> torch.Tensor:
     rc = lib().bra_linear(_ptr(x), _ptr(w), _ptr(b), M, K, Nout, _dtype_code(x), _ptr(out), _stream(stream))
     _raise(rc, "bra_linear")
     return out
+
+
+def linear_act(x, w, b, act: int, res=None, out=None, stream=None) -> torch.Tensor:
+    """bra_linear_act: act(x w^T + b) for act ACT_NONE / ACT_GELU, or res + (x w^T + b) for
+    ACT_RESIDUAL (res of the output's shape)."""
+    K = x.shape[-1]
+    Nout = w.shape[0]
+    M = x.numel() // K if K else 0
+    out = torch.empty(x.shape[:-1] + (Nout,), dtype=x.dtype, device=x.device) if out is None else out
+    _check_dev(*(t for t in (x, w, b, res, out) if t is not None))
+    rc = lib().bra_linear_act(_ptr(x), _ptr(w), _ptr(b), _ptr(res) if res is not None else None, M, K, Nout, act,
+                              _dtype_code(x), _ptr(out), _stream(stream))
+    _raise(rc, "bra_linear_act")
+    return out
+
+
+BLOCK_PARAMS = ("pos_w", "pos_b", "ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o", "lce_w", "lce_b", "ln2_g",
+                "ln2_b", "mlp_w1", "mlp_b1", "mlp_w2", "mlp_b2")
+
+
+def block(x, p: dict, heads: int, S: int, topk: int, out=None, r_idx=None, r_weight=None, stream=None):
+    """bra_block: one BiFormer block (pos-embed, norm1, attention layer, norm2, MLP, residuals)
+    on x (N,H,W,C); p maps BLOCK_PARAMS names to device tensors."""
+    N, H, W, C = x.shape
+    P = S * S
+    out = torch.empty_like(x) if out is None else out
+    r_idx = torch.empty((N, P, topk), dtype=torch.int32, device=x.device) if r_idx is None else r_idx
+    r_weight = torch.empty((N, P, topk), dtype=torch.float32, device=x.device) if r_weight is None else r_weight
+    _check_dev(x, *(p[k] for k in BLOCK_PARAMS), out, r_idx, r_weight)
+    rc = lib().bra_block(_ptr(x), *(_ptr(p[k]) for k in BLOCK_PARAMS), N, H, W, C, heads, S, topk, _dtype_code(x),
+                         _ptr(out), _ptr(r_idx), _ptr(r_weight), _stream(stream))
+    _raise(rc, "bra_block")
+    return out, r_idx, r_weight
 
 
 def qkv(x, w_qkv, b_qkv, q=None, k=None, v=None, stream=None):

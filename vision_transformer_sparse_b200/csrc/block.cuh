@@ -1,0 +1,205 @@
+// block.cuh — the BiFormer block's per-pixel steps around the attention layer and the MLP
+// GEMMs: the positional embedding with its residual, and the two pre-norm LayerNorms.
+//
+// Source: "BiFormer ... 前向传播过程" (niftyadmin), section "2、BiFormer Block" (the block's
+// forward: x = x + pos_embed(x), then x = x + drop_path(attn(norm1(x)))) and the module
+// printout of section "网络结构": pos_embed = Conv2d(C, C, 3, padding 1, groups C) (with its
+// bias), norm1 / norm2 = LayerNorm(C, eps 1e-6), mlp = Linear(C, 3C) -> GELU ->
+// Linear(3C, C), drop_path = Identity. The MLP line is read as the same pre-norm residual
+// form, x = x + mlp(norm2(x)).
+//
+//   pos_ln_kernel:  x1 = x + b + dwconv3x3(x)  (zero pad 1)   -> stored;  h = LN1(x1) -> stored
+//   add_ln_kernel:  x2 = x1 + a                                -> stored;  h = LN2(x2) -> stored
+//
+// LayerNorm: (x - mean) / sqrt(var + 1e-6) * gamma + beta over the C channels of a pixel,
+// var the mean squared deviation (two passes over registers). Arithmetic in float32; every
+// stored value is rounded once to the storage type, and each LayerNorm reads the rounded
+// value that was stored (as a bf16 model stores its activations).
+//
+// One warp per pixel (pixels in warp-strided order, so that neighbouring warps read
+// neighbouring pixels and the 3x3 taps hit L1): lane l owns channel pairs l, l + 32, ...
+// (NP of them, C <= 64 * NP), whose weights it keeps in registers; loads and stores are
+// whole pairs (bf16x2 or float2), so a warp moves one pixel's channels contiguously.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+namespace bra {
+
+constexpr int kBlockThreads = 256;
+
+struct BlockParams {
+    const void *x;       // pos_ln: the block input; add_ln: x1
+    const void *a;       // add_ln: the attention layer's output
+    const void *pos_w;   // (C, 3, 3)
+    const void *pos_b;   // (C)
+    const void *ln_g;    // (C)
+    const void *ln_b;    // (C)
+    void *xo;            // x1 (pos_ln) or x2 (add_ln)
+    void *h;             // the LayerNorm output
+    long long pixels;    // N * H * W
+    int H, W, C;
+};
+
+template <typename T> struct PairIO;
+template <> struct PairIO<__nv_bfloat16> {
+    static __device__ __forceinline__ float2 ld(const void *p, size_t pair) {
+        const uint32_t u = __ldg(static_cast<const unsigned int *>(p) + pair);
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+    }
+    static __device__ __forceinline__ float2 round(float2 v) {
+        return make_float2(__bfloat162float(__float2bfloat16_rn(v.x)), __bfloat162float(__float2bfloat16_rn(v.y)));
+    }
+    static __device__ __forceinline__ void st(void *p, size_t pair, float2 v) {  // v already representable
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+        static_cast<__nv_bfloat162 *>(p)[pair] = h;
+    }
+};
+template <> struct PairIO<float> {
+    static __device__ __forceinline__ float2 ld(const void *p, size_t pair) {
+        return __ldg(static_cast<const float2 *>(p) + pair);
+    }
+    static __device__ __forceinline__ float2 round(float2 v) { return v; }
+    static __device__ __forceinline__ void st(void *p, size_t pair, float2 v) { static_cast<float2 *>(p)[pair] = v; }
+};
+
+// One parameter element (weights and per-channel vectors need only element alignment).
+template <typename T> __device__ __forceinline__ float ld_elem(const void *p, int i) {
+    if constexpr (sizeof(T) == 2)
+        return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+    else
+        return static_cast<const float *>(p)[i];
+}
+template <typename T> __device__ __forceinline__ float2 ld_pair_elems(const void *p, int cp) {
+    return make_float2(ld_elem<T>(p, 2 * cp), ld_elem<T>(p, 2 * cp + 1));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// LayerNorm of one pixel whose channel pairs v[j] (pair lane + 32 j, valid while < C/2)
+// sit in the warp's registers; writes the rounded result.
+template <typename T, int NP>
+__device__ __forceinline__ void ln_store(const float2 (&v)[NP], const float2 (&g)[NP], const float2 (&b)[NP],
+                                         int lane, int pairs, int C, void *out, size_t pix_pair0) {
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+        if (lane + 32 * j < pairs) s += v[j].x + v[j].y;
+    const float mean = warp_sum(s) / (float)C;
+    float q = 0.f;
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+        if (lane + 32 * j < pairs) {
+            const float dx = v[j].x - mean, dy = v[j].y - mean;
+            q = fmaf(dx, dx, fmaf(dy, dy, q));
+        }
+    const float rstd = rsqrtf(warp_sum(q) / (float)C + 1e-6f);
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int cp = lane + 32 * j;
+        if (cp < pairs) {
+            const float2 o = make_float2(fmaf((v[j].x - mean) * rstd, g[j].x, b[j].x),
+                                         fmaf((v[j].y - mean) * rstd, g[j].y, b[j].y));
+            PairIO<T>::st(out, pix_pair0 + cp, PairIO<T>::round(o));
+        }
+    }
+}
+
+template <typename T, int NP>
+__global__ void __launch_bounds__(kBlockThreads) pos_ln_kernel(const BlockParams p) {
+    const int lane = threadIdx.x & 31;
+    const int pairs = p.C >> 1;
+    float2 w[NP][9], bias[NP], g[NP], bb[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int cp = lane + 32 * j;
+        const bool ok = cp < pairs;
+        const int c = 2 * cp;
+#pragma unroll
+        for (int t = 0; t < 9; ++t)  // weights (C,3,3): channel c's tap t at c * 9 + t
+            w[j][t] = ok ? make_float2(ld_elem<T>(p.pos_w, c * 9 + t), ld_elem<T>(p.pos_w, (c + 1) * 9 + t))
+                         : make_float2(0.f, 0.f);
+        bias[j] = ok ? ld_pair_elems<T>(p.pos_b, cp) : make_float2(0.f, 0.f);
+        g[j] = ok ? ld_pair_elems<T>(p.ln_g, cp) : make_float2(0.f, 0.f);
+        bb[j] = ok ? ld_pair_elems<T>(p.ln_b, cp) : make_float2(0.f, 0.f);
+    }
+    const long long warps = (long long)gridDim.x * (kBlockThreads / 32);
+    for (long long pix = (long long)blockIdx.x * (kBlockThreads / 32) + (threadIdx.x >> 5); pix < p.pixels;
+         pix += warps) {
+        const int xx = (int)(pix % p.W);
+        const long long rowi = pix / p.W;
+        const int yy = (int)(rowi % p.H);
+        float2 acc[NP];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) acc[j] = bias[j];
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            const int y2 = yy + a - 1;
+            if (y2 < 0 || y2 >= p.H) continue;
+#pragma unroll
+            for (int e = 0; e < 3; ++e) {
+                const int x2 = xx + e - 1;
+                if (x2 < 0 || x2 >= p.W) continue;
+                const size_t q0 = (size_t)(pix + (long long)(a - 1) * p.W + (e - 1)) * pairs;
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    const int cp = lane + 32 * j;
+                    if (cp < pairs) {
+                        const float2 v = PairIO<T>::ld(p.x, q0 + cp);
+                        acc[j].x = fmaf(w[j][3 * a + e].x, v.x, acc[j].x);
+                        acc[j].y = fmaf(w[j][3 * a + e].y, v.y, acc[j].y);
+                        if (a == 1 && e == 1) {  // the residual: x itself
+                            acc[j].x += v.x;
+                            acc[j].y += v.y;
+                        }
+                    }
+                }
+            }
+        }
+        const size_t q0 = (size_t)pix * pairs;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            acc[j] = PairIO<T>::round(acc[j]);
+            if (lane + 32 * j < pairs) PairIO<T>::st(p.xo, q0 + lane + 32 * j, acc[j]);
+        }
+        ln_store<T, NP>(acc, g, bb, lane, pairs, p.C, p.h, q0);
+    }
+}
+
+template <typename T, int NP>
+__global__ void __launch_bounds__(kBlockThreads) add_ln_kernel(const BlockParams p) {
+    const int lane = threadIdx.x & 31;
+    const int pairs = p.C >> 1;
+    float2 g[NP], bb[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int cp = lane + 32 * j;
+        g[j] = cp < pairs ? ld_pair_elems<T>(p.ln_g, cp) : make_float2(0.f, 0.f);
+        bb[j] = cp < pairs ? ld_pair_elems<T>(p.ln_b, cp) : make_float2(0.f, 0.f);
+    }
+    const long long warps = (long long)gridDim.x * (kBlockThreads / 32);
+    for (long long pix = (long long)blockIdx.x * (kBlockThreads / 32) + (threadIdx.x >> 5); pix < p.pixels;
+         pix += warps) {
+        const size_t q0 = (size_t)pix * pairs;
+        float2 v[NP];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            const int cp = lane + 32 * j;
+            v[j] = make_float2(0.f, 0.f);
+            if (cp < pairs) {
+                const float2 x1 = PairIO<T>::ld(p.x, q0 + cp), a = PairIO<T>::ld(p.a, q0 + cp);
+                v[j] = PairIO<T>::round(make_float2(x1.x + a.x, x1.y + a.y));
+                PairIO<T>::st(p.xo, q0 + cp, v[j]);
+            }
+        }
+        ln_store<T, NP>(v, g, bb, lane, pairs, p.C, p.h, q0);
+    }
+}
+
+}  // namespace bra

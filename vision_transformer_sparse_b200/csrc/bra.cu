@@ -34,8 +34,10 @@
 #include "attn_tma.cuh"
 #include "attn_umma.cuh"
 #include "backward.cuh"
+#include "block.cuh"
 #include "fused_image.cuh"
 #include "linear.cuh"
+#include "pad.cuh"
 #include "route.cuh"
 
 namespace bra {
@@ -95,6 +97,8 @@ class LaunchScope {
 struct Shape {
     int N, H, W, C, heads, S, topk, dtype;
     int P, hr, wr, w2, d;
+    int Hp, Wp;  // the padded grid: S * hr, S * wr (== H, W when S divides them)
+    bool padded() const { return Hp != H || Wp != W; }
 };
 
 static bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -103,28 +107,39 @@ static bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintp
 static int check_shape(const Shape &s) {
     if (s.dtype != BRA_F32 && s.dtype != BRA_BF16) return BRA_ERR_DTYPE;
     if (s.N < 0 || s.H <= 0 || s.W <= 0 || s.C <= 0 || s.heads <= 0 || s.S <= 0) return BRA_ERR_SHAPE;
-    if (s.S > 16 || s.H % s.S != 0 || s.W % s.S != 0) return BRA_ERR_SHAPE;
+    if (s.S > 16) return BRA_ERR_SHAPE;
     if (s.topk < 1 || s.topk > s.S * s.S) return BRA_ERR_SHAPE;
     if (s.C % s.heads != 0 || s.C > 1024) return BRA_ERR_SHAPE;
     const int d = s.C / s.heads;
     if (d != 32 && d != 64) return BRA_ERR_SHAPE;
-    if (s.W / s.S > 128) return BRA_ERR_SHAPE;
-    // element offsets are formed in 64-bit; grid sizes must fit in int
-    if ((long long)s.N * s.S * s.S * s.H > INT_MAX) return BRA_ERR_SHAPE;
-    if ((long long)s.H * s.W > INT_MAX / 4) return BRA_ERR_SHAPE;
+    if (s.wr > 128) return BRA_ERR_SHAPE;
+    // element offsets are formed in 64-bit; grid sizes (the padded copies: one CTA per
+    // row of three maps) must fit in int
+    if ((long long)s.N * s.S * s.S * s.Hp > INT_MAX / 3) return BRA_ERR_SHAPE;
+    if ((long long)s.Hp * s.Wp > INT_MAX / 4) return BRA_ERR_SHAPE;
     return BRA_OK;
 }
 
 static Shape make_shape(int N, int H, int W, int C, int heads, int S, int topk, int dtype) {
-    Shape s{N, H, W, C, heads, S, topk, dtype, 0, 0, 0, 0, 0};
-    if (S > 0 && heads > 0) {
+    Shape s{N, H, W, C, heads, S, topk, dtype, 0, 0, 0, 0, 0, H, W};
+    if (S > 0 && heads > 0 && H > 0 && W > 0) {
         s.P = S * S;
-        s.hr = H / S;
-        s.wr = W / S;
+        s.hr = (H + S - 1) / S;  // ceil: the padded grid when S does not divide H
+        s.wr = (W + S - 1) / S;
         s.w2 = s.hr * s.wr;
         s.d = C / heads;
+        s.Hp = S * s.hr;
+        s.Wp = S * s.wr;
     }
     return s;
+}
+
+// The same problem on the zero-padded maps (Hp x Wp), which S divides.
+static Shape padded_shape(const Shape &s) {
+    Shape p = s;
+    p.H = s.Hp;
+    p.W = s.Wp;
+    return p;
 }
 
 static int largest_divisor_at_most(int n, int cap) {
@@ -913,7 +928,7 @@ static int check_linear(int M, int K, int Nout, int nsplit, int dtype) {
 
 // y[i] (M x Nout/nsplit, row-major) = column block i of x w^T + b.
 static int launch_linear(const void *x, const void *w, const void *b, int M, int K, int Nout, int nsplit,
-                         void *const *y, int dtype, cudaStream_t st) {
+                         void *const *y, int dtype, cudaStream_t st, int epi = kEpiBias, const void *res = nullptr) {
     if (M == 0) return BRA_OK;
     const int ny = Nout / nsplit;
     if (dtype == BRA_F32) {
@@ -921,6 +936,8 @@ static int launch_linear(const void *x, const void *w, const void *b, int M, int
         p.x = static_cast<const float *>(x);
         p.w = static_cast<const float *>(w);
         p.b = static_cast<const float *>(b);
+        p.res = static_cast<const float *>(res);
+        p.epi = epi;
         for (int i = 0; i < 3; ++i) p.y[i] = static_cast<float *>(y[i < nsplit ? i : 0]);
         p.M = M;
         p.K = K;
@@ -940,6 +957,8 @@ static int launch_linear(const void *x, const void *w, const void *b, int M, int
     for (int i = 0; i < nsplit; ++i)
         if (!encode_map_rows(&p.tmY[i], y[i], M, ny, 32)) return BRA_ERR_CUDA;
     p.bias = static_cast<const __nv_bfloat16 *>(b);
+    p.res = static_cast<const __nv_bfloat16 *>(res);
+    p.epi = epi;
     p.M = M;
     p.K = K;
     p.Nout = Nout;
@@ -987,10 +1006,79 @@ static int launch_linear(const void *x, const void *w, const void *b, int M, int
 static int check_plan(const Shape &s) {
     int rc = check_shape(s);
     if (rc) return rc;
+    const Shape sp = padded_shape(s);  // the kernels run on the padded grid
     AttnParams p{};
     int t, m;
-    if (s.dtype == BRA_BF16 ? !plan_bf16(s, p, t, m) : !plan_f32(s, p, t, m)) return BRA_ERR_SHAPE;
+    if (sp.dtype == BRA_BF16 ? !plan_bf16(sp, p, t, m) : !plan_f32(sp, p, t, m)) return BRA_ERR_SHAPE;
     return BRA_OK;
+}
+
+// ----------------------------------------------------------------------------- padded grid
+
+// Zero-padded copies of up to three (N,H,W,C) maps into (N,Hp,Wp,C) buffers.
+static int launch_pad(const Shape &s, int nmaps, const void *const *src, void *const *dst, cudaStream_t st) {
+    PadParams p{};
+    for (int i = 0; i < nmaps; ++i) {
+        p.src[i] = static_cast<const uint4 *>(src[i]);
+        p.dst[i] = static_cast<uint4 *>(dst[i]);
+    }
+    p.N = s.N;
+    p.H = s.H;
+    p.W = s.W;
+    p.Hp = s.Hp;
+    p.Wp = s.Wp;
+    p.cv = s.C * (s.dtype == BRA_BF16 ? 2 : 4) / 16;
+    LaunchScope ls(BRA_KERNEL_PAD, st);
+    pad_maps_kernel<<<(unsigned)(nmaps * s.N * s.Hp), kPadThreads, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
+// The H x W real pixels of a padded (N,Hp,Wp,C) map into out (N,H,W,C).
+static int launch_crop(const Shape &s, const void *src, void *out, cudaStream_t st) {
+    LaunchScope ls(BRA_KERNEL_PAD, st);
+    crop_map_kernel<<<(unsigned)(s.N * s.H), kPadThreads, 0, st>>>(
+        static_cast<const uint4 *>(src), static_cast<uint4 *>(out), s.H, s.W, s.Hp, s.Wp,
+        s.C * (s.dtype == BRA_BF16 ? 2 : 4) / 16);
+    return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------------- BiFormer block
+
+// The block's per-pixel kernels (pos-embed + LN1, residual + LN2), C <= 256.
+template <typename T>
+static int launch_block_pixels(bool pos, const BlockParams &p, cudaStream_t st) {
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc) return rc;
+    const long long want = (p.pixels + kBlockThreads / 32 - 1) / (kBlockThreads / 32);
+    const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(want, (long long)sms * 8));
+    const int np = (p.C + 63) / 64;
+    LaunchScope ls(BRA_KERNEL_BLOCK, st);
+    switch (np) {
+#define BRA_BLOCK_CASE(NP)                                                                         \
+    case NP:                                                                                       \
+        if (pos)                                                                                   \
+            pos_ln_kernel<T, NP><<<grid, kBlockThreads, 0, st>>>(p);                               \
+        else                                                                                       \
+            add_ln_kernel<T, NP><<<grid, kBlockThreads, 0, st>>>(p);                               \
+        break;
+        BRA_BLOCK_CASE(1)
+        BRA_BLOCK_CASE(2)
+        BRA_BLOCK_CASE(3)
+        BRA_BLOCK_CASE(4)
+#undef BRA_BLOCK_CASE
+        default: return BRA_ERR_SHAPE;
+    }
+    return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
+static int launch_block(bool pos, int dtype, const BlockParams &p, cudaStream_t st) {
+    return dtype == BRA_BF16 ? launch_block_pixels<__nv_bfloat16>(pos, p, st) : launch_block_pixels<float>(pos, p, st);
+}
+
+// Bytes of one padded (N,Hp,Wp,C) map, rounded up to 256.
+static size_t padded_map_bytes(const Shape &s) {
+    return ((size_t)s.N * s.Hp * s.Wp * s.C * (s.dtype == BRA_BF16 ? 2 : 4) + 255) / 256 * 256;
 }
 
 }  // namespace bra
@@ -1086,6 +1174,8 @@ const char *bra_kernel_name(int kernel_class) {
         case BRA_KERNEL_LINEAR_BF16: return "linear_umma_kernel";
         case BRA_KERNEL_LINEAR_F32: return "linear_f32_kernel";
         case BRA_KERNEL_BACKWARD: return "bwd_kernels";
+        case BRA_KERNEL_PAD: return "pad_crop_kernels";
+        case BRA_KERNEL_BLOCK: return "block_pixel_kernels";
         default: return "unknown";
     }
 }
@@ -1094,7 +1184,7 @@ const char *bra_status_string(int status) {
     switch (status) {
         case BRA_OK: return "ok";
         case BRA_ERR_NULL: return "a required pointer is NULL";
-        case BRA_ERR_SHAPE: return "unsupported shape (H%S, W%S, C%heads, topk, S*S<=256, d in {32,64}, C<=1024, W/S<=128)";
+        case BRA_ERR_SHAPE: return "unsupported shape (C%heads, topk, S*S<=256, d in {32,64}, C<=1024, ceil(W/S)<=128; bra_backward: H%S, W%S)";
         case BRA_ERR_ALIGN: return "pointer misaligned (q, k, v, out need 16 bytes; r_idx, r_weight 4)";
         case BRA_ERR_DTYPE: return "dtype must be BRA_F32 or BRA_BF16";
         case BRA_ERR_CUDA: return "a CUDA allocation, copy or kernel launch failed";
@@ -1114,11 +1204,20 @@ int bra_route(const void *q, const void *k, int N, int H, int W, int C, int head
     if (!q || !k || !r_idx || !r_weight) return BRA_ERR_NULL;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(r_idx, 4) || !aligned(r_weight, 4)) return BRA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    float *ws = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), 2 * (size_t)N * s.P * C * sizeof(float), st) != cudaSuccess)
-        return BRA_ERR_CUDA;
-    rc = launch_route_into(s, q, k, r_idx, r_weight, ws, st);
-    if (cudaFreeAsync(ws, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    const size_t pooled = 2 * (size_t)N * s.P * C * sizeof(float);
+    const size_t map = s.padded() ? padded_map_bytes(s) : 0;  // padded grid: copies of q, k
+    unsigned char *buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&buf), pooled + 2 * map, st) != cudaSuccess) return BRA_ERR_CUDA;
+    float *ws = reinterpret_cast<float *>(buf + 2 * map);
+    if (s.padded()) {
+        const void *src[2] = {q, k};
+        void *dst[2] = {buf, buf + map};
+        rc = launch_pad(s, 2, src, dst, st);
+        if (rc == BRA_OK) rc = launch_route_into(padded_shape(s), dst[0], dst[1], r_idx, r_weight, ws, st);
+    } else {
+        rc = launch_route_into(s, q, k, r_idx, r_weight, ws, st);
+    }
+    if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     return rc;
 }
 
@@ -1130,6 +1229,21 @@ int bra_route(const void *q, const void *k, int N, int H, int W, int C, int head
 static int forward_device(const Shape &s, const void *q, const void *k, const void *v, const void *lce_w,
                           const void *lce_b, void *out, int32_t *r_idx, float *r_weight, cudaStream_t st,
                           float *ws_given = nullptr) {
+    if (s.padded()) {
+        // the padded grid: zero-padded copies of q, k, v, the forward on them, the crop
+        const size_t map = padded_map_bytes(s);
+        unsigned char *buf = nullptr;
+        if (cudaMallocAsync(reinterpret_cast<void **>(&buf), 4 * map, st) != cudaSuccess) return BRA_ERR_CUDA;
+        const void *src[3] = {q, k, v};
+        void *dst[3] = {buf, buf + map, buf + 2 * map};
+        int rc = launch_pad(s, 3, src, dst, st);
+        if (rc == BRA_OK)
+            rc = forward_device(padded_shape(s), dst[0], dst[1], dst[2], lce_w, lce_b, buf + 3 * map, r_idx, r_weight,
+                                st, ws_given);
+        if (rc == BRA_OK) rc = launch_crop(s, buf + 3 * map, out, st);
+        if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+        return rc;
+    }
     bool fused = false;
     const bool routed = fused_routed(s) && fused_image_shape_ok(s, lce_w, lce_b);
     if (!routed) {
@@ -1190,6 +1304,45 @@ int bra_qkv(const void *x, const void *w_qkv, const void *b_qkv, int M, int C, i
     return launch_linear(x, w_qkv, b_qkv, M, C, 3 * C, 3, ys, dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Layer scratch: q, k, v and the attention output (one map each), then the pooled means.
+static size_t map_bytes(const Shape &s) {
+    return ((size_t)s.N * s.H * s.W * s.C * (s.dtype == BRA_BF16 ? 2 : 4) + 255) / 256 * 256;
+}
+static size_t layer_scratch_bytes(const Shape &s) { return 4 * map_bytes(s) + 2 * (size_t)s.N * s.P * s.C * 4; }
+
+// qkv projection -> BRA forward -> output projection, on caller scratch of
+// layer_scratch_bytes(s).
+static int layer_device(const Shape &s, const void *x, const void *w_qkv, const void *b_qkv, const void *w_o,
+                        const void *b_o, const void *lce_w, const void *lce_b, void *out, int32_t *r_idx,
+                        float *r_weight, cudaStream_t st, unsigned char *buf) {
+    const int T = s.N * s.H * s.W;
+    const size_t plane = map_bytes(s);
+    void *qkv[3] = {buf, buf + plane, buf + 2 * plane};
+    void *o = buf + 3 * plane;
+    float *ws = reinterpret_cast<float *>(buf + 4 * plane);
+    int rc = launch_linear(x, w_qkv, b_qkv, T, s.C, 3 * s.C, 3, qkv, s.dtype, st);
+    if (rc == BRA_OK) rc = forward_device(s, qkv[0], qkv[1], qkv[2], lce_w, lce_b, o, r_idx, r_weight, st, ws);
+    if (rc == BRA_OK) rc = launch_linear(o, w_o, b_o, T, s.C, s.C, 1, &out, s.dtype, st);
+    return rc;
+}
+
+// Scratch of `bytes` taken stream-ordered: outside a stream capture from the library's
+// per-device pool that keeps its memory between calls (mapping tens of MB again on every
+// call costs milliseconds); inside one, from the default pool (a memory node of the graph).
+static int scratch_alloc(unsigned char **buf, size_t bytes, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return BRA_ERR_CUDA;
+    if (cs == cudaStreamCaptureStatusNone) {
+        cudaMemPool_t pool = nullptr;
+        cudaStream_t up = nullptr, back = nullptr;
+        int rc = host_call_pool(&pool, &up, &back);
+        if (rc) return rc;
+        return cudaMallocFromPoolAsync(reinterpret_cast<void **>(buf), bytes, pool, st) == cudaSuccess ? BRA_OK
+                                                                                                      : BRA_ERR_CUDA;
+    }
+    return cudaMallocAsync(reinterpret_cast<void **>(buf), bytes, st) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
 int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, const void *w_o, const void *b_o,
                         const void *lce_w, const void *lce_b, int N, int H, int W, int C, int heads, int S,
                         int topk, int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream) {
@@ -1208,29 +1361,90 @@ int bra_attention_layer(const void *x, const void *w_qkv, const void *b_qkv, con
         !aligned(r_weight, 4))
         return BRA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const size_t plane = ((size_t)T * C * es + 255) / 256 * 256;  // one (N,H,W,C) tensor
-    const size_t route = 2 * (size_t)N * s.P * C * sizeof(float);
-    // outside a stream capture the scratch comes from the library's pool that keeps its
-    // memory between calls (mapping tens of MB again on every call costs milliseconds);
-    // inside one, from the default pool (a memory node of the graph)
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return BRA_ERR_CUDA;
     unsigned char *buf = nullptr;
-    if (cs == cudaStreamCaptureStatusNone) {
-        cudaMemPool_t pool = nullptr;
-        cudaStream_t up = nullptr, back = nullptr;
-        if ((rc = host_call_pool(&pool, &up, &back))) return rc;
-        if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&buf), 4 * plane + route, pool, st) != cudaSuccess)
-            return BRA_ERR_CUDA;
-    } else if (cudaMallocAsync(reinterpret_cast<void **>(&buf), 4 * plane + route, st) != cudaSuccess) {
-        return BRA_ERR_CUDA;
+    if ((rc = scratch_alloc(&buf, layer_scratch_bytes(s), st))) return rc;
+    rc = layer_device(s, x, w_qkv, b_qkv, w_o, b_o, lce_w, lce_b, out, r_idx, r_weight, st, buf);
+    if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    return rc;
+}
+
+int bra_linear_act(const void *x, const void *w, const void *b, const void *res, int M, int K, int Nout, int act,
+                   int dtype, void *y, bra_stream_t stream) {
+    int rc = check_linear(M, K, Nout, 1, dtype);
+    if (rc) return rc;
+    if (act != BRA_ACT_NONE && act != BRA_ACT_GELU && act != BRA_ACT_RESIDUAL) return BRA_ERR_SHAPE;
+    if (M == 0) return BRA_OK;
+    if (!x || !w || !b || !y || (act == BRA_ACT_RESIDUAL && !res)) return BRA_ERR_NULL;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 16) || !aligned(b, es) ||
+        (act == BRA_ACT_RESIDUAL && !aligned(res, 16)))
+        return BRA_ERR_ALIGN;
+    void *ys[1] = {y};
+    return launch_linear(x, w, b, M, K, Nout, 1, ys, dtype, reinterpret_cast<cudaStream_t>(stream), act, res);
+}
+
+int bra_block(const void *x, const void *pos_w, const void *pos_b, const void *ln1_g, const void *ln1_b,
+              const void *w_qkv, const void *b_qkv, const void *w_o, const void *b_o, const void *lce_w,
+              const void *lce_b, const void *ln2_g, const void *ln2_b, const void *mlp_w1, const void *mlp_b1,
+              const void *mlp_w2, const void *mlp_b2, int N, int H, int W, int C, int heads, int S, int topk,
+              int dtype, void *out, int32_t *r_idx, float *r_weight, bra_stream_t stream) {
+    const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
+    int rc = check_plan(s);
+    if (rc) return rc;
+    if (C > 256) return BRA_ERR_SHAPE;
+    const long long T = (long long)N * H * W;
+    if (T > INT_MAX) return BRA_ERR_SHAPE;
+    if ((rc = check_linear((int)T, C, 3 * C, 3, dtype)) || (rc = check_linear((int)T, C, C, 1, dtype)) ||
+        (rc = check_linear((int)T, C, 3 * C, 1, dtype)) || (rc = check_linear((int)T, 3 * C, C, 1, dtype)))
+        return rc;
+    if (N == 0) return BRA_OK;
+    const void *params[] = {pos_w, pos_b, ln1_g, ln1_b, b_qkv, b_o, lce_w, lce_b, ln2_g, ln2_b, mlp_b1, mlp_b2};
+    for (const void *q : params)
+        if (!q) return BRA_ERR_NULL;
+    if (!x || !w_qkv || !w_o || !mlp_w1 || !mlp_w2 || !out || !r_idx || !r_weight) return BRA_ERR_NULL;
+    const size_t es = dtype == BRA_BF16 ? 2 : 4;
+    for (const void *q : params)
+        if (!aligned(q, es)) return BRA_ERR_ALIGN;
+    if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(w_o, 16) || !aligned(mlp_w1, 16) ||
+        !aligned(mlp_w2, 16) || !aligned(out, 16) || !aligned(r_idx, 4) || !aligned(r_weight, 4))
+        return BRA_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t plane = map_bytes(s);
+    // x1, h (reused for h2), a, x2, the MLP hidden layer (three planes), the layer's scratch
+    unsigned char *buf = nullptr;
+    if ((rc = scratch_alloc(&buf, 7 * plane + layer_scratch_bytes(s), st))) return rc;
+    unsigned char *x1 = buf, *h = buf + plane, *a = buf + 2 * plane, *x2 = buf + 3 * plane, *m = buf + 4 * plane;
+    unsigned char *lbuf = buf + 7 * plane;
+    BlockParams bp{};
+    bp.pixels = T;
+    bp.H = H;
+    bp.W = W;
+    bp.C = C;
+    // x1 = x + pos_embed(x), h = norm1(x1)
+    bp.x = x;
+    bp.pos_w = pos_w;
+    bp.pos_b = pos_b;
+    bp.ln_g = ln1_g;
+    bp.ln_b = ln1_b;
+    bp.xo = x1;
+    bp.h = h;
+    rc = launch_block(true, dtype, bp, st);
+    // a = attn(h)
+    if (rc == BRA_OK) rc = layer_device(s, h, w_qkv, b_qkv, w_o, b_o, lce_w, lce_b, a, r_idx, r_weight, st, lbuf);
+    // x2 = x1 + a, h = norm2(x2)
+    if (rc == BRA_OK) {
+        bp.x = x1;
+        bp.a = a;
+        bp.ln_g = ln2_g;
+        bp.ln_b = ln2_b;
+        bp.xo = x2;
+        bp.h = h;
+        rc = launch_block(false, dtype, bp, st);
     }
-    void *qkv[3] = {buf, buf + plane, buf + 2 * plane};
-    void *o = buf + 3 * plane;
-    float *ws = reinterpret_cast<float *>(buf + 4 * plane);
-    rc = launch_linear(x, w_qkv, b_qkv, (int)T, C, 3 * C, 3, qkv, dtype, st);
-    if (rc == BRA_OK) rc = forward_device(s, qkv[0], qkv[1], qkv[2], lce_w, lce_b, o, r_idx, r_weight, st, ws);
-    if (rc == BRA_OK) rc = launch_linear(o, w_o, b_o, (int)T, C, C, 1, &out, dtype, st);
+    // out = x2 + mlp(h): Linear(C, 3C) + GELU, then Linear(3C, C) with the residual
+    void *mp[1] = {m}, *op[1] = {out};
+    if (rc == BRA_OK) rc = launch_linear(h, mlp_w1, mlp_b1, (int)T, C, 3 * C, 1, mp, dtype, st, kEpiGelu);
+    if (rc == BRA_OK) rc = launch_linear(m, mlp_w2, mlp_b2, (int)T, 3 * C, C, 1, op, dtype, st, kEpiResidual, x2);
     if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     return rc;
 }
@@ -1241,6 +1455,7 @@ int bra_backward(const void *q, const void *k, const void *v, const void *lce_w,
     const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
     int rc = check_shape(s);
     if (rc) return rc;
+    if (s.padded()) return BRA_ERR_SHAPE;  // the backward runs on multiples of S only
     if (!lce_w || !dlce_w || !dlce_b) return BRA_ERR_NULL;
     if (!aligned(dlce_w, 4) || !aligned(dlce_b, 4)) return BRA_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1308,7 +1523,25 @@ int bra_attend(const void *q, const void *k, const void *v, const void *lce_w, c
     if (cudaMallocAsync(reinterpret_cast<void **>(&flag), sizeof(int), st) != cudaSuccess) return BRA_ERR_CUDA;
     int host_flag = 0;
     rc = cudaMemsetAsync(flag, 0, sizeof(int), st) == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
-    if (rc == BRA_OK) rc = launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, flag, st);
+    if (rc == BRA_OK && s.padded()) {
+        // the padded grid: zero-padded copies of q, k, v, the attention on them, the crop
+        const size_t map = padded_map_bytes(s);
+        unsigned char *buf = nullptr;
+        if (cudaMallocAsync(reinterpret_cast<void **>(&buf), 4 * map, st) != cudaSuccess) {
+            rc = BRA_ERR_CUDA;
+        } else {
+            const void *src[3] = {q, k, v};
+            void *dst[3] = {buf, buf + map, buf + 2 * map};
+            rc = launch_pad(s, 3, src, dst, st);
+            if (rc == BRA_OK)
+                rc = launch_attend(padded_shape(s), dst[0], dst[1], dst[2], lce_w, lce_b, buf + 3 * map, r_idx, flag,
+                                   st);
+            if (rc == BRA_OK) rc = launch_crop(s, buf + 3 * map, out, st);
+            if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+        }
+    } else if (rc == BRA_OK) {
+        rc = launch_attend(s, q, k, v, lce_w, lce_b, out, r_idx, flag, st);
+    }
     if (rc == BRA_OK &&
         cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
         rc = BRA_ERR_CUDA;
@@ -1430,6 +1663,7 @@ int bra_forward_noalloc(const void *q, const void *k, const void *v, const void 
     const size_t es = dtype == BRA_BF16 ? 2 : 4;
     if (!aligned(lce_w, es) || !aligned(lce_b, es)) return BRA_ERR_ALIGN;
     if (2 * (size_t)N * s.P * C > (size_t)BRA_STATIC_SCRATCH_FLOATS) return BRA_ERR_SCRATCH;
+    if (s.padded()) return BRA_ERR_SCRATCH;  // the padded copies would need more scratch
     float *ws = nullptr;
     rc = static_scratch(&ws);
     if (rc) return rc;

@@ -35,12 +35,21 @@ struct LinearParams {
     CUtensorMap tmW;     // W (Nout, K): box (KC, BN), KC-matched swizzle
     CUtensorMap tmY[3];  // Y_i (M, Ny): box (32, 32), 64-byte swizzle
     const __nv_bfloat16 *bias;
+    const __nv_bfloat16 *res;  // epilogue kEpiResidual: (M, Nout) row-major, added after the bias
+    int epi;                   // kEpiBias, kEpiGelu or kEpiResidual
     int M, K, Nout, Ny, BN, tiles_n, tiles_m, stages;
     int kc_elems;    // K-elements per chunk: 64 (128-byte rows) or 32 (64-byte rows)
     int w_resident;  // 1: all of W stays in shared memory, the stages carry X chunks only
     uint32_t tmem_cols;
     unsigned wait_limit;
 };
+
+// Epilogues: y = round(acc + b); y = round(GELU(acc + b)) (the BiFormer MLP's first layer,
+// GELU in its exact erf form); y = round(res + round(acc + b)) (the MLP's second layer
+// with the block's residual: the projection is stored in the dtype, then added).
+enum { kEpiBias = 0, kEpiGelu = 1, kEpiResidual = 2 };
+
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
 constexpr int kLinEpiWarps = 8;                     // two per tensor-memory lane quarter
 constexpr int kLinThreads = 64 + 32 * kLinEpiWarps;  // warp 0 copies, warp 1 MMA, then the epilogue
@@ -275,16 +284,32 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_umma_kernel(const __gri
                     if (lane == 0) lin_bulk_wait_read<kLinOutSlots - 1>();
                     __syncwarp();
                 }
+                // the residual's row `lane`, columns c .. c + 31 of the unit (64 bytes)
+                uint4 rv[4] = {};
+                if (prm.epi == kEpiResidual && m0 + 32 * q + lane < prm.M) {
+                    const uint4 *rp = reinterpret_cast<const uint4 *>(prm.res + (size_t)(m0 + 32 * q + lane) * prm.Nout +
+                                                                      n0 + c);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) rv[j] = __ldg(rp + j);
+                }
                 // row `lane` of the block: four 16-byte chunks, 64-byte swizzle
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     uint32_t pk[4];
+                    const uint32_t *rw = reinterpret_cast<const uint32_t *>(&rv[j]);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int col = 8 * j + 2 * e;
                         const float2 bb = *reinterpret_cast<const float2 *>(sBias + n0 + c + col);
-                        const __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(r[col]) + bb.x,
-                                                                        __uint_as_float(r[col + 1]) + bb.y);
+                        float v0 = __uint_as_float(r[col]) + bb.x, v1 = __uint_as_float(r[col + 1]) + bb.y;
+                        if (prm.epi == kEpiGelu) {
+                            v0 = gelu_erf(v0);
+                            v1 = gelu_erf(v1);
+                        } else if (prm.epi == kEpiResidual) {
+                            v0 = __bfloat162float(__float2bfloat16_rn(v0)) + __uint_as_float(rw[e] << 16);
+                            v1 = __bfloat162float(__float2bfloat16_rn(v1)) + __uint_as_float(rw[e] & 0xFFFF0000u);
+                        }
+                        const __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
                         pk[e] = *reinterpret_cast<const uint32_t *>(&hv);
                     }
                     const uint32_t dst = sb + lane * 64 + (((j ^ (lane >> 1)) & 3) << 4);
@@ -336,8 +361,9 @@ __global__ void __launch_bounds__(kLinThreads, 1) linear_umma_kernel(const __gri
 
 struct LinearF32Params {
     const float *x, *w, *b;
+    const float *res;  // kEpiResidual: (M, Nout) row-major
     float *y[3];
-    int M, K, Nout, Ny;
+    int M, K, Nout, Ny, epi;
 };
 
 // 64 x 64 output tiles, one column block per blockIdx.x, row blocks blockIdx.y,
@@ -382,7 +408,10 @@ __global__ void __launch_bounds__(256) linear_f32_kernel(const LinearF32Params p
             const int n = n0 + tx + 16 * j;
             if (n >= prm.Nout) continue;
             const int which = n / prm.Ny;
-            prm.y[which][(size_t)m * prm.Ny + (n - which * prm.Ny)] = acc[i][j] + prm.b[n];
+            float v = acc[i][j] + prm.b[n];
+            if (prm.epi == kEpiGelu) v = gelu_erf(v);
+            else if (prm.epi == kEpiResidual) v += prm.res[(size_t)m * prm.Nout + n];
+            prm.y[which][(size_t)m * prm.Ny + (n - which * prm.Ny)] = v;
         }
     }
     }

@@ -10,7 +10,9 @@ Workload shapes follow the BiFormer stage shapes of the pages:
     section "BRA模块": x (1,56,56,64), 49 regions of 8x8 tokens, 2 heads of 32,
     topk 1);
   * per-stage top-k 1, 4, 16, S^2 and S = 7 / 16 / 8 for classification /
-    detection / segmentation (bernice.tw, "Biformer" and "消融實驗" sections).
+    detection / segmentation (bernice.tw, "Biformer" and "消融實驗" sections);
+  * one detection map whose size is not a multiple of S (a 1000x1000 input: 250x250
+    at stage 1, S = 16), for the padded grid.
 
 Value recipe (stated once, used everywhere):
   * q, k, v ~ N(0, 1) i.i.d.;
@@ -71,8 +73,17 @@ class Workload:
         return self.S * self.S
 
     @property
+    def hr(self) -> int:
+        """Region height: ceil(H / S) (the padded grid when S does not divide H)."""
+        return -(-self.H // self.S)
+
+    @property
+    def wr(self) -> int:
+        return -(-self.W // self.S)
+
+    @property
     def w2(self) -> int:
-        return (self.H // self.S) * (self.W // self.S)
+        return self.hr * self.wr
 
     @property
     def tokens(self) -> int:
@@ -92,6 +103,9 @@ WORKLOADS: Dict[str, Workload] = {
         Workload("cls_stage3_224_dense", 6, 128, 14, 14, 256, 8, 7, 49, "bf16", lce_b_std=0.01),
         Workload("det_stage1_1024", 4, 2, 256, 256, 64, 2, 16, 1, "bf16", region_bias=0.5),
         Workload("seg_stage2_512", 5, 8, 64, 64, 128, 4, 8, 4, "bf16", region_bias=0.5),
+        # a detection input whose stage-1 map (1000 / 4 = 250) is not a multiple of S = 16:
+        # the padded grid (250 -> 256)
+        Workload("det_stage1_1000", 7, 2, 250, 250, 64, 2, 16, 1, "bf16", region_bias=0.5),
     ]
 }
 
@@ -118,6 +132,14 @@ def _store(x: np.ndarray, dtype: str) -> np.ndarray:
     return round_bf16(x32) if dtype == "bf16" else x32
 
 
+def _region_field(off: np.ndarray, w: Workload) -> np.ndarray:
+    """Spread per-region offsets (N,S,1,S,1,C) over the pixels of their regions, on the
+    (padded) grid of ceil(H/S) x ceil(W/S) regions, cropped to H x W."""
+    N, C = off.shape[0], off.shape[-1]
+    full = np.broadcast_to(off, (N, w.S, w.hr, w.S, w.wr, C)).reshape(N, w.S * w.hr, w.S * w.wr, C)
+    return full[:, :w.H, :w.W]
+
+
 def make_inputs(w: Workload, seed_base: Optional[int] = None, batch: Optional[int] = None) -> Dict[str, np.ndarray]:
     """Return q, k, v (N,H,W,C), lce_w (C,5,5), lce_b (C) as float32 arrays.
 
@@ -128,12 +150,11 @@ def make_inputs(w: Workload, seed_base: Optional[int] = None, batch: Optional[in
     N = w.N if batch is None else batch
     shape = (N, w.H, w.W, w.C)
     out = {}
-    hr, wr = w.H // w.S, w.W // w.S
     for name in ("q", "k", "v"):
         x = _rng(w, name, seed_base).standard_normal(shape)
         if w.region_bias > 0:
             off = _rng(w, name + "_off", seed_base).standard_normal((N, w.S, 1, w.S, 1, w.C)) * w.region_bias
-            x = (x.reshape(N, w.S, hr, w.S, wr, w.C) + off).reshape(shape)
+            x = x + _region_field(off, w)
         out[name] = _store(x, w.dtype)
     out["lce_w"] = _store(_rng(w, "lce_w", seed_base).standard_normal((w.C, 5, 5)) * w.lce_w_std, w.dtype)
     if w.lce_b_std > 0:
@@ -152,11 +173,10 @@ def make_layer_inputs(w: Workload, seed_base: Optional[int] = None, batch: Optio
     """
     N = w.N if batch is None else batch
     shape = (N, w.H, w.W, w.C)
-    hr, wr = w.H // w.S, w.W // w.S
     x = _rng(w, "x", seed_base).standard_normal(shape)
     if w.region_bias > 0:
         off = _rng(w, "x_off", seed_base).standard_normal((N, w.S, 1, w.S, 1, w.C)) * w.region_bias
-        x = (x.reshape(N, w.S, hr, w.S, wr, w.C) + off).reshape(shape)
+        x = x + _region_field(off, w)
     g = 1.0 / np.sqrt(w.C)
     out = {
         "x": _store(x, w.dtype),
