@@ -441,14 +441,19 @@ def main():
         if not backward:  # the backward reads the forward's routing (copied with the set)
             s["r_idx"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.int32, device=dev)
         s["r_w"] = torch.empty((w.N, w.regions, w.topk), dtype=torch.float32, device=dev)
+        if backward:  # the gradients of each set, written in place by every step
+            f32 = dict(dtype=torch.float32, device=dev)
+            s["grads"] = {"dq": torch.empty((w.N, w.H, w.W, w.C), **f32), "dk": torch.empty((w.N, w.H, w.W, w.C), **f32),
+                          "dv": torch.empty((w.N, w.H, w.W, w.C), **f32), "dlce_w": torch.empty((w.C, 5, 5), **f32),
+                          "dlce_b": torch.empty((w.C,), **f32)}
         sets.append(s)
 
     stream = torch.cuda.Stream(device=dev)
 
-    def fwd(s):
-        if backward:
-            s["grads"] = bra.backward(s["q"], s["k"], s["v"], s["lce_w"], s["r_idx"], s["dout"], w.heads, w.S,
-                                      stream=stream)
+    def fwd(s, sync=False):
+        if backward:  # timed and traced: the asynchronous entry point (graph-capturable)
+            bra.backward(s["q"], s["k"], s["v"], s["lce_w"], s["r_idx"], s["dout"], w.heads, w.S, stream=stream,
+                         grads=s["grads"], sync=sync)
         elif layer:
             bra.attention_layer(s["x"], s["w_qkv"], s["b_qkv"], s["w_o"], s["b_o"], s["lce_w"], s["lce_b"],
                                 w.heads, w.S, w.topk, out=s["out"], r_idx=s["r_idx"], r_weight=s["r_w"],
@@ -463,7 +468,7 @@ def main():
     with torch.cuda.stream(stream):
         fwd(sets[0])  # first call outside capture: lazy module load, pool init
     stream.synchronize()
-    if not args.no_graph and not backward:  # bra_backward synchronises: direct launches
+    if not args.no_graph:
         for s in sets:
             g = torch.cuda.CUDAGraph()
             c0 = bra.launch_count()
@@ -519,33 +524,25 @@ def main():
     torch.cuda.synchronize(dev)
     bra.trace_begin()
     trace = {}
-    if backward:
+    traced = []
+    with torch.cuda.stream(stream):
+        for s_ in sets:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fwd(s_)
+            traced.append(g)
+    rounds = max(1, math.ceil(args.steps / n_sets))
+    for _ in range(rounds):
         with torch.cuda.stream(stream):
-            for i in range(args.steps):
-                fwd(sets[i % n_sets])
+            for g in traced:
+                g.replay()
         torch.cuda.synchronize(dev)
-        trace = {k_: [t_ms, t_n] for k_, (t_ms, t_n) in bra.trace_read().items()}
-        traced_steps = args.steps
-    else:
-        traced = []
-        with torch.cuda.stream(stream):
-            for s_ in sets:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    fwd(s_)
-                traced.append(g)
-        rounds = max(1, math.ceil(args.steps / n_sets))
-        for _ in range(rounds):
-            with torch.cuda.stream(stream):
-                for g in traced:
-                    g.replay()
-            torch.cuda.synchronize(dev)
-            for k_, (t_ms, t_n) in bra.trace_read().items():
-                a_ = trace.setdefault(k_, [0.0, 0])
-                a_[0] += t_ms
-                a_[1] += t_n
-        del traced
-        traced_steps = rounds * n_sets
+        for k_, (t_ms, t_n) in bra.trace_read().items():
+            a_ = trace.setdefault(k_, [0.0, 0])
+            a_[0] += t_ms
+            a_[1] += t_n
+    del traced
+    traced_steps = rounds * n_sets
     bra.trace_end()
     clocks.stop()
 
@@ -566,7 +563,7 @@ def main():
             with torch.cuda.stream(stream):
                 for k_, v_ in host.items():
                     d_in[k_].copy_(v_, non_blocking=True)
-                fwd(d_in)
+                fwd(d_in, sync=True)  # the synchronising public entry point
                 for k_, t_ in d_in["grads"].items():
                     h_grads[k_].copy_(t_, non_blocking=True)
             stream.synchronize()
@@ -626,8 +623,9 @@ def main():
     alg_bytes = {"bra_image_kernel": acc["fused_bytes"], "region_mean_kernel": acc["pool_bytes"],
                  "route_kernel": acc["route_bytes"], "linear_umma_kernel": acc["linear_bytes"],
                  "linear_f32_kernel": acc["linear_bytes"]}.get(attn_name, acc["attn_bytes"])
-    if backward:  # the backward's three kernels form one traced class: time per call
-        traced_s = attn_s = t_ms / max(traced_steps, 1) / 1e3
+    if backward:  # the backward's kernels form one traced class: time per call
+        traced_s = t_ms / max(traced_steps, 1) / 1e3
+        attn_s = min(traced_s, ms_step / 1e3)
         alg_bytes = acc["bwd_bytes"]
     step_traced_ms = sum(v[0] for v in trace.values()) / traced_steps
     share = {k: round(v[0] / max(1e-12, sum(x[0] for x in trace.values())), 4) for k, v in trace.items() if v[1]}
@@ -658,7 +656,7 @@ def main():
                          % (n_sets, set_bytes / 1e6, n_sets * set_bytes / 1e6, l2 / 1e6),
                    "launch": "CUDA graph per step" if graphs else "direct launches",
                    "attention_kernel": args.variant,
-                   "step": "bra_backward (routing detached, the forward's r_idx)" if backward else
+                   "step": "bra_backward_async (routing detached, the forward's r_idx)" if backward else
                            ("bra_attention_layer (qkv projection, BRA, output projection)" if layer
                             else "bra_forward"),
                    "parallelism": "dp%d (independent images, no collective)" % world},
@@ -672,7 +670,7 @@ def main():
         "clocks": clocks.summary(),
         "e2e": {"value": tokens_all * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-                "entry": "bra_backward with stream copies (pinned host buffers)" if backward else
+                "entry": "bra_backward (synchronising) with stream copies (pinned host buffers)" if backward else
                          ("bra_attention_layer with stream copies (pinned host buffers)" if layer
                           else "bra_forward_host (pinned host buffers)")},
     }

@@ -244,17 +244,32 @@ int bra_block(const void *x, const void *pos_w, const void *pos_b, const void *l
  * r_weight does not scale K or V, so gradients flow through the token attention and the
  * LCE only. Given dout = dL/dout (N,H,W,C) in `dtype` and the forward's r_idx, writes
  *   dq, dk, dv: (N,H,W,C) float32;  dlce_w: (C,5,5) float32;  dlce_b: (C) float32.
- * Arithmetic in float32; dk and dv are accumulated with atomics (the summation order,
- * and so the last bits, can differ between calls). The attention softmax is recomputed
- * from q and k. Every r_idx entry must lie in [0, S*S): an entry outside is skipped and
- * the call returns BRA_ERR_INDEX; like bra_attend, this call synchronises `stream` to
- * read that flag. Shapes as bra_forward, with H and W multiples of S (no padded grid:
+ * The attention softmax is recomputed from q and k.
+ *   - BRA_BF16 with 32 channels per head: tensor-core kernels (bf16 products, float32
+ *     accumulation; the probabilities and dS enter their products as bf16 high + low
+ *     parts). Deterministic: every output element has one writer and every sum a fixed
+ *     order, so repeated calls give identical bits. Scratch (the transposed routing,
+ *     per-query statistics, LCE partial sums) is taken like bra_attention_layer's.
+ *   - otherwise (float32, or 64 channels per head): float32 SIMT kernels; dk and dv are
+ *     accumulated with atomics (the summation order, and so the last bits, can differ
+ *     between calls).
+ * Every r_idx entry must lie in [0, S*S): an entry outside is skipped and the call
+ * returns BRA_ERR_INDEX; like bra_attend, this call synchronises `stream` to read that
+ * flag. Shapes as bra_forward, with H and W multiples of S (no padded grid:
  * BRA_ERR_SHAPE otherwise); q, k, v, dout, lce_w aligned to their element,
- * the float32 outputs and r_idx to 4 bytes. N = 0 zeroes dlce_w and dlce_b only.
- * Plain SIMT kernels: a first, correct form of this step, not yet tuned. */
+ * the float32 outputs and r_idx to 4 bytes. N = 0 zeroes dlce_w and dlce_b only. */
 int bra_backward(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
                  const void *dout, int N, int H, int W, int C, int heads, int S, int topk, int dtype, float *dq,
                  float *dk, float *dv, float *dlce_w, float *dlce_b, bra_stream_t stream);
+
+/* bra_backward without the host synchronisation, so that it can be enqueued back to back
+ * or captured in a CUDA graph: same arguments, kernels and results. An r_idx entry outside
+ * [0, S*S) is skipped as in bra_backward and raises the library's device flag, which the
+ * next bra_device_status call reports as BRA_ERR_INDEX (and clears); the return value
+ * covers argument checks and launches only. */
+int bra_backward_async(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
+                       const void *dout, int N, int H, int W, int C, int heads, int S, int topk, int dtype,
+                       float *dq, float *dk, float *dv, float *dlce_w, float *dlce_b, bra_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Tracing (measurement support; no part of the computation).
@@ -338,8 +353,9 @@ enum {
 int bra_set_kernel_variant(int variant);
 
 /* Synchronise `stream`, then report whether any kernel of this library gave up a
- * bounded wait since the last call (BRA_ERR_TIMEOUT; the flag is cleared) or not
- * (BRA_OK). BRA_ERR_CUDA if the synchronisation or the read fails. Kernels never
+ * bounded wait since the last call (BRA_ERR_TIMEOUT), else whether a bra_backward_async
+ * call met an r_idx entry outside [0, S*S) (BRA_ERR_INDEX), else BRA_OK; the flags are
+ * cleared. BRA_ERR_CUDA if the synchronisation or the read fails. Kernels never
  * spin without a limit: a wait that runs out raises this flag and the kernel
  * returns. */
 int bra_device_status(bra_stream_t stream);

@@ -189,18 +189,23 @@ def linear(x, w, b) -> np.ndarray:
 
 
 def layer_forward(x, w_qkv, b_qkv, w_o, b_o, lce_w, lce_b, heads: int, S: int, topk: int, dtype: str,
-                  intermediates: bool = False):
+                  intermediates: bool = False, r_idx_given=None):
     """The attention layer around the path: out = wo(BRA(qkv(x))).
 
     x (N,H,W,C); w_qkv (3C, C), b_qkv (3C); w_o (C, C), b_o (C); lce_w (C,5,5), lce_b (C).
     Returns (out, r_idx, r_weight), plus {"q","k","v","o"} (the stored intermediates)
     when `intermediates` is set. `out` is the float64 value before the final rounding.
+    With `r_idx_given`, the attention runs over that routing instead of its own (r_idx and
+    r_weight are still the layer's own routing), so that a result routed differently on a
+    near tie can be checked element by element.
     """
     x = _d(x)
     N, H, W, C = x.shape
     qkv = linear(x.reshape(-1, C), w_qkv, b_qkv)
     q, k, v = (round_to(qkv[:, i * C:(i + 1) * C], dtype).reshape(N, H, W, C) for i in range(3))
     o, r_idx, r_w = forward(q, k, v, lce_w, lce_b, heads, S, topk)
+    if r_idx_given is not None:
+        o = attend(q, k, v, lce_w, lce_b, heads, S, r_idx_given)
     o = round_to(o, dtype)
     out = linear(o.reshape(-1, C), w_o, b_o).reshape(N, H, W, C)
     if intermediates:

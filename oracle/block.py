@@ -57,20 +57,27 @@ def gelu(x) -> np.ndarray:
     return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
 
 
-def block_forward(x, p: Dict[str, np.ndarray], heads: int, S: int, topk: int, dtype: str):
+def block_forward(x, p: Dict[str, np.ndarray], heads: int, S: int, topk: int, dtype: str, r_idx_given=None,
+                  intermediates: bool = False):
     """One BiFormer block. p holds pos_w (C,3,3), pos_b (C), ln1_g, ln1_b, ln2_g, ln2_b (C),
     w_qkv (3C,C), b_qkv (3C), w_o (C,C), b_o (C), lce_w (C,5,5), lce_b (C),
     mlp_w1 (3C,C), mlp_b1 (3C), mlp_w2 (C,3C), mlp_b2 (C).
-    Returns (out, r_idx, r_weight); out is the float64 value before its final rounding."""
+    Returns (out, r_idx, r_weight); out is the float64 value before its final rounding.
+    `r_idx_given`: the attention runs over that routing (see oracle.layer_forward).
+    `intermediates`: also return {"h": norm1's stored output (the attention layer's input),
+    "x2": the stored residual x1 + attn, "m": the stored MLP output} (the output is x2 + m)."""
     r = lambda a: oracle.round_to(a, dtype)
     x = np.asarray(x, dtype=np.float64)
     N, H, W, C = x.shape
     x = r(x + dwconv3(x, p["pos_w"], p["pos_b"]))
     h = r(layer_norm(x, p["ln1_g"], p["ln1_b"]))
+    h1 = h
     a, r_idx, r_w = oracle.layer_forward(h, p["w_qkv"], p["b_qkv"], p["w_o"], p["b_o"], p["lce_w"], p["lce_b"],
-                                         heads, S, topk, dtype)
+                                         heads, S, topk, dtype, r_idx_given=r_idx_given)
     x = r(x + r(a))
     h = r(layer_norm(x, p["ln2_g"], p["ln2_b"]))
     m = r(gelu(oracle.linear(h.reshape(-1, C), p["mlp_w1"], p["mlp_b1"])))
     m = oracle.linear(m, p["mlp_w2"], p["mlp_b2"]).reshape(N, H, W, C)
+    if intermediates:
+        return x + r(m), r_idx, r_w, {"h": h1, "x2": x, "m": r(m)}
     return x + r(m), r_idx, r_w

@@ -90,14 +90,17 @@ def check_routing(logits: np.ndarray, ref_idx: np.ndarray, ref_w: np.ndarray, id
         rep.fail("r_weight err %.3g > %.1g" % (rep.weight_max_err, tol_weight))
 
 
-def check_output(out: np.ndarray, ref: np.ndarray, dtype: str, rep: Report) -> None:
+def check_output(out: np.ndarray, ref: np.ndarray, dtype: str, rep: Report, scale: Optional[np.ndarray] = None
+                 ) -> None:
+    """`scale`: the magnitude the relative bf16 term is taken of (default |ref|); a result
+    that is a sum of separately rounded terms passes the sum of the terms' magnitudes."""
     out = out.astype(np.float64)
     err = np.abs(out - ref)
     rep.out_max_abs_err = float(err.max()) if err.size else 0.0
     if dtype == "f32":
         allowed = np.full_like(ref, TOL_F32_ABS)
     else:
-        allowed = TOL_BF16_ABS + TOL_BF16_REL * np.abs(ref)
+        allowed = TOL_BF16_ABS + TOL_BF16_REL * (np.abs(ref) if scale is None else scale)
     ratio = err / allowed
     rep.out_worst_ratio = float(ratio.max()) if ratio.size else 0.0
     if not np.all(np.isfinite(out)):

@@ -1,10 +1,13 @@
 """Parity of bra_backward (routing detached) with the float64 backward oracle, on a B200.
 
-The cases of tests/test_backward_host.py, which runs the kernels' per-item code on the
+The cases of tests/test_backward_host.py, which runs the SIMT kernels' per-item code on the
 host with every access bounds-checked (the file name keeps these tests after the rest of
-the GPU suite). Tolerance:
-float32 arithmetic with atomically accumulated dk and dv against float64, normwise per
-tensor: max |gpu - ref| <= 1e-4 * max(1, max |ref|)."""
+the GPU suite), plus shapes for the tensor-core path that bf16 maps with 32 channels per
+head take (regions of 4, 25, 32, 64 and 256 tokens, the dense limit with a ragged last key
+chunk, repeated and out-of-range regions). Tolerance: float32 arithmetic against float64,
+normwise per tensor: max |gpu - ref| <= 1e-4 * max(1, max |ref|). The tensor-core path
+multiplies the probabilities and dS as bf16 high + low parts, so it meets the same bound,
+and it is deterministic: two calls give the same bits."""
 import numpy as np
 import pytest
 import torch
@@ -58,3 +61,76 @@ def test_backward_repeated_and_invalid_regions():
     with pytest.raises(bra.BraError) as e:
         run_gpu(q, k, v, dout, w, r_bad, heads, S, "f32")
     assert e.value.status == 6  # BRA_ERR_INDEX
+
+
+TC_CASES = [
+    # N, H, W, C, heads, S, topk  (bf16, d = 32: the tensor-core path)
+    (2, 14, 14, 256, 8, 7, 16),   # 2x2-token regions: one warp with 12 padded rows
+    (1, 14, 14, 64, 2, 7, 49),    # dense limit: 196 keys, a ragged last 32-key chunk
+    (1, 15, 15, 64, 2, 3, 3),     # 5x5-token regions: 25 queries, 75 keys
+    (1, 12, 24, 64, 2, 3, 2),     # non-square 4x8-token regions
+    (1, 32, 32, 128, 4, 4, 4),    # 64-token regions, 256 keys (the segmentation shape)
+    (1, 32, 32, 64, 2, 2, 1),     # 256-token regions, 16 warps (the detection shape)
+]
+
+
+@pytest.mark.parametrize("N,H,W,C,heads,S,topk", TC_CASES)
+def test_tensor_core_backward_matches_oracle(N, H, W, C, heads, S, topk):
+    q, k, v, dout, w = inputs(N, H, W, C, 120 + C + topk + H, "bf16")
+    r_idx, _ = oracle.route(q, k, heads, S, topk)
+    got = run_gpu(q, k, v, dout, w, r_idx, heads, S, "bf16")
+    check(got, ob.backward(q, k, v, w, np.zeros(C), heads, S, r_idx, dout))
+    assert bra.device_status() == 0
+
+
+def test_tensor_core_backward_repeated_and_invalid_regions():
+    N, H, W, C, heads, S = 1, 16, 16, 64, 2, 4
+    q, k, v, dout, w = inputs(N, H, W, C, 95, "bf16")
+    r_idx, _ = oracle.route(q, k, heads, S, 3)
+    r_idx = r_idx.copy()
+    r_idx[0, 1] = [5, 5, 2]   # a region routed twice: its keys count twice in the softmax
+    r_idx[0, 7] = [7, 0, 7]
+    check(run_gpu(q, k, v, dout, w, r_idx, heads, S, "bf16"), ob.backward(q, k, v, w, np.zeros(C), heads, S, r_idx, dout))
+    r_bad = r_idx.copy()
+    r_bad[0, 2, 1] = 16
+    with pytest.raises(bra.BraError) as e:
+        run_gpu(q, k, v, dout, w, r_bad, heads, S, "bf16")
+    assert e.value.status == 6  # BRA_ERR_INDEX
+
+
+def test_tensor_core_backward_is_deterministic():
+    """Two calls on the classification stage-2 batch give identical bits in every output
+    (no atomics: each element has one writer, and every sum runs in a fixed order)."""
+    w = synth.WORKLOADS["cls_stage2_224"].with_(N=8)
+    q, k, v, dout, lw = inputs(w.N, w.H, w.W, w.C, 130, "bf16")
+    r_idx, _ = oracle.route(q, k, w.heads, w.S, w.topk)
+    a = run_gpu(q, k, v, dout, lw, r_idx, w.heads, w.S, "bf16")
+    b = run_gpu(q, k, v, dout, lw, r_idx, w.heads, w.S, "bf16")
+    for name in a:
+        assert np.array_equal(a[name].view(np.uint32), b[name].view(np.uint32)), name
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_async_backward_equals_backward_and_reports_index_errors(dtype):
+    """bra_backward_async: the same kernels without the host synchronisation; identical
+    results (bits, on the deterministic bf16 path), and an out-of-range routing entry
+    surfaces through bra_device_status as BRA_ERR_INDEX."""
+    N, H, W, C, heads, S = 2, 16, 16, 64, 2, 4
+    q, k, v, dout, w = inputs(N, H, W, C, 140, dtype)
+    r_idx, _ = oracle.route(q, k, heads, S, 3)
+    d = [dev(x, dtype) for x in (q, k, v, w)]
+    ri = torch.from_numpy(np.ascontiguousarray(r_idx, np.int32)).cuda()
+    do = dev(dout, dtype)
+    a = bra.backward(d[0], d[1], d[2], d[3], ri, do, heads, S)
+    b = bra.backward(d[0], d[1], d[2], d[3], ri, do, heads, S, sync=False)
+    assert bra.device_status() == 0
+    ref = ob.backward(q, k, v, w, np.zeros(C), heads, S, r_idx, dout)
+    check({n_: t.cpu().numpy() for n_, t in b.items()}, ref)
+    if dtype == "bf16":
+        for n_ in a:
+            assert torch.equal(a[n_].view(torch.int32), b[n_].view(torch.int32)), n_
+    bad = r_idx.copy()
+    bad[1, 3, 2] = -1
+    bra.backward(d[0], d[1], d[2], d[3], torch.from_numpy(bad).cuda(), do, heads, S, sync=False)
+    assert bra.device_status() == 6  # BRA_ERR_INDEX, then cleared
+    assert bra.device_status() == 0

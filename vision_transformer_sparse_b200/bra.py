@@ -27,7 +27,7 @@ SYMBOLS = ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_fo
            "bra_status_string",
            "bra_version", "bra_launch_count", "bra_trace_begin", "bra_trace_end", "bra_kernel_name",
            "bra_set_kernel_variant", "bra_device_status", "bra_selftest_wait_timeout", "bra_trace_read",
-           "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward", "bra_linear_act", "bra_block")
+           "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward", "bra_linear_act", "bra_block", "bra_backward_async")
 ACT_NONE, ACT_GELU, ACT_RESIDUAL = 0, 1, 2
 KERNEL_CLASSES = 11
 
@@ -56,11 +56,12 @@ def lib() -> ctypes.CDLL:
         L.bra_qkv.argtypes = [vp] * 3 + [i] * 3 + [vp] * 4
         L.bra_attention_layer.argtypes = [vp] * 7 + shape + [vp, vp, vp, vp]
         L.bra_backward.argtypes = [vp] * 6 + shape + [vp] * 6
+        L.bra_backward_async.argtypes = [vp] * 6 + shape + [vp] * 6
         L.bra_linear_act.argtypes = [vp] * 4 + [i] * 5 + [vp, vp]
         L.bra_block.argtypes = [vp] * 17 + shape + [vp, vp, vp, vp]
         for f in ("bra_forward", "bra_route", "bra_attend", "bra_forward_host", "bra_forward_noalloc",
                   "bra_version", "bra_linear", "bra_qkv", "bra_attention_layer", "bra_backward",
-                  "bra_linear_act", "bra_block"):
+                  "bra_linear_act", "bra_block", "bra_backward_async"):
             getattr(L, f).restype = i
         L.bra_status_string.argtypes = [i]
         L.bra_status_string.restype = ctypes.c_char_p
@@ -202,20 +203,23 @@ def attention_layer(x, w_qkv, b_qkv, w_o, b_o, lce_w, lce_b, heads: int, S: int,
     return out, r_idx, r_weight
 
 
-def backward(q, k, v, lce_w, r_idx, dout, heads: int, S: int, stream=None) -> dict:
-    """bra_backward: gradients (float32) of sum(dout * forward output) for the routing
-    r_idx (N, S*S, topk), routing detached -> {dq, dk, dv, dlce_w, dlce_b}."""
+def backward(q, k, v, lce_w, r_idx, dout, heads: int, S: int, stream=None, grads=None, sync: bool = True) -> dict:
+    """bra_backward (sync=True) or bra_backward_async: gradients (float32) of
+    sum(dout * forward output) for the routing r_idx (N, S*S, topk), routing detached ->
+    {dq, dk, dv, dlce_w, dlce_b} (allocated here unless `grads` holds them)."""
     N, H, W, C = q.shape
     topk = r_idx.shape[-1]
     f32 = dict(dtype=torch.float32, device=q.device)
-    g = {"dq": torch.empty((N, H, W, C), **f32), "dk": torch.empty((N, H, W, C), **f32),
-         "dv": torch.empty((N, H, W, C), **f32), "dlce_w": torch.empty((C, 5, 5), **f32),
-         "dlce_b": torch.empty((C,), **f32)}
+    g = grads if grads is not None else {
+        "dq": torch.empty((N, H, W, C), **f32), "dk": torch.empty((N, H, W, C), **f32),
+        "dv": torch.empty((N, H, W, C), **f32), "dlce_w": torch.empty((C, 5, 5), **f32),
+        "dlce_b": torch.empty((C,), **f32)}
     _check_dev(q, k, v, lce_w, r_idx, dout, *g.values())
-    rc = lib().bra_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(r_idx), _ptr(dout), N, H, W, C, heads, S,
-                            topk, _dtype_code(q), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlce_w"]),
-                            _ptr(g["dlce_b"]), _stream(stream))
-    _raise(rc, "bra_backward")
+    fn = lib().bra_backward if sync else lib().bra_backward_async
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(lce_w), _ptr(r_idx), _ptr(dout), N, H, W, C, heads, S,
+            topk, _dtype_code(q), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlce_w"]),
+            _ptr(g["dlce_b"]), _stream(stream))
+    _raise(rc, "bra_backward" if sync else "bra_backward_async")
     return g
 
 
@@ -313,7 +317,8 @@ def set_kernel_variant(variant: int) -> int:
 
 
 def device_status(stream=None) -> int:
-    """bra_device_status: 0, or 8 (BRA_ERR_TIMEOUT) if a kernel's bounded wait ran out."""
+    """bra_device_status: 0; 8 (BRA_ERR_TIMEOUT) if a kernel's bounded wait ran out; 6 (BRA_ERR_INDEX) if
+    a bra_backward_async call met an out-of-range routing entry. Clears the flags."""
     return int(lib().bra_device_status(_stream(stream)))
 
 

@@ -29,9 +29,6 @@
 
 namespace bra {
 
-// Set by any kernel whose bounded wait ran out; read and cleared by bra_device_status.
-__device__ int g_bra_timeout_flag = 0;
-
 struct TmaAttnParams {
     CUtensorMap tmQ;  // q, box (64, wr, RB, 1)
     CUtensorMap tmK;  // k, box (64, wr, hr, 1)

@@ -422,58 +422,50 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
                 // reference: the exact max of the first valid 32-key chunk. Every p is
                 // taken relative to it; a row whose later keys exceed it by so much that p,
                 // the row sum or O overflows is recomputed exactly in the epilogue.
+                // Chunk c (32 keys) sits at F + 32 c for c < 4, at G + 32 (c - 4) after; even
+                // chunks go through buffer ra, odd ones through rb, so that the next chunk's
+                // scores load while the current chunk's exponentials are computed.
+                const int nch = 2 * np;
+                auto chunk_col = [&](int c) { return c < 4 ? F + 32 * c : G + 32 * (c - 4); };
+                auto chunk_valid = [&](int c) { return (c << 5) < prm.w2 ? v0 : v1; };
                 uint32_t ra[32], rb[32];
                 float m = -INFINITY;
-                bool have = false;  // ra, rb hold the scores of the next pair
                 if (v0) {
-                    tmem_ld32_nowait(F, ra);
-                    tmem_ld32_nowait(F + 32, rb);
-                    tmem_wait_ld(ra);
-                    tmem_regs_after_wait(rb);
+                    tmem_ld32(F, ra);  // chunk 0, kept for its exponentials
                     m = max32(ra, -INFINITY);
-                    have = true;
                 } else if (np == 4 && prm.topk > 1 && v1) {  // keys 128..255: the second region
                     if (!wait_g()) break;
-                    tmem_ld32(G, ra);
-                    m = max32(ra, -INFINITY);
+                    tmem_ld32(G, rb);
+                    m = max32(rb, -INFINITY);
                 }
-                // single pass over chunk pairs (64 independent exponentials in flight per
-                // thread): probabilities, row sum, P (bf16) over scores already read. Each
-                // pair's P is handed to the MMA issuer as soon as it is stored, the next
-                // pair's scores being loaded meanwhile.
                 const float mneg = m == -INFINITY ? 0.f : -m * sl2;
                 const float2 sl2v = make_float2(sl2, sl2), mnv = make_float2(mneg, mneg);
                 float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
                 float2 lc = make_float2(0.f, 0.f), ld = make_float2(0.f, 0.f);
-                for (int j = 0; j < np; ++j) {
-                    const bool valid = (j << 6) < prm.w2 ? v0 : v1;  // both chunks of a pair lie in one region
-                    if (valid && !have) {
-                        if (j >= 2 && !wait_g()) {
+                uint32_t pk[16];  // P of one chunk (bf16 pairs)
+                for (int c = 0; c < nch && !fail; c += 2) {
+                    const int j = c >> 1;  // the pair
+                    // ---- even chunk c (in ra); the odd chunk c + 1 loads into rb meanwhile
+                    const bool ve = chunk_valid(c), vo = chunk_valid(c + 1);
+                    if (vo) {
+                        if (c + 1 >= 4 && !wait_g()) {
                             fail = true;
                             break;
                         }
-                        const uint32_t c = j < 2 ? F + 64 * j : G + 64 * (j - 2);
-                        tmem_ld32_nowait(c, ra);
-                        tmem_ld32_nowait(c + 32, rb);
-                        tmem_wait_ld(ra);
-                        tmem_regs_after_wait(rb);
+                        tmem_ld32_nowait(chunk_col(c + 1), rb);
                     }
-                    if (j == 3) {  // every score of G has been read: the next unit may take G
-                        if (!wait_g()) {
-                            fail = true;
-                            break;
-                        }
-                        tc_fence_before();
-                        umma_arrive(bars + 8 * (kUbGRead + t));
-                    }
-                    uint32_t pa[16], pb[16];
-                    if (valid) {
-                        exp32(ra, sl2v, mnv, la, lb, pa);
-                        exp32(rb, sl2v, mnv, lc, ld, pb);
-                    } else {
+                    if (ve)
+                        exp32(ra, sl2v, mnv, la, lb, pk);
+                    else {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) pa[e] = pb[e] = 0u;
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
                     }
+                    if (j > 0) {  // pair j - 1's P was stored a chunk ago: hand it to the MMA
+                        tmem_wait_st();
+                        tc_fence_before();
+                        umma_arrive(bars + 8 * (kUbP + 4 * t + j - 1));
+                    }
+                    if (vo) tmem_wait_ld(rb);
                     if (j == 3) {  // P_3 goes over P_0: wait for pair 0's MMAs
                         if (!umma_wait_warp(bars + 8 * (kUbPFree + t), k & 1, lim)) {
                             fail = true;
@@ -481,33 +473,43 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
                         }
                         tc_fence_after();
                     }
+                    // P of pair j over scores already read (both chunks of the pair are in
+                    // registers now): F + 32 (j + 1) for j < 3, over P_0 for j = 3
                     const uint32_t pcol = F + 32 * (j < 3 ? j + 1 : 1);
-                    tmem_st16_nowait(pcol, pa);
-                    tmem_st16_nowait(pcol + 16, pb);
-                    // the next pair's scores are loaded while the stores drain (the load and
-                    // its wait stay in one branch, so no copy of a pending register is made)
-                    const int jn = j + 1;
-                    have = jn < np && ((jn << 6) < prm.w2 ? v0 : v1);
-                    if (have && jn >= 2 && !wait_g()) {
-                        fail = true;
-                        have = false;
+                    tmem_st16_nowait(pcol, pk);
+                    // every score of G is in registers once the last chunk is: the next unit
+                    // may take G
+                    if (np == 4 && c + 1 == nch - 1) {
+                        if (!wait_g()) {
+                            fail = true;
+                            break;
+                        }
+                        tc_fence_before();
+                        umma_arrive(bars + 8 * (kUbGRead + t));
                     }
-                    if (have) {
-                        const uint32_t c = jn < 2 ? F + 64 * jn : G + 64 * (jn - 2);
-                        tmem_ld32_nowait(c, ra);
-                        tmem_ld32_nowait(c + 32, rb);
+                    // ---- odd chunk c + 1 (in rb); the next pair's first chunk loads into ra
+                    const bool vn = c + 2 < nch && chunk_valid(c + 2);
+                    if (vn) {
+                        if (c + 2 >= 4 && !wait_g()) {
+                            fail = true;
+                            break;
+                        }
+                        tmem_ld32_nowait(chunk_col(c + 2), ra);
+                    }
+                    if (vo)
+                        exp32(rb, sl2v, mnv, lc, ld, pk);
+                    else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    }
+                    tmem_st16_nowait(pcol + 16, pk);
+                    if (j == np - 1) {  // the last pair: no later chunk to wait behind
                         tmem_wait_st();
+                        *rsum = ((la.x + la.y) + (lb.x + lb.y)) + ((lc.x + lc.y) + (ld.x + ld.y));
                         tc_fence_before();
                         umma_arrive(bars + 8 * (kUbP + 4 * t + j));
-                        tmem_wait_ld(ra);
-                        tmem_regs_after_wait(rb);
-                    } else {
-                        tmem_wait_st();
-                        if (j == np - 1) *rsum = ((la.x + la.y) + (lb.x + lb.y)) + ((lc.x + lc.y) + (ld.x + ld.y));
-                        tc_fence_before();
-                        umma_arrive(bars + 8 * (kUbP + 4 * t + j));
                     }
-                    if (fail) break;
+                    if (vn) tmem_wait_ld(ra);
                 }
                 if (fail) break;
             }

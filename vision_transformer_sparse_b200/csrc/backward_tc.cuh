@@ -1,0 +1,502 @@
+// backward_tc.cuh — the BRA backward with the routing detached, on the tensor cores
+// (warp-level mma.sync, bf16 operands, float32 accumulation) and deterministic: every
+// output element is written by exactly one thread, in a fixed order, without atomics.
+//
+// Source: the walk-through's router ("BiFormer ... 前向传播过程", niftyadmin, section
+// "BRA模块", `TopkRouting`) detaches the region-level query and key when `diff_routing` is
+// off, its default; the top-k index is a discrete choice and r_weight does not scale K or
+// V, so gradients flow through the token-to-token attention and the LCE only. Per image
+// n, query region p and head m, with the routed keys j (the tokens of r_idx[n][p][*]):
+//     s_ij = scale q_i . k_j,   A = softmax_j(s),   D_i = sum_j A_ij dA_ij = dO_i . o_i
+//     dA_ij = dO_i . v_j,       dS_ij = A_ij (dA_ij - D_i)
+//     dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i A_ij dO_i
+//
+// Kernels (bf16 maps, 32 channels per head):
+//   bwd_tc_transpose_kernel: per image, the transposed routing: for every key region the
+//       list of (query region, slot) entries e = p * topk + a that route to it, ascending;
+//   bwd_tc_query_kernel: one CTA per (image, query region, head), a warp per 16 queries.
+//       Three passes over the keys in chunks of 32, recomputing S = Q K^T each time: the
+//       row statistics (max and sum, online), then D = sum A dA (dA = dO V^T), then
+//       dS and dQ = scale dS K. Stores dq and, per query, (lse, D) for the key side;
+//   bwd_tc_key_kernel: one CTA per (image, key region, head), a warp per 16 keys. For each
+//       entry of the key region's list (in list order) it recomputes S^T = K Q^T and
+//       dA^T = V dO^T for the entry's queries, then dK += dS^T Q and dV += A^T dO in
+//       registers; it stores dk and adds dv to the LCE part already stored (so no key is
+//       written by two CTAs).
+// A and dS enter their products split into a bf16 high part and a bf16 low part (two
+// MMAs, about 16 mantissa bits), so that the float32 result is not limited by one bf16
+// rounding of the probabilities; S and dA are exact products of the bf16 inputs.
+//
+// Shared-memory tiles hold rows of 32 channels (64 bytes) with the 64-byte swizzle (16-byte
+// chunk c of row r at c ^ ((r >> 1) & 3)), so that ldmatrix reads of 8 rows are
+// conflict-free. Masked keys (an r_idx entry outside [0, S*S), or padding of the last
+// chunk) take no part in the softmax; padded query rows carry lse = +inf, so their
+// probabilities and gradients are zero.
+#pragma once
+
+#include "common.cuh"
+
+namespace bra {
+
+constexpr int kBwdTcMaxWarps = 16;  // 256 tokens per region
+
+struct BwdTcParams {
+    const __nv_bfloat16 *q, *k, *v, *dout;  // (N,H,W,C)
+    const int32_t *r_idx;                   // (N,P,topk)
+    int *kv_off;                            // (N, P+1): start of each key region's list
+    int *kv_list;                           // (N, P*topk): entries p*topk + a by key region
+    float *dq, *dk, *dv;                    // (N,H,W,C) float32; dv holds the LCE part
+    float *stats;                           // (N,P,heads,w2,2): lse (base 2) and D per query
+    int *bad;                               // set to 1 when an r_idx entry is out of range
+    int N, H, W, C, heads, S, topk, P, hr, wr, w2, L, nw;
+    float scale, sl2;                       // scale and scale * log2(e)
+};
+
+__device__ __forceinline__ uint32_t tc_sw64(int row, int chunk) {
+    return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+
+// Element offset of channel 0 of token t of region r of image n.
+__device__ __forceinline__ size_t tc_pix(const BwdTcParams &p, int n, int r, int t) {
+    const int y = (r / p.S) * p.hr + t / p.wr, x = (r % p.S) * p.wr + t % p.wr;
+    return (((size_t)n * p.H + y) * p.W + x) * p.C;
+}
+
+__device__ __forceinline__ void tc_split(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// ----------------------------------------------------------------------------- routing
+
+// One CTA per image: kv_off[n][pk] .. kv_off[n][pk+1] index the entries e = p * topk + a
+// with r_idx[n][p][a] == pk, in ascending e. Thread pk scans the image's entries in order
+// (from shared memory when they fit), so the order does not depend on scheduling.
+__global__ void __launch_bounds__(256) bwd_tc_transpose_kernel(const BwdTcParams p) {
+    extern __shared__ int tr_s[];  // [P * topk] entries when they fit, then [P + 1] counts
+    const int n = blockIdx.x, E = p.P * p.topk;
+    const int32_t *ri = p.r_idx + (size_t)n * E;
+    const bool staged = E <= 10000;  // staged entries + counts stay within 48 KB
+    int *cnt = tr_s + (staged ? E : 0);
+    if (staged)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) tr_s[e] = ri[e];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int r = ri[e];
+        if (r < 0 || r >= p.P) atomicExch(p.bad, 1);
+    }
+    __syncthreads();
+    for (int pk = threadIdx.x; pk < p.P; pk += blockDim.x) {
+        int c = 0;
+        for (int e = 0; e < E; ++e) c += (staged ? tr_s[e] : ri[e]) == pk;
+        cnt[pk] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        int *off = p.kv_off + (size_t)n * (p.P + 1);
+        for (int pk = 0; pk < p.P; ++pk) {
+            off[pk] = acc;
+            acc += cnt[pk];
+            cnt[pk] = off[pk];
+        }
+        off[p.P] = acc;
+    }
+    __syncthreads();
+    int *list = p.kv_list + (size_t)n * E;
+    for (int pk = threadIdx.x; pk < p.P; pk += blockDim.x) {
+        int w = cnt[pk];
+        for (int e = 0; e < E; ++e)
+            if ((staged ? tr_s[e] : ri[e]) == pk) list[w++] = e;
+    }
+}
+
+// ----------------------------------------------------------------------------- query side
+
+// Shared memory of the query kernel: Q and dO tiles (nw*16 rows), K and V tiles (L
+// rounded up to 32 rows), the routed regions, the per-chunk key masks.
+__host__ __device__ inline int bwd_tc_query_smem(int nw, int L, int topk) {
+    const int Lp = (L + 31) & ~31;
+    return 2 * nw * 16 * 64 + 2 * Lp * 64 + topk * 4 + (Lp / 32) * 4 + 128;
+}
+
+__global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const BwdTcParams p) {
+    extern __shared__ __align__(128) unsigned char tc_q_s[];
+    const int unit = blockIdx.x;
+    const int m = unit % p.heads, npr = unit / p.heads, pr = npr % p.P, n = npr / p.P;
+    const int Rp = p.nw * 16, Lp = (p.L + 31) & ~31, nch = Lp / 32;
+    unsigned char *sQ = tc_q_s, *sO = sQ + Rp * 64, *sK = sO + Rp * 64, *sV = sK + Lp * 64;
+    int *sRoute = reinterpret_cast<int *>(sV + Lp * 64);
+    uint32_t *sMask = reinterpret_cast<uint32_t *>(sRoute + p.topk);
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int c0 = m * 32;
+    for (int a = tid; a < p.topk; a += nthr) {
+        int r = p.r_idx[(size_t)npr * p.topk + a];
+        if (r < 0 || r >= p.P) r = -1;  // flagged by the transpose kernel
+        sRoute[a] = r;
+    }
+    __syncthreads();
+    for (int w = tid; w < nch; w += nthr) {
+        uint32_t mk = 0;
+        for (int b = 0; b < 32; ++b) {
+            const int j = w * 32 + b;
+            if (j < p.L && sRoute[j / p.w2] >= 0) mk |= 1u << b;
+        }
+        sMask[w] = mk;
+    }
+    const uint32_t q_s = smem_u32(sQ), o_s = smem_u32(sO), k_s = smem_u32(sK), v_s = smem_u32(sV);
+    for (int i = tid; i < Rp * 4; i += nthr) {
+        const int row = i >> 2, ch = i & 3;
+        const bool ok = row < p.w2;
+        const size_t g = ok ? tc_pix(p, n, pr, row) + c0 + 8 * ch : 0;
+        cp_async16_s(q_s + tc_sw64(row, ch), p.q + g, ok);
+        cp_async16_s(o_s + tc_sw64(row, ch), p.dout + g, ok);
+    }
+    for (int i = tid; i < Lp * 4; i += nthr) {
+        const int j = i >> 2, ch = i & 3;
+        const int a = j / p.w2, t = j - a * p.w2;
+        const int r = j < p.L ? sRoute[a] : -1;
+        const bool ok = r >= 0;
+        const size_t g = ok ? tc_pix(p, n, r, t) + c0 + 8 * ch : 0;
+        cp_async16_s(k_s + tc_sw64(j, ch), p.k + g, ok);
+        cp_async16_s(v_s + tc_sw64(j, ch), p.v + g, ok);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3, mat = lane >> 3;
+    const int r0 = warp * 16;
+    uint32_t aq[2][4], ado[2][4];
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+        const int row = r0 + (lane & 7) + 8 * (mat & 1), chunk = 2 * kk + (mat >> 1);
+        ldsm_x4(aq[kk][0], aq[kk][1], aq[kk][2], aq[kk][3], sQ + tc_sw64(row, chunk));
+        ldsm_x4(ado[kk][0], ado[kk][1], ado[kk][2], ado[kk][3], sO + tc_sw64(row, chunk));
+    }
+    // S (or dA) of the 32-key chunk kc: acc[n-tile][c0..c3], rows g / g + 8, key 8 nt + 2 tq (+1)
+    auto chunk_mma = [&](const uint32_t (&af)[2][4], const unsigned char *tile, int kc, float (&acc)[4][4]) {
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+            for (int hp = 0; hp < 2; ++hp) {
+                const int key = kc * 32 + 16 * hp + (lane & 7) + 8 * (mat >> 1), chunk = 2 * kk + (mat & 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(b0, b1, b2, b3, tile + tc_sw64(key, chunk));
+                mma_bf16_16816(acc[2 * hp], af[kk], b0, b1);
+                mma_bf16_16816(acc[2 * hp + 1], af[kk], b2, b3);
+            }
+    };
+    // scaled logits (base 2) of the chunk, -inf where the key is masked
+    auto logits = [&](int kc, float (&s)[4][4]) {
+        chunk_mma(aq, sK, kc, s);
+        const uint32_t mk = sMask[kc];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                s[nt][e] = ((mk >> (8 * nt + 2 * tq + (e & 1))) & 1u) ? s[nt][e] * p.sl2 : -INFINITY;
+    };
+    // pass 1: row max and sum (online); this thread holds rows g (e < 2) and g + 8 (e >= 2)
+    float mx[2] = {-INFINITY, -INFINITY}, sm[2] = {0.f, 0.f};
+    for (int kc = 0; kc < nch; ++kc) {
+        float s[4][4];
+        logits(kc, s);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float cm = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) cm = fmaxf(cm, fmaxf(s[nt][2 * h], s[nt][2 * h + 1]));
+            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+            const float mn = fmaxf(mx[h], cm);
+            if (mn == -INFINITY) continue;  // every key so far masked
+            float acc = mx[h] == -INFINITY ? 0.f : sm[h] * exp2f(mx[h] - mn);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) acc += exp2f(s[nt][2 * h] - mn) + exp2f(s[nt][2 * h + 1] - mn);
+            sm[h] = acc;
+            mx[h] = mn;
+        }
+    }
+    float lse[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float t = sm[h];
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        lse[h] = t > 0.f ? mx[h] + log2f(t) : INFINITY;  // no valid key: probabilities 0
+    }
+    // probabilities and dA of chunk kc
+    auto probs = [&](int kc, float (&a)[4][4], float (&da)[4][4]) {
+        logits(kc, a);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) a[nt][e] = exp2f(a[nt][e] - lse[e >> 1]);
+        chunk_mma(ado, sV, kc, da);
+    };
+    // pass 2: D = sum_j A dA
+    float dsum[2] = {0.f, 0.f};
+    for (int kc = 0; kc < nch; ++kc) {
+        float a[4][4], da[4][4];
+        probs(kc, a, da);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dsum[e >> 1] = fmaf(a[nt][e], da[nt][e], dsum[e >> 1]);
+    }
+    float D[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float t = dsum[h];
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        D[h] = t;
+    }
+    // pass 3: dS and dQ += dS K (keys as the contraction index)
+    float dqa[4][4];
+#pragma unroll
+    for (int ct = 0; ct < 4; ++ct)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dqa[ct][e] = 0.f;
+    for (int kc = 0; kc < nch; ++kc) {
+        float a[4][4], da[4][4];
+        probs(kc, a, da);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int nt = 2 * ks + u;
+                tc_split(a[nt][0] * (da[nt][0] - D[0]), a[nt][1] * (da[nt][1] - D[0]), hi[2 * u], lo[2 * u]);
+                tc_split(a[nt][2] * (da[nt][2] - D[1]), a[nt][3] * (da[nt][3] - D[1]), hi[2 * u + 1], lo[2 * u + 1]);
+            }
+#pragma unroll
+            for (int cp2 = 0; cp2 < 2; ++cp2) {
+                const int key = kc * 32 + 16 * ks + (lane & 7) + 8 * (mat & 1), chunk = 2 * cp2 + (mat >> 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(b0, b1, b2, b3, sK + tc_sw64(key, chunk));
+                mma_bf16_16816(dqa[2 * cp2], hi, b0, b1);
+                mma_bf16_16816(dqa[2 * cp2], lo, b0, b1);
+                mma_bf16_16816(dqa[2 * cp2 + 1], hi, b2, b3);
+                mma_bf16_16816(dqa[2 * cp2 + 1], lo, b2, b3);
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int row = r0 + g + 8 * h;
+        if (row >= p.w2) continue;
+        float *dst = p.dq + tc_pix(p, n, pr, row) + c0;
+#pragma unroll
+        for (int ct = 0; ct < 4; ++ct)
+            *reinterpret_cast<float2 *>(dst + 8 * ct + 2 * tq) =
+                make_float2(p.scale * dqa[ct][2 * h], p.scale * dqa[ct][2 * h + 1]);
+        if (tq == 0)
+            *reinterpret_cast<float2 *>(p.stats + (((size_t)npr * p.heads + m) * p.w2 + row) * 2) =
+                make_float2(lse[h], D[h]);
+    }
+}
+
+// ----------------------------------------------------------------------------- key side
+
+// Shared memory of the key kernel: K and V tiles (nw*16 rows), two stages of the
+// entry's Q and dO tiles (Rp = w2 rounded up to 16 rows) and its per-query (lse, D).
+__host__ __device__ inline int bwd_tc_key_smem(int nw, int w2) {
+    const int Rp = (w2 + 15) & ~15;
+    return 2 * nw * 16 * 64 + 2 * (2 * Rp * 64 + Rp * 8) + 128;
+}
+
+__global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const BwdTcParams p) {
+    extern __shared__ __align__(128) unsigned char tc_k_s[];
+    const int unit = blockIdx.x;
+    const int m = unit % p.heads, npk = unit / p.heads, pk = npk % p.P, n = npk / p.P;
+    const int Kp = p.nw * 16, Rp = (p.w2 + 15) & ~15;
+    unsigned char *sK = tc_k_s, *sV = sK + Kp * 64, *stage0 = sV + Kp * 64;
+    const int stage_bytes = 2 * Rp * 64 + Rp * 8;
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int c0 = m * 32;
+    const int *off = p.kv_off + (size_t)n * (p.P + 1);
+    const int e0 = off[pk], cnt = off[pk + 1] - e0;
+    const int *list = p.kv_list + (size_t)n * p.P * p.topk + e0;
+    const uint32_t k_s = smem_u32(sK), v_s = smem_u32(sV);
+    for (int i = tid; i < Kp * 4; i += nthr) {
+        const int row = i >> 2, ch = i & 3;
+        const bool ok = row < p.w2;
+        const size_t g = ok ? tc_pix(p, n, pk, row) + c0 + 8 * ch : 0;
+        cp_async16_s(k_s + tc_sw64(row, ch), p.k + g, ok);
+        cp_async16_s(v_s + tc_sw64(row, ch), p.v + g, ok);
+    }
+    // the entry's queries: Q and dO rows, (lse, D) per row (padding: lse = +inf, D = 0)
+    auto load_entry = [&](int idx, int s) {
+        unsigned char *st = stage0 + s * stage_bytes;
+        const uint32_t sq = smem_u32(st), so = sq + Rp * 64;
+        float2 *sst = reinterpret_cast<float2 *>(st + 2 * Rp * 64);
+        const int pr = list[idx] / p.topk;
+        for (int i = tid; i < Rp * 4; i += nthr) {
+            const int row = i >> 2, ch = i & 3;
+            const bool ok = row < p.w2;
+            const size_t g = ok ? tc_pix(p, n, pr, row) + c0 + 8 * ch : 0;
+            cp_async16_s(sq + tc_sw64(row, ch), p.q + g, ok);
+            cp_async16_s(so + tc_sw64(row, ch), p.dout + g, ok);
+        }
+        for (int row = tid; row < Rp; row += nthr)
+            sst[row] = row < p.w2 ? *reinterpret_cast<const float2 *>(
+                                        p.stats + ((((size_t)n * p.P + pr) * p.heads + m) * p.w2 + row) * 2)
+                                  : make_float2(INFINITY, 0.f);
+    };
+    if (cnt > 0) load_entry(0, 0);
+    cp_async_commit();
+
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3, mat = lane >> 3;
+    const int k0 = warp * 16;
+    float dka[4][4], dva[4][4];
+#pragma unroll
+    for (int ct = 0; ct < 4; ++ct)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dka[ct][e] = dva[ct][e] = 0.f;
+    uint32_t ak[2][4], av[2][4];
+    for (int idx = 0; idx < cnt; ++idx) {
+        if (idx + 1 < cnt) load_entry(idx + 1, (idx + 1) & 1);  // the other stage is free
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        if (idx == 0) {
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+                const int row = k0 + (lane & 7) + 8 * (mat & 1), chunk = 2 * kk + (mat >> 1);
+                ldsm_x4(ak[kk][0], ak[kk][1], ak[kk][2], ak[kk][3], sK + tc_sw64(row, chunk));
+                ldsm_x4(av[kk][0], av[kk][1], av[kk][2], av[kk][3], sV + tc_sw64(row, chunk));
+            }
+        }
+        const unsigned char *sQ = stage0 + (idx & 1) * stage_bytes, *sO = sQ + Rp * 64;
+        const float2 *sst = reinterpret_cast<const float2 *>(sQ + 2 * Rp * 64);
+        for (int qc = 0; qc < Rp / 16; ++qc) {
+            // S^T and dA^T of these 16 keys x 16 queries: rows = keys g / g + 8, columns =
+            // queries 16 qc + 8 nt + 2 tq (+1)
+            float sT[2][4], dT[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sT[nt][e] = dT[nt][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+                const int row = qc * 16 + (lane & 7) + 8 * (mat >> 1), chunk = 2 * kk + (mat & 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(b0, b1, b2, b3, sQ + tc_sw64(row, chunk));
+                mma_bf16_16816(sT[0], ak[kk], b0, b1);
+                mma_bf16_16816(sT[1], ak[kk], b2, b3);
+                ldsm_x4(b0, b1, b2, b3, sO + tc_sw64(row, chunk));
+                mma_bf16_16816(dT[0], av[kk], b0, b1);
+                mma_bf16_16816(dT[1], av[kk], b2, b3);
+            }
+            uint32_t dh[4], dl[4], ah[4], al[4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const float2 st0 = sst[qc * 16 + 8 * nt + 2 * tq], st1 = sst[qc * 16 + 8 * nt + 2 * tq + 1];
+                float a[4], ds[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 st = (e & 1) ? st1 : st0;
+                    a[e] = exp2f(sT[nt][e] * p.sl2 - st.x);
+                    ds[e] = a[e] * (dT[nt][e] - st.y);
+                }
+                // A fragments (keys x queries, k = queries): this tile's columns are k 8 nt + 2 tq
+                tc_split(ds[0], ds[1], dh[2 * nt], dl[2 * nt]);
+                tc_split(ds[2], ds[3], dh[2 * nt + 1], dl[2 * nt + 1]);
+                tc_split(a[0], a[1], ah[2 * nt], al[2 * nt]);
+                tc_split(a[2], a[3], ah[2 * nt + 1], al[2 * nt + 1]);
+            }
+#pragma unroll
+            for (int cp2 = 0; cp2 < 2; ++cp2) {
+                const int row = qc * 16 + (lane & 7) + 8 * (mat & 1), chunk = 2 * cp2 + (mat >> 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(b0, b1, b2, b3, sQ + tc_sw64(row, chunk));
+                mma_bf16_16816(dka[2 * cp2], dh, b0, b1);
+                mma_bf16_16816(dka[2 * cp2], dl, b0, b1);
+                mma_bf16_16816(dka[2 * cp2 + 1], dh, b2, b3);
+                mma_bf16_16816(dka[2 * cp2 + 1], dl, b2, b3);
+                ldsm_x4_t(b0, b1, b2, b3, sO + tc_sw64(row, chunk));
+                mma_bf16_16816(dva[2 * cp2], ah, b0, b1);
+                mma_bf16_16816(dva[2 * cp2], al, b0, b1);
+                mma_bf16_16816(dva[2 * cp2 + 1], ah, b2, b3);
+                mma_bf16_16816(dva[2 * cp2 + 1], al, b2, b3);
+            }
+        }
+        __syncthreads();  // the stage is read: the next prefetch may overwrite it
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int row = k0 + g + 8 * h;
+        if (row >= p.w2) continue;
+        const size_t o = tc_pix(p, n, pk, row) + c0;
+#pragma unroll
+        for (int ct = 0; ct < 4; ++ct) {
+            const int c = 8 * ct + 2 * tq;
+            *reinterpret_cast<float2 *>(p.dk + o + c) = make_float2(p.scale * dka[ct][2 * h], p.scale * dka[ct][2 * h + 1]);
+            float2 *dv = reinterpret_cast<float2 *>(p.dv + o + c);
+            const float2 lce = *dv;
+            *dv = make_float2(lce.x + dva[ct][2 * h], lce.y + dva[ct][2 * h + 1]);
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- LCE parameters
+
+// dw[c][a][b] = sum over images and pixels of dout[n,y,x,c] V[n, y+a-2, x+b-2, c] (zero
+// outside), db[c] = sum of dout[..., c]: per (row block b, image n) a CTA writes the partial
+// sums of its kBwdLceRows rows, thread = channel (coalesced across the warp); a second
+// kernel adds the partials of each (channel, tap) in a fixed order.
+constexpr int kBwdLceRows = 4;
+
+__global__ void __launch_bounds__(256) bwd_tc_lce_partial_kernel(const BwdTcParams p, float *part, int nb) {
+    const int b = blockIdx.x, n = blockIdx.y;
+    const int y0 = b * kBwdLceRows, y1 = min(p.H, y0 + kBwdLceRows);
+    for (int c = threadIdx.x; c < p.C; c += blockDim.x) {
+        float acc[26];
+#pragma unroll
+        for (int t = 0; t < 26; ++t) acc[t] = 0.f;
+        for (int y = y0; y < y1; ++y)
+            for (int x = 0; x < p.W; ++x) {
+                const float d = __bfloat162float(p.dout[(((size_t)n * p.H + y) * p.W + x) * p.C + c]);
+                acc[25] += d;
+#pragma unroll
+                for (int a = 0; a < 5; ++a) {
+                    const int yy = y + a - 2;
+                    if (yy < 0 || yy >= p.H) continue;
+#pragma unroll
+                    for (int bb = 0; bb < 5; ++bb) {
+                        const int xx = x + bb - 2;
+                        if (xx < 0 || xx >= p.W) continue;
+                        acc[a * 5 + bb] =
+                            fmaf(d, __bfloat162float(p.v[(((size_t)n * p.H + yy) * p.W + xx) * p.C + c]), acc[a * 5 + bb]);
+                    }
+                }
+            }
+        float *dst = part + (((size_t)n * nb + b) * p.C + c) * 26;
+#pragma unroll
+        for (int t = 0; t < 26; ++t) dst[t] = acc[t];
+    }
+}
+
+__global__ void __launch_bounds__(256) bwd_tc_lce_final_kernel(const float *part, int nparts, int C, float *dw,
+                                                                float *db) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= C * 26) return;
+    const int c = i / 26, t = i - c * 26;
+    float s = 0.f;
+    for (int k = 0; k < nparts; ++k) s += part[((size_t)k * C + c) * 26 + t];
+    if (t < 25)
+        dw[c * 25 + t] = s;
+    else
+        db[c] = s;
+}
+
+}  // namespace bra

@@ -34,6 +34,7 @@
 #include "attn_tma.cuh"
 #include "attn_umma.cuh"
 #include "backward.cuh"
+#include "backward_tc.cuh"
 #include "block.cuh"
 #include "fused_image.cuh"
 #include "linear.cuh"
@@ -202,6 +203,11 @@ template <typename K> static cudaError_t allow_smem(K kern, int bytes) {
     auto it = g_smem_set.find(key);
     if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    // every kernel with dynamic shared memory asks for the same (largest) carveout, so that
+    // consecutive kernels of a forward do not make the SMs change their L1 / shared split
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess) g_smem_set[key] = bytes;
     return e;
 }
@@ -339,9 +345,11 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
     // more than 128 regions: the column-per-lane kernel with 4 or 8 rows per CTA
     const int cols_rows = (long long)s.N * ((s.P + 7) / 8) >= sms ? 8 : 4;
     const int rows = E == 8 ? cols_rows : kRouteWarps * rpw;
+    // route_kernel stages key means in passes of cc channels; route_cols_kernel reads them
+    // straight into registers
     int cc = route_chunk(32 * E, rows, s.C);
     while (s.C % cc) cc -= 32;  // equal passes: one divisor for the staging index
-    const int smem = route_smem_bytes(32 * E, rows, cc);
+    const int smem = E == 8 ? route_cols_smem_bytes(rows, s.C) : route_smem_bytes(32 * E, rows, cc);
     const FastDiv div_q4((uint32_t)(cc / 4));
     int rc = BRA_OK;
     auto go = [&](auto kern) {
@@ -354,19 +362,35 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
             const dim3 g((s.P + rows - 1) / rows, nb, 1);
             LaunchScope ls(BRA_KERNEL_ROUTE, st);
             if (launch_pdl(kern, g, dim3(kRouteWarps * 32), smem, st, (const float *)(ws + (size_t)n0 * s.P * s.C),
+                           (const float *)(ws + pooled + (size_t)n0 * s.P * s.C), s.C, s.P, s.topk, scale,
+                           r_idx + (size_t)n0 * s.P * s.topk, r_weight + (size_t)n0 * s.P * s.topk) != cudaSuccess)
+                rc = BRA_ERR_CUDA;
+        }
+    };
+    auto go_staged = [&](auto kern) {
+        if (allow_smem(kern, smem) != cudaSuccess) {
+            rc = BRA_ERR_CUDA;
+            return;
+        }
+        for (int n0 = 0; n0 < s.N && rc == BRA_OK; n0 += 65535) {
+            const int nb = s.N - n0 < 65535 ? s.N - n0 : 65535;
+            const dim3 g((s.P + rows - 1) / rows, nb, 1);
+            LaunchScope ls(BRA_KERNEL_ROUTE, st);
+            if (launch_pdl(kern, g, dim3(kRouteWarps * 32), smem, st, (const float *)(ws + (size_t)n0 * s.P * s.C),
                            (const float *)(ws + pooled + (size_t)n0 * s.P * s.C), s.C, s.P, s.topk, cc, scale,
-                           r_idx + (size_t)n0 * s.P * s.topk, r_weight + (size_t)n0 * s.P * s.topk, div_q4) != cudaSuccess)
+                           r_idx + (size_t)n0 * s.P * s.topk, r_weight + (size_t)n0 * s.P * s.topk, div_q4) !=
+                cudaSuccess)
                 rc = BRA_ERR_CUDA;
         }
     };
     auto by_rpw = [&](auto e_tag) {
         constexpr int EE = decltype(e_tag)::value;
         if (rpw == 4)
-            go(route_kernel<EE, 4>);
+            go_staged(route_kernel<EE, 4>);
         else if (rpw == 2)
-            go(route_kernel<EE, 2>);
+            go_staged(route_kernel<EE, 2>);
         else
-            go(route_kernel<EE, 1>);
+            go_staged(route_kernel<EE, 1>);
     };
     if (E == 1)
         by_rpw(std::integral_constant<int, 1>{});
@@ -1097,11 +1121,14 @@ int bra_set_kernel_variant(int variant) {
 int bra_device_status(bra_stream_t stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return BRA_ERR_CUDA;
-    int flag = 0;
+    int flag = 0, index = 0;
     const int zero = 0;
-    if (cudaMemcpyFromSymbol(&flag, g_bra_timeout_flag, sizeof(int)) != cudaSuccess) return BRA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&flag, g_bra_timeout_flag, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&index, g_bra_index_flag, sizeof(int)) != cudaSuccess)
+        return BRA_ERR_CUDA;
     if (flag && cudaMemcpyToSymbol(g_bra_timeout_flag, &zero, sizeof(int)) != cudaSuccess) return BRA_ERR_CUDA;
-    return flag ? BRA_ERR_TIMEOUT : BRA_OK;
+    if (index && cudaMemcpyToSymbol(g_bra_index_flag, &zero, sizeof(int)) != cudaSuccess) return BRA_ERR_CUDA;
+    return flag ? BRA_ERR_TIMEOUT : index ? BRA_ERR_INDEX : BRA_OK;
 }
 
 int bra_selftest_wait_timeout(unsigned polls, bra_stream_t stream) {
@@ -1449,9 +1476,121 @@ int bra_block(const void *x, const void *pos_w, const void *pos_b, const void *l
     return rc;
 }
 
-int bra_backward(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
-                 const void *dout, int N, int H, int W, int C, int heads, int S, int topk, int dtype, float *dq,
-                 float *dk, float *dv, float *dlce_w, float *dlce_b, bra_stream_t stream) {
+// Device address of the library's out-of-range flag (g_bra_index_flag) on the current device.
+static int index_flag(int **out) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bra_index_flag) != cudaSuccess || p == nullptr) return BRA_ERR_CUDA;
+    *out = static_cast<int *>(p);
+    return BRA_OK;
+}
+
+// The backward on the tensor cores (bf16 maps, 32 channels per head), deterministic: the
+// transposed routing, the LCE part of dv, the query-side pass (dq and the per-query
+// statistics), the key-side pass (dk, and dv added to its LCE part), the LCE parameter
+// gradients (partials, then a fixed-order sum). Scratch from the library's pool outside a
+// capture. Synchronises `stream` to read the out-of-range flag, as the other backward.
+static int backward_tc(const Shape &s, const void *q, const void *k, const void *v, const void *lce_w,
+                       const int32_t *r_idx, const void *dout, float *dq, float *dk, float *dv, float *dlce_w,
+                       float *dlce_b, cudaStream_t st, bool sync) {
+    const int nw = (s.w2 + 15) / 16;
+    if (nw > kBwdTcMaxWarps) return BRA_ERR_SHAPE;
+    const int L = s.topk * s.w2;
+    const int nb = (s.H + kBwdLceRows - 1) / kBwdLceRows;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t b_off = up((size_t)s.N * (s.P + 1) * 4), b_list = up((size_t)s.N * s.P * s.topk * 4);
+    const size_t b_stats = up((size_t)s.N * s.P * s.heads * s.w2 * 8), b_part = up((size_t)s.N * nb * s.C * 26 * 4);
+    unsigned char *buf = nullptr;
+    int rc = scratch_alloc(&buf, b_off + b_list + b_stats + b_part + 256, st);
+    if (rc) return rc;
+    BwdTcParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.dout = static_cast<const __nv_bfloat16 *>(dout);
+    p.r_idx = r_idx;
+    p.kv_off = reinterpret_cast<int *>(buf);
+    p.kv_list = reinterpret_cast<int *>(buf + b_off);
+    p.stats = reinterpret_cast<float *>(buf + b_off + b_list);
+    float *part = reinterpret_cast<float *>(buf + b_off + b_list + b_stats);
+    // the out-of-range flag: per call (read back here) or the library's device flag
+    p.bad = reinterpret_cast<int *>(buf + b_off + b_list + b_stats + b_part);
+    if (!sync && (rc = index_flag(&p.bad))) {
+        cudaFreeAsync(buf, st);
+        return rc;
+    }
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.N = s.N;
+    p.H = s.H;
+    p.W = s.W;
+    p.C = s.C;
+    p.heads = s.heads;
+    p.S = s.S;
+    p.topk = s.topk;
+    p.P = s.P;
+    p.hr = s.hr;
+    p.wr = s.wr;
+    p.w2 = s.w2;
+    p.L = L;
+    p.nw = nw;
+    p.scale = 1.0f / sqrtf((float)s.d);
+    p.sl2 = p.scale * 1.4426950408889634f;
+    // the LCE part of dv through the SIMT kernel of the other path (one thread per element)
+    const BwdParams lp = make_bwd_params(q, k, v, dout, lce_w, r_idx, s.N, s.H, s.W, s.C, s.heads, s.S, s.topk, 1,
+                                         dq, dk, dv, dlce_w, dlce_b, p.bad);
+    int sms = 0;
+    if ((rc = sm_count(&sms)) == BRA_OK) {
+        const int tr_smem = ((s.P * s.topk <= 10000 ? s.P * s.topk : 0) + s.P + 1) * 4;
+        const int q_smem = bwd_tc_query_smem(nw, L, s.topk), k_smem = bwd_tc_key_smem(nw, s.w2);
+        const size_t elems = (size_t)s.N * s.H * s.W * s.C;
+        const unsigned units = (unsigned)((size_t)s.N * s.P * s.heads);
+        if ((sync && cudaMemsetAsync(p.bad, 0, sizeof(int), st) != cudaSuccess) ||
+            allow_smem(bwd_tc_query_kernel, q_smem) != cudaSuccess ||
+            allow_smem(bwd_tc_key_kernel, k_smem) != cudaSuccess) {
+            rc = BRA_ERR_CUDA;
+        } else {
+            {
+                LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+                bwd_tc_transpose_kernel<<<s.N, 256, tr_smem, st>>>(p);
+            }
+            {
+                LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+                bwd_lce_dv_kernel<<<(unsigned)std::min<size_t>((elems + 255) / 256, (size_t)sms * 8), 256, 0, st>>>(lp);
+            }
+            {
+                LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+                bwd_tc_query_kernel<<<units, 32 * nw, q_smem, st>>>(p);
+            }
+            {
+                LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+                bwd_tc_key_kernel<<<units, 32 * nw, k_smem, st>>>(p);
+            }
+            {
+                LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+                bwd_tc_lce_partial_kernel<<<dim3(nb, s.N), std::min(256, (s.C + 31) / 32 * 32), 0, st>>>(p, part, nb);
+            }
+            {
+                LaunchScope ls(BRA_KERNEL_BACKWARD, st);
+                bwd_tc_lce_final_kernel<<<(s.C * 26 + 255) / 256, 256, 0, st>>>(part, s.N * nb, s.C, dlce_w, dlce_b);
+            }
+            if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
+        }
+    }
+    int host_flag = 0;
+    if (sync && rc == BRA_OK &&
+        cudaMemcpyAsync(&host_flag, p.bad, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        rc = BRA_ERR_CUDA;
+    if (cudaFreeAsync(buf, st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    if (sync && cudaStreamSynchronize(st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
+    if (rc == BRA_OK && host_flag) rc = BRA_ERR_INDEX;
+    return rc;
+}
+
+static int backward_impl(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
+                         const void *dout, int N, int H, int W, int C, int heads, int S, int topk, int dtype,
+                         float *dq, float *dk, float *dv, float *dlce_w, float *dlce_b, bra_stream_t stream,
+                         bool sync) {
     const Shape s = make_shape(N, H, W, C, heads, S, topk, dtype);
     int rc = check_shape(s);
     if (rc) return rc;
@@ -1472,12 +1611,15 @@ int bra_backward(const void *q, const void *k, const void *v, const void *lce_w,
         return BRA_ERR_ALIGN;
     int sms = 0;
     if ((rc = sm_count(&sms))) return rc;
-    int *flag = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&flag), sizeof(int), st) != cudaSuccess) return BRA_ERR_CUDA;
+    if (dtype == BRA_BF16 && s.d == 32) return backward_tc(s, q, k, v, lce_w, r_idx, dout, dq, dk, dv, dlce_w, dlce_b, st, sync);
+    int *flag = nullptr;  // per call (read back here), or the library's device flag
+    if (sync ? cudaMallocAsync(reinterpret_cast<void **>(&flag), sizeof(int), st) != cudaSuccess
+             : index_flag(&flag) != BRA_OK)
+        return BRA_ERR_CUDA;
     const BwdParams p = make_bwd_params(q, k, v, dout, lce_w, r_idx, N, H, W, C, heads, S, topk, dtype == BRA_BF16,
                                         dq, dk, dv, dlce_w, dlce_b, flag);
     const size_t elems = bwd_elems(p), items = bwd_attn_items(p);
-    rc = cudaMemsetAsync(flag, 0, sizeof(int), st) == cudaSuccess &&
+    rc = (!sync || cudaMemsetAsync(flag, 0, sizeof(int), st) == cudaSuccess) &&
                  cudaMemsetAsync(dk, 0, elems * sizeof(float), st) == cudaSuccess
              ? BRA_OK
              : BRA_ERR_CUDA;
@@ -1496,6 +1638,7 @@ int bra_backward(const void *q, const void *k, const void *v, const void *lce_w,
         }
         if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
     }
+    if (!sync) return rc;
     int host_flag = 0;
     if (rc == BRA_OK &&
         cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
@@ -1504,6 +1647,20 @@ int bra_backward(const void *q, const void *k, const void *v, const void *lce_w,
     if (cudaStreamSynchronize(st) != cudaSuccess && rc == BRA_OK) rc = BRA_ERR_CUDA;
     if (rc == BRA_OK && host_flag) rc = BRA_ERR_INDEX;
     return rc;
+}
+
+int bra_backward(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
+                 const void *dout, int N, int H, int W, int C, int heads, int S, int topk, int dtype, float *dq,
+                 float *dk, float *dv, float *dlce_w, float *dlce_b, bra_stream_t stream) {
+    return backward_impl(q, k, v, lce_w, r_idx, dout, N, H, W, C, heads, S, topk, dtype, dq, dk, dv, dlce_w, dlce_b,
+                         stream, true);
+}
+
+int bra_backward_async(const void *q, const void *k, const void *v, const void *lce_w, const int32_t *r_idx,
+                       const void *dout, int N, int H, int W, int C, int heads, int S, int topk, int dtype,
+                       float *dq, float *dk, float *dv, float *dlce_w, float *dlce_b, bra_stream_t stream) {
+    return backward_impl(q, k, v, lce_w, r_idx, dout, N, H, W, C, heads, S, topk, dtype, dq, dk, dv, dlce_w, dlce_b,
+                         stream, false);
 }
 
 int bra_attend(const void *q, const void *k, const void *v, const void *lce_w, const void *lce_b, int N,

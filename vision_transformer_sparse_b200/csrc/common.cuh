@@ -7,6 +7,12 @@
 
 namespace bra {
 
+// Set by any kernel whose bounded wait ran out; read and cleared by bra_device_status.
+__device__ int g_bra_timeout_flag = 0;
+// Set by bra_backward_async's kernels when an r_idx entry lies outside [0, S*S); read and
+// cleared by bra_device_status.
+__device__ int g_bra_index_flag = 0;
+
 // ----------------------------------------------------------------------------- element types
 
 template <typename T> struct Elem;

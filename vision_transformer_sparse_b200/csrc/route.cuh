@@ -168,6 +168,9 @@ inline int route_smem_bytes(int PP, int rows, int cc) {
     return (tile > dots ? tile : dots) * 4;
 }
 
+// Shared memory of route_cols_kernel: the scaled query means and the logits of its rows.
+inline int route_cols_smem_bytes(int rows, int C) { return (rows * C + rows * 256) * 4; }
+
 // Top-k selection and softmax of one affinity row (dots: the row's PP = 32E logits in
 // shared memory), run by one warp; writes topk (index, weight) pairs at out_idx /
 // out_w. topk <= 8 by repeated warp argmax, larger topk by a bitonic sort of all 32E
@@ -391,13 +394,14 @@ route_kernel(const float *__restrict__ q_r, const float *__restrict__ k_r, int C
 }
 
 // Many regions (32E = 256 columns): one CTA per (image n, block of ROWS affinity rows),
-// eight warps; warp w owns the 32 columns 32w + lane for all ROWS rows, so every key
-// float4 read from shared memory feeds 4*ROWS FMAs (the query float4s are broadcast).
-// Staging, layout and the selection are those of route_kernel.
+// eight warps; thread t owns column t for all ROWS rows. It loads its own column's key
+// means straight into registers, 64 channels at a time (16 independent float4 loads in
+// flight), and multiplies them with the ROWS scaled query means broadcast from shared
+// memory; no key mean is staged. Selection as in route_kernel.
 template <int ROWS>
 __global__ void __launch_bounds__(kRouteWarps * 32)
-route_cols_kernel(const float *__restrict__ q_r, const float *__restrict__ k_r, int C, int P, int topk, int cc,
-                  float scale, int32_t *__restrict__ r_idx, float *__restrict__ r_weight, FastDiv div_q4) {
+route_cols_kernel(const float *__restrict__ q_r, const float *__restrict__ k_r, int C, int P, int topk, float scale,
+                  int32_t *__restrict__ r_idx, float *__restrict__ r_weight) {
     extern __shared__ __align__(16) float route_s[];
     constexpr int E = 8, PP = 32 * E;
     griddep_wait();               // pooled means come from the preceding kernel
@@ -407,65 +411,46 @@ route_cols_kernel(const float *__restrict__ q_r, const float *__restrict__ k_r, 
     const int p0 = blockIdx.x * ROWS;
     const float *kimg = k_r + (size_t)n * P * C;
     const float *qimg = q_r + (size_t)n * P * C;
-    const int kp = cc + 4;
-    float *kr_s = route_s;           // [PP][kp]
-    float *q_s = route_s + PP * kp;  // [ROWS][cc]
-    const int col = warp * 32 + lane;
-
+    float *q_s = route_s;              // [ROWS][C]
+    float *dots = route_s + ROWS * C;  // [ROWS][PP]
+    const int col = threadIdx.x;
+    const float4 *kc = reinterpret_cast<const float4 *>(kimg + (size_t)min(col, P - 1) * C);
+    float4 kv[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) kv[b] = 4 * b < C ? __ldg(kc + b) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int c4n = C >> 2;
+    for (int i = threadIdx.x; i < ROWS * c4n; i += blockDim.x) {
+        const int r = i / c4n, c4 = i - r * c4n;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p0 + r < P) v = __ldg(reinterpret_cast<const float4 *>(qimg + (size_t)(p0 + r) * C) + c4);
+        v.x *= scale;  // the walk-through scales the region query before the product
+        v.y *= scale;
+        v.z *= scale;
+        v.w *= scale;
+        reinterpret_cast<float4 *>(q_s + r * C)[c4] = v;
+    }
+    __syncthreads();
     float dot[ROWS];
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) dot[r] = 0.f;
-
-    for (int c0 = 0; c0 < C; c0 += cc) {
-        const int cw = min(cc, C - c0), q4 = cw >> 2;
-        __syncthreads();
-        for (int i0 = threadIdx.x; i0 < (PP + ROWS) * q4; i0 += 8 * blockDim.x) {
-            float4 buf[8];
-            int rr[8], cc4[8];
+    for (int c0 = 0; c0 < C; c0 += 64) {
+        if (c0 > 0) {
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                const int idx = i0 + b * blockDim.x;
-                uint32_t cm;
-                rr[b] = (int)div_q4.divmod((uint32_t)idx, cm);
-                cc4[b] = (int)cm * 4;
-                buf[b] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (rr[b] < P) {
-                    buf[b] = __ldg(reinterpret_cast<const float4 *>(kimg + (size_t)rr[b] * C + c0 + cc4[b]));
-                } else if (rr[b] >= PP && rr[b] < PP + ROWS) {
-                    buf[b] = __ldg(reinterpret_cast<const float4 *>(qimg + (size_t)min(p0 + rr[b] - PP, P - 1) * C + c0 +
-                                                                   cc4[b]));
-                }
-            }
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                if (rr[b] < PP) {
-                    *reinterpret_cast<float4 *>(kr_s + rr[b] * kp + cc4[b]) = buf[b];
-                } else if (rr[b] < PP + ROWS) {
-                    float4 v = buf[b];
-                    v.x *= scale;  // the walk-through scales the region query before the product
-                    v.y *= scale;
-                    v.z *= scale;
-                    v.w *= scale;
-                    *reinterpret_cast<float4 *>(q_s + (rr[b] - PP) * cc + cc4[b]) = v;
-                }
-            }
+            for (int b = 0; b < 16; ++b) kv[b] = c0 + 4 * b < C ? __ldg(kc + c0 / 4 + b) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        __syncthreads();
-        for (int c = 0; c < cw; c += 4) {
-            const float4 kv = *reinterpret_cast<const float4 *>(kr_s + col * kp + c);
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+            if (c0 + 4 * b >= C) break;
 #pragma unroll
             for (int r = 0; r < ROWS; ++r) {
-                const float4 qv = *reinterpret_cast<const float4 *>(q_s + r * cc + c);
-                dot[r] = fmaf(qv.x, kv.x, dot[r]);
-                dot[r] = fmaf(qv.y, kv.y, dot[r]);
-                dot[r] = fmaf(qv.z, kv.z, dot[r]);
-                dot[r] = fmaf(qv.w, kv.w, dot[r]);
+                const float4 qv = *reinterpret_cast<const float4 *>(q_s + r * C + c0 + 4 * b);
+                dot[r] = fmaf(qv.x, kv[b].x, dot[r]);
+                dot[r] = fmaf(qv.y, kv[b].y, dot[r]);
+                dot[r] = fmaf(qv.z, kv[b].z, dot[r]);
+                dot[r] = fmaf(qv.w, kv[b].w, dot[r]);
             }
         }
     }
-
-    __syncthreads();
-    float *dots = route_s;  // [ROWS][PP]
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) dots[r * PP + col] = dot[r];
     __syncthreads();

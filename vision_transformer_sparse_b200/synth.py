@@ -34,6 +34,12 @@ the output projection after it) draw the layer input x instead of q, k, v:
     layer output have unit scale; both biases ~ N(0, 0.02^2);
   * LCE weight and bias as above; slots x=8, x offset=9, qkv weight/bias=10/11,
     output weight/bias=12/13.
+
+BiFormer-block inputs (make_block_inputs) add the block's own parameters to the layer's:
+  * pos-embed depthwise 3x3 weight ~ N(0, 0.2^2), bias ~ N(0, 0.05^2);
+  * LayerNorm gains 1 + N(0, 0.1^2), shifts ~ N(0, 0.05^2);
+  * MLP weights (3C, C) ~ N(0, 1/C) and (C, 3C) ~ N(0, 1/(3C)), biases ~ N(0, 0.02^2);
+  * slots 14-23.
 """
 from __future__ import annotations
 
@@ -43,7 +49,9 @@ from typing import Dict, Optional
 import numpy as np
 
 SLOT = {"q": 0, "k": 1, "v": 2, "lce_w": 3, "lce_b": 4, "q_off": 5, "k_off": 6, "v_off": 7,
-        "x": 8, "x_off": 9, "w_qkv": 10, "b_qkv": 11, "w_o": 12, "b_o": 13}
+        "x": 8, "x_off": 9, "w_qkv": 10, "b_qkv": 11, "w_o": 12, "b_o": 13,
+        "pos_w": 14, "pos_b": 15, "ln1_g": 16, "ln1_b": 17, "ln2_g": 18, "ln2_b": 19,
+        "mlp_w1": 20, "mlp_b1": 21, "mlp_w2": 22, "mlp_b2": 23}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -188,4 +196,23 @@ def make_layer_inputs(w: Workload, seed_base: Optional[int] = None, batch: Optio
     base = make_inputs(w, seed_base, batch)
     out["lce_w"] = base["lce_w"]
     out["lce_b"] = base["lce_b"]
+    return out
+
+
+def make_block_inputs(w: Workload, seed_base: Optional[int] = None, batch: Optional[int] = None
+                      ) -> Dict[str, np.ndarray]:
+    """make_layer_inputs plus pos_w (C,3,3), pos_b, ln1_g, ln1_b, ln2_g, ln2_b (C),
+    mlp_w1 (3C,C), mlp_b1 (3C), mlp_w2 (C,3C), mlp_b2 (C): float32 arrays exactly
+    representable in the workload dtype."""
+    out = make_layer_inputs(w, seed_base, batch)
+    C = w.C
+    draw = lambda slot, shape, scale, shift=0.0: _store(
+        shift + _rng(w, slot, seed_base).standard_normal(shape) * scale, w.dtype)
+    out.update({
+        "pos_w": draw("pos_w", (C, 3, 3), 0.2), "pos_b": draw("pos_b", (C,), 0.05),
+        "ln1_g": draw("ln1_g", (C,), 0.1, 1.0), "ln1_b": draw("ln1_b", (C,), 0.05),
+        "ln2_g": draw("ln2_g", (C,), 0.1, 1.0), "ln2_b": draw("ln2_b", (C,), 0.05),
+        "mlp_w1": draw("mlp_w1", (3 * C, C), C ** -0.5), "mlp_b1": draw("mlp_b1", (3 * C,), 0.02),
+        "mlp_w2": draw("mlp_w2", (C, 3 * C), (3 * C) ** -0.5), "mlp_b2": draw("mlp_b2", (C,), 0.02),
+    })
     return out
