@@ -21,6 +21,9 @@ the tokens of all ranks over the slowest rank's time.
 --impl reference times the float64 CPU oracle on this host's cores (the only
 reference this method has): each step is a bounded sample of the same workload.
 
+--block times the whole BiFormer block (bra_block: pos-embed, LayerNorms, the attention
+layer, the MLP) with the block's seeded inputs, under its own metric name.
+
 --layer times the attention layer around BRA instead (bra_attention_layer: the qkv
 projection, the BRA forward, the output projection) on the same workload shape, with
 the layer's seeded inputs (x and the two projections' weights); its line carries its
@@ -48,6 +51,7 @@ from vision_transformer_sparse_b200 import synth  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "BRA fwd tokens/s and TFLOP/s at 1 B200; % of bf16 tensor/HBM roofline"
 METRIC_LAYER = "BRA attention layer fwd (qkv projection + BRA + output projection) tokens/s at 1 B200"
+METRIC_BLOCK = "BiFormer block fwd (pos-embed, LayerNorms, BRA attention layer, MLP) tokens/s at 1 B200"
 METRIC_BWD = "BRA backward (routing detached) tokens/s at 1 B200"
 
 
@@ -63,6 +67,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch each step directly")
     ap.add_argument("--layer", action="store_true",
                     help="time the whole attention layer (bra_attention_layer) instead of the BRA forward")
+    ap.add_argument("--block", action="store_true",
+                    help="time the whole BiFormer block (bra_block) instead of the BRA forward")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (bra_backward, routing detached) instead of the forward")
     ap.add_argument("--variant", default="auto", choices=["auto", "generic", "tma", "split", "pipe"],
@@ -97,7 +103,11 @@ def algorithmic(w: synth.Workload):
     # the backward: q, k, v and dout read, dq, dk, dv written in float32, the routing and
     # the LCE weight read, its float32 gradients written (per call, all its kernels)
     bwd_bytes = 4.0 * T * w.C * b + 3.0 * T * w.C * 4 + w.N * w.regions * w.topk * 4 + w.C * 25 * (b + 4) + w.C * 4
+    # the block's per-pixel kernels: pos_ln reads x and writes x1 and norm1's output; add_ln
+    # reads x1 and the attention output and writes x2 and norm2's output (mean per launch)
+    block_bytes = (3.0 * T * w.C * b + 4.0 * T * w.C * b) / 2
     return {"tokens": T, "flops": flops, "gathered_bytes": gathered, "attn_bytes": attn_unique,
+            "block_bytes": block_bytes,
             "pool_bytes": pool_bytes, "route_bytes": route_bytes, "fused_bytes": fused_bytes,
             "linear_bytes": lin_bytes, "linear_flops": lin_flops, "bwd_bytes": bwd_bytes, "elem_bytes": b}
 
@@ -143,7 +153,9 @@ KERNEL_HEADERS = {
     "route_kernel": ["route.cuh"],
     "linear_umma_kernel": ["linear.cuh"],
     "linear_f32_kernel": ["linear.cuh"],
-    "bwd_kernels": ["backward.cuh"],
+    "bwd_kernels": ["backward.cuh", "backward_tc.cuh"],
+    "block_pixel_kernels": ["block.cuh"],
+    "pad_crop_kernels": ["pad.cuh"],
 }
 
 
@@ -305,10 +317,15 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- reference arm
 
-def oracle_step(w: synth.Workload, sample: synth.Workload, layer: bool, backward: bool = False):
-    """One call of the oracle on `sample` (the BRA forward, the whole layer, or the backward
-    for the forward's routing)."""
+def oracle_step(w: synth.Workload, sample: synth.Workload, layer: bool, backward: bool = False, block: bool = False):
+    """One call of the oracle on `sample` (the BRA forward, the whole layer, the block, or the
+    backward for the forward's routing)."""
     import oracle
+    if block:
+        from oracle import block as ob
+        inp = {k: v.astype(np.float64) for k, v in synth.make_block_inputs(sample).items()}
+        prm = {k: v for k, v in inp.items() if k != "x"}
+        return lambda: ob.block_forward(inp["x"], prm, w.heads, w.S, w.topk, w.dtype)
     if backward:
         from oracle import backward as ob
         inp = {k: v.astype(np.float64) for k, v in synth.make_inputs(sample).items()}
@@ -329,7 +346,7 @@ def bench_reference(args, w: synth.Workload, rank: int):
     if rank != 0:
         return None
     sample = w.with_(N=1)
-    step = oracle_step(w, sample, args.layer, args.backward)
+    step = oracle_step(w, sample, args.layer, args.backward, args.block)
 
     for _ in range(args.warmup):
         step()
@@ -340,7 +357,8 @@ def bench_reference(args, w: synth.Workload, rank: int):
     value = sample.tokens * args.steps / dt
     cores = oracle.threads()
     line = {
-        "impl": "reference", "metric": METRIC_BWD if args.backward else (METRIC_LAYER if args.layer else METRIC),
+        "impl": "reference", "metric": METRIC_BWD if args.backward else (
+            METRIC_BLOCK if args.block else (METRIC_LAYER if args.layer else METRIC)),
         "value": value, "unit": "tokens/s", "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -356,12 +374,13 @@ def bench_reference(args, w: synth.Workload, rank: int):
     return line
 
 
-def cpu_baseline(w: synth.Workload, budget_s: float = 12.0, layer: bool = False, backward: bool = False):
+def cpu_baseline(w: synth.Workload, budget_s: float = 12.0, layer: bool = False, backward: bool = False,
+                 block: bool = False):
     """The oracle as it stands on a bounded sample: whole images (at most 8), repeated
     until about `budget_s` seconds of host time are used (at least once)."""
     import oracle
     sample = w.with_(N=max(1, min(w.N, 8)))
-    step = oracle_step(w, sample, layer, backward)
+    step = oracle_step(w, sample, layer, backward, block)
     reps, t0 = 0, time.perf_counter()
     while True:
         step()
@@ -371,7 +390,8 @@ def cpu_baseline(w: synth.Workload, budget_s: float = 12.0, layer: bool = False,
             break
     return {"value": sample.tokens * reps / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
             "sample": "%d x %s of %d images (%d tokens), %.1f s" % (reps, "backward" if backward else
-                                                                   ("layer" if layer else "forward"),
+                                                                   ("block" if block else
+                                                                    ("layer" if layer else "forward")),
                                                                    sample.N, sample.tokens, dt)}
 
 
@@ -417,8 +437,10 @@ def main():
 
     # inputs: this rank's own batch (weak scaling); seeded per rank
     seed = None if rank == 0 else 0xB1F0 + 16 * w.index + 1000 * rank
-    layer, backward = args.layer, args.backward
-    inp = synth.make_layer_inputs(w, seed_base=seed) if layer else synth.make_inputs(w, seed_base=seed)
+    block = args.block
+    layer, backward = args.layer or block, args.backward
+    inp = (synth.make_block_inputs(w, seed_base=seed) if block else
+           synth.make_layer_inputs(w, seed_base=seed) if layer else synth.make_inputs(w, seed_base=seed))
     if backward:  # dL/dout: another seeded map of the same shape, stored in the dtype
         inp["dout"] = synth.make_inputs(w, seed_base=0xB0D0 + w.index + 1000 * rank)["q"]
     base = {k: torch.from_numpy(v).to(dev).to(tdt).contiguous() for k, v in inp.items()}
@@ -454,6 +476,9 @@ def main():
         if backward:  # timed and traced: the asynchronous entry point (graph-capturable)
             bra.backward(s["q"], s["k"], s["v"], s["lce_w"], s["r_idx"], s["dout"], w.heads, w.S, stream=stream,
                          grads=s["grads"], sync=sync)
+        elif block:
+            bra.block(s["x"], s, w.heads, w.S, w.topk, out=s["out"], r_idx=s["r_idx"], r_weight=s["r_w"],
+                      stream=stream)
         elif layer:
             bra.attention_layer(s["x"], s["w_qkv"], s["b_qkv"], s["w_o"], s["b_o"], s["lce_w"], s["lce_b"],
                                 w.heads, w.S, w.topk, out=s["out"], r_idx=s["r_idx"], r_weight=s["r_w"],
@@ -622,7 +647,8 @@ def main():
     attn_s = min(traced_s, ms_step / 1e3 / max(launches_per_step, 1e-9))
     alg_bytes = {"bra_image_kernel": acc["fused_bytes"], "region_mean_kernel": acc["pool_bytes"],
                  "route_kernel": acc["route_bytes"], "linear_umma_kernel": acc["linear_bytes"],
-                 "linear_f32_kernel": acc["linear_bytes"]}.get(attn_name, acc["attn_bytes"])
+                 "linear_f32_kernel": acc["linear_bytes"],
+                 "block_pixel_kernels": acc["block_bytes"]}.get(attn_name, acc["attn_bytes"])
     if backward:  # the backward's kernels form one traced class: time per call
         traced_s = t_ms / max(traced_steps, 1) / 1e3
         attn_s = min(traced_s, ms_step / 1e3)
@@ -644,7 +670,8 @@ def main():
                          "traced_launch_us": traced_s * 1e6, "step_frac": roofline["roofline_us"] / (ms_step * 1e3),
                          "peak_source": peak_kind + (" (burst bf16)" if roofline["bound"] == "tensor" else "")})
     line = {
-        "metric": METRIC_BWD if backward else (METRIC_LAYER if layer else METRIC), "value": value,
+        "metric": METRIC_BWD if backward else (METRIC_BLOCK if block else (METRIC_LAYER if layer else METRIC)),
+        "value": value,
         "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -657,7 +684,8 @@ def main():
                    "launch": "CUDA graph per step" if graphs else "direct launches",
                    "attention_kernel": args.variant,
                    "step": "bra_backward_async (routing detached, the forward's r_idx)" if backward else
-                           ("bra_attention_layer (qkv projection, BRA, output projection)" if layer
+                           ("bra_block (pos-embed, norm1, attention layer, norm2, MLP)" if block else
+                            "bra_attention_layer (qkv projection, BRA, output projection)" if layer
                             else "bra_forward"),
                    "parallelism": "dp%d (independent images, no collective)" % world},
         "tflops": tflops,
@@ -671,7 +699,8 @@ def main():
         "e2e": {"value": tokens_all * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                 "entry": "bra_backward (synchronising) with stream copies (pinned host buffers)" if backward else
-                         ("bra_attention_layer with stream copies (pinned host buffers)" if layer
+                         ("bra_block with stream copies (pinned host buffers)" if block else
+                          "bra_attention_layer with stream copies (pinned host buffers)" if layer
                           else "bra_forward_host (pinned host buffers)")},
     }
     if backward:  # the forward's FLOP accounting does not describe this step
@@ -679,7 +708,7 @@ def main():
     if backward or layer:
         line.pop("roofline_unique")
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, layer=layer, backward=backward)
+        line["cpu_baseline"] = cpu_baseline(w, layer=layer, backward=backward, block=block)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -29,9 +29,9 @@ def test_kernel_sources_are_the_include_closure(bench):
         assert set(heads) <= got, kernel
         for name in got:  # closed under #include
             assert set(includes(name)) <= got, (kernel, name)
-        # every kernel builds on the shared helpers, except the backward's, which is
-        # self-contained so that its per-item code also compiles for the host
-        assert "common.cuh" in got or kernel == "bwd_kernels", kernel
+        # every kernel builds on the shared helpers, except the self-contained per-element
+        # ones (the block's per-pixel kernels and the padded grid's copies)
+        assert "common.cuh" in got or kernel in ("block_pixel_kernels", "pad_crop_kernels"), kernel
 
 
 def test_fp32_kernel_does_not_depend_on_the_tensor_core_kernels(bench):

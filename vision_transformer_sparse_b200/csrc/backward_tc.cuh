@@ -448,55 +448,132 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
     }
 }
 
-// ----------------------------------------------------------------------------- LCE parameters
+// ----------------------------------------------------------------------------- LCE gradients
 
-// dw[c][a][b] = sum over images and pixels of dout[n,y,x,c] V[n, y+a-2, x+b-2, c] (zero
-// outside), db[c] = sum of dout[..., c]: per (row block b, image n) a CTA writes the partial
-// sums of its kBwdLceRows rows, thread = channel (coalesced across the warp); a second
-// kernel adds the partials of each (channel, tap) in a fixed order.
-constexpr int kBwdLceRows = 4;
+// The LCE term out[y,x,c] += b[c] + sum_{a,b} w[c][a][b] V[y+a-2, x+b-2, c] (zero outside) gives
+//   dv[y,x,c]   = sum_{a,b} w[c][a][b] dout[y-a+2, x-b+2, c]      (the LCE part of dv)
+//   dw[c][a][b] = sum_{n,y,x} dout[n,y,x,c] V[n, y+a-2, x+b-2, c],  db[c] = sum dout[..., c].
+// bwd_tc_lce_kernel: tiles of kLceTH x kLceTW pixels and up to kLceGroup channel pairs; the
+// CTA stages the tile's dout and V with a 2-pixel zero border (bf16 pairs, coalesced
+// across channels), thread = (channel pair, pixel slot). Each thread writes the dv of its
+// pixels and keeps the 25 dw taps and db of its channel pair in registers over every tile
+// of its CTA; CTA (g, j) takes the tiles j, j + G, ... of channel group g, in that order.
+// The slots then meet in shared memory and the CTA writes its partial sums;
+// bwd_tc_lce_final_kernel adds the G partials of each (channel, tap) with one warp, in a
+// fixed order (lane stride, then a shuffle tree): no atomics, the same bits every call.
+constexpr int kLceTH = 4, kLceTW = 16, kLceGroup = 64, kLceThreads = 256;
 
-__global__ void __launch_bounds__(256) bwd_tc_lce_partial_kernel(const BwdTcParams p, float *part, int nb) {
-    const int b = blockIdx.x, n = blockIdx.y;
-    const int y0 = b * kBwdLceRows, y1 = min(p.H, y0 + kBwdLceRows);
-    for (int c = threadIdx.x; c < p.C; c += blockDim.x) {
-        float acc[26];
+// The staged tile, and after the last tile the per-thread partial sums (the same memory).
+__host__ __device__ inline int bwd_tc_lce_smem(int pairs_g) {
+    const int stage = 2 * (kLceTH + 4) * (kLceTW + 4) * pairs_g * 4, red = kLceThreads * 52 * 4;
+    return stage > red ? stage : red;
+}
+
+__global__ void __launch_bounds__(kLceThreads) bwd_tc_lce_kernel(const BwdTcParams p, const __nv_bfloat16 *lce_w,
+                                                                 float *part, int G) {
+    extern __shared__ __align__(16) uint32_t lce_s[];
+    const int pairs = p.C >> 1;
+    const int g = blockIdx.x / G, j0 = blockIdx.x - g * G;
+    const int cp0 = g * kLceGroup, pg = min(kLceGroup, pairs - cp0);  // channel pairs of this group
+    const int HW = (kLceTH + 4) * (kLceTW + 4);
+    uint32_t *sD = lce_s, *sV = lce_s + HW * pg;
+    float *red = reinterpret_cast<float *>(lce_s);  // [threads][52], over the staging after the tiles
+    const int slots = kLceThreads / pg;
+    const int cpl = threadIdx.x % pg, slot = threadIdx.x / pg;
+    const bool active = slot < slots;
+    const int cp = cp0 + cpl, c = 2 * cp;
+    float2 w[25];
 #pragma unroll
-        for (int t = 0; t < 26; ++t) acc[t] = 0.f;
-        for (int y = y0; y < y1; ++y)
-            for (int x = 0; x < p.W; ++x) {
-                const float d = __bfloat162float(p.dout[(((size_t)n * p.H + y) * p.W + x) * p.C + c]);
-                acc[25] += d;
+    for (int t = 0; t < 25; ++t)
+        w[t] = active ? make_float2(__bfloat162float(lce_w[c * 25 + t]), __bfloat162float(lce_w[(c + 1) * 25 + t]))
+                      : make_float2(0.f, 0.f);
+    float2 dw[25], db = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int a = 0; a < 5; ++a) {
-                    const int yy = y + a - 2;
-                    if (yy < 0 || yy >= p.H) continue;
-#pragma unroll
-                    for (int bb = 0; bb < 5; ++bb) {
-                        const int xx = x + bb - 2;
-                        if (xx < 0 || xx >= p.W) continue;
-                        acc[a * 5 + bb] =
-                            fmaf(d, __bfloat162float(p.v[(((size_t)n * p.H + yy) * p.W + xx) * p.C + c]), acc[a * 5 + bb]);
-                    }
-                }
+    for (int t = 0; t < 25; ++t) dw[t] = make_float2(0.f, 0.f);
+    const int nrb = (p.H + kLceTH - 1) / kLceTH, ncb = (p.W + kLceTW - 1) / kLceTW;
+    const int tiles = p.N * nrb * ncb;
+    const uint32_t *dout32 = reinterpret_cast<const uint32_t *>(p.dout);
+    const uint32_t *v32 = reinterpret_cast<const uint32_t *>(p.v);
+    auto bf2 = [](uint32_t u) { return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)); };
+    for (int tile = j0; tile < tiles; tile += G) {
+        const int n = tile / (nrb * ncb), rc = tile - n * nrb * ncb, rb = rc / ncb, cb = rc - rb * ncb;
+        const int y0 = rb * kLceTH, x0 = cb * kLceTW;
+        __syncthreads();  // the previous tile's staging is read
+        for (int i = threadIdx.x; i < HW * pg; i += kLceThreads) {
+            const int px = i / pg, q = i - px * pg;
+            const int hy = px / (kLceTW + 4), hx = px - hy * (kLceTW + 4);
+            const int y = y0 + hy - 2, x = x0 + hx - 2;
+            uint32_t d = 0u, vv = 0u;
+            if (y >= 0 && y < p.H && x >= 0 && x < p.W) {
+                const size_t o = (((size_t)n * p.H + y) * p.W + x) * pairs + cp0 + q;
+                d = __ldg(dout32 + o);
+                vv = __ldg(v32 + o);
             }
-        float *dst = part + (((size_t)n * nb + b) * p.C + c) * 26;
+            sD[i] = d;
+            sV[i] = vv;
+        }
+        __syncthreads();
+        if (!active) continue;
+        for (int pix = slot; pix < kLceTH * kLceTW; pix += slots) {
+            const int ly = pix / kLceTW, lx = pix - ly * kLceTW;
+            const int y = y0 + ly, x = x0 + lx;
+            if (y >= p.H || x >= p.W) continue;
+            const float2 d = bf2(sD[((ly + 2) * (kLceTW + 4) + lx + 2) * pg + cpl]);
+            db.x += d.x;
+            db.y += d.y;
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int t = 0; t < 26; ++t) dst[t] = acc[t];
+            for (int a = 0; a < 5; ++a)
+#pragma unroll
+                for (int b = 0; b < 5; ++b) {
+                    const float2 vn = bf2(sV[((ly + a) * (kLceTW + 4) + lx + b) * pg + cpl]);
+                    dw[a * 5 + b].x = fmaf(d.x, vn.x, dw[a * 5 + b].x);
+                    dw[a * 5 + b].y = fmaf(d.y, vn.y, dw[a * 5 + b].y);
+                    const float2 dn = bf2(sD[((ly + 4 - a) * (kLceTW + 4) + lx + 4 - b) * pg + cpl]);
+                    acc.x = fmaf(w[a * 5 + b].x, dn.x, acc.x);
+                    acc.y = fmaf(w[a * 5 + b].y, dn.y, acc.y);
+                }
+            *reinterpret_cast<float2 *>(p.dv + (((size_t)n * p.H + y) * p.W + x) * p.C + c) = acc;
+        }
+    }
+    // the slots of a channel pair meet in shared memory, then the CTA writes its partial
+    __syncthreads();  // every thread is done with the staged tile
+    float *mine = red + threadIdx.x * 52;
+#pragma unroll
+    for (int t = 0; t < 25; ++t) {
+        mine[2 * t] = dw[t].x;
+        mine[2 * t + 1] = dw[t].y;
+    }
+    mine[50] = db.x;
+    mine[51] = db.y;
+    __syncthreads();
+    float *dst = part + (size_t)blockIdx.x * kLceGroup * 2 * 26;  // [pairs of the group][2][26]
+    for (int i = threadIdx.x; i < pg * 52; i += kLceThreads) {
+        const int q = i / 52, e = i - q * 52;  // e: tap * 2 + channel, or 50 / 51 for db
+        float s2 = 0.f;
+        for (int sl = 0; sl < slots; ++sl) s2 += red[(sl * pg + q) * 52 + e];
+        const int ch = e & 1, tap = e >> 1;  // tap 25 = db
+        dst[(q * 2 + ch) * 26 + tap] = s2;
     }
 }
 
-__global__ void __launch_bounds__(256) bwd_tc_lce_final_kernel(const float *part, int nparts, int C, float *dw,
+// dw[c][t] (t < 25) and db[c] (t = 25): one warp per (c, t) adds the G partials of c's group.
+__global__ void __launch_bounds__(256) bwd_tc_lce_final_kernel(const float *part, int G, int C, float *dw,
                                                                 float *db) {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= C * 26) return;
-    const int c = i / 26, t = i - c * 26;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (gw >= C * 26) return;
+    const int c = gw / 26, t = gw - c * 26;
+    const int cp = c >> 1, g = cp / kLceGroup, ql = (cp - g * kLceGroup) * 2 + (c & 1);
     float s = 0.f;
-    for (int k = 0; k < nparts; ++k) s += part[((size_t)k * C + c) * 26 + t];
-    if (t < 25)
-        dw[c * 25 + t] = s;
-    else
-        db[c] = s;
+    for (int j = lane; j < G; j += 32) s += part[((size_t)(g * G + j) * kLceGroup * 2 + ql) * 26 + t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) {
+        if (t < 25)
+            dw[c * 25 + t] = s;
+        else
+            db[c] = s;
+    }
 }
 
 }  // namespace bra

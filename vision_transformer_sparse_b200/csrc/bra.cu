@@ -1495,13 +1495,19 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
     const int nw = (s.w2 + 15) / 16;
     if (nw > kBwdTcMaxWarps) return BRA_ERR_SHAPE;
     const int L = s.topk * s.w2;
-    const int nb = (s.H + kBwdLceRows - 1) / kBwdLceRows;
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc) return rc;
+    // LCE gradients: ng channel groups of up to kLceGroup pairs, G CTAs per group
+    const int pairs = s.C / 2, ng = (pairs + kLceGroup - 1) / kLceGroup;
+    const int lce_tiles = s.N * ((s.H + kLceTH - 1) / kLceTH) * ((s.W + kLceTW - 1) / kLceTW);
+    const int G = std::max(1, std::min(lce_tiles, sms / ng));  // one wave (one CTA per SM)
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
     const size_t b_off = up((size_t)s.N * (s.P + 1) * 4), b_list = up((size_t)s.N * s.P * s.topk * 4);
-    const size_t b_stats = up((size_t)s.N * s.P * s.heads * s.w2 * 8), b_part = up((size_t)s.N * nb * s.C * 26 * 4);
+    const size_t b_stats = up((size_t)s.N * s.P * s.heads * s.w2 * 8);
+    const size_t b_part = up((size_t)ng * G * kLceGroup * 2 * 26 * 4);
     unsigned char *buf = nullptr;
-    int rc = scratch_alloc(&buf, b_off + b_list + b_stats + b_part + 256, st);
-    if (rc) return rc;
+    if ((rc = scratch_alloc(&buf, b_off + b_list + b_stats + b_part + 256, st))) return rc;
     BwdTcParams p{};
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.k = static_cast<const __nv_bfloat16 *>(k);
@@ -1536,27 +1542,25 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
     p.nw = nw;
     p.scale = 1.0f / sqrtf((float)s.d);
     p.sl2 = p.scale * 1.4426950408889634f;
-    // the LCE part of dv through the SIMT kernel of the other path (one thread per element)
-    const BwdParams lp = make_bwd_params(q, k, v, dout, lce_w, r_idx, s.N, s.H, s.W, s.C, s.heads, s.S, s.topk, 1,
-                                         dq, dk, dv, dlce_w, dlce_b, p.bad);
-    int sms = 0;
-    if ((rc = sm_count(&sms)) == BRA_OK) {
+    {
         const int tr_smem = ((s.P * s.topk <= 10000 ? s.P * s.topk : 0) + s.P + 1) * 4;
         const int q_smem = bwd_tc_query_smem(nw, L, s.topk), k_smem = bwd_tc_key_smem(nw, s.w2);
-        const size_t elems = (size_t)s.N * s.H * s.W * s.C;
+        const int l_smem = bwd_tc_lce_smem(std::min(pairs, kLceGroup));
         const unsigned units = (unsigned)((size_t)s.N * s.P * s.heads);
         if ((sync && cudaMemsetAsync(p.bad, 0, sizeof(int), st) != cudaSuccess) ||
             allow_smem(bwd_tc_query_kernel, q_smem) != cudaSuccess ||
-            allow_smem(bwd_tc_key_kernel, k_smem) != cudaSuccess) {
+            allow_smem(bwd_tc_key_kernel, k_smem) != cudaSuccess ||
+            allow_smem(bwd_tc_lce_kernel, l_smem) != cudaSuccess) {
             rc = BRA_ERR_CUDA;
         } else {
             {
                 LaunchScope ls(BRA_KERNEL_BACKWARD, st);
                 bwd_tc_transpose_kernel<<<s.N, 256, tr_smem, st>>>(p);
             }
-            {
+            {  // the LCE part of dv (the key kernel adds the attention part) and the LCE partials
                 LaunchScope ls(BRA_KERNEL_BACKWARD, st);
-                bwd_lce_dv_kernel<<<(unsigned)std::min<size_t>((elems + 255) / 256, (size_t)sms * 8), 256, 0, st>>>(lp);
+                bwd_tc_lce_kernel<<<ng * G, kLceThreads, l_smem, st>>>(p, static_cast<const __nv_bfloat16 *>(lce_w),
+                                                                      part, G);
             }
             {
                 LaunchScope ls(BRA_KERNEL_BACKWARD, st);
@@ -1568,11 +1572,7 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
             }
             {
                 LaunchScope ls(BRA_KERNEL_BACKWARD, st);
-                bwd_tc_lce_partial_kernel<<<dim3(nb, s.N), std::min(256, (s.C + 31) / 32 * 32), 0, st>>>(p, part, nb);
-            }
-            {
-                LaunchScope ls(BRA_KERNEL_BACKWARD, st);
-                bwd_tc_lce_final_kernel<<<(s.C * 26 + 255) / 256, 256, 0, st>>>(part, s.N * nb, s.C, dlce_w, dlce_b);
+                bwd_tc_lce_final_kernel<<<(s.C * 26 * 32 + 255) / 256, 256, 0, st>>>(part, G, s.C, dlce_w, dlce_b);
             }
             if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
         }
