@@ -15,8 +15,8 @@
 //   bwd_tc_transpose_kernel: per image, the transposed routing: for every key region the
 //       list of (query region, slot) entries e = p * topk + a that route to it, ascending;
 //   bwd_tc_query_kernel: one CTA per (image, query region, head), a warp per 16 queries.
-//       Three passes over the keys in chunks of 32, recomputing S = Q K^T each time: the
-//       row statistics (max and sum, online), then D = sum A dA (dA = dO V^T), then
+//       Two passes over the keys in chunks of 32, recomputing S = Q K^T: the row statistics
+//       and O' = sum 2^(s - m) V (online), hence D = dO . O' / l = sum A dA; then dA = dO V^T,
 //       dS and dQ = scale dS K. Stores dq and, per query, (lse, D) for the key side;
 //   bwd_tc_key_kernel: one CTA per (image, key region, head), a warp per 16 keys. For each
 //       entry of the key region's list (in list order) it recomputes S^T = K Q^T and
@@ -203,8 +203,15 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
             for (int e = 0; e < 4; ++e)
                 s[nt][e] = ((mk >> (8 * nt + 2 * tq + (e & 1))) & 1u) ? s[nt][e] * p.sl2 : -INFINITY;
     };
-    // pass 1: row max and sum (online); this thread holds rows g (e < 2) and g + 8 (e >= 2)
+    // pass 1 (online over the chunks): row max m, row sum l and O' = sum_j 2^(s_j - m) v_j
+    // (this thread holds rows g (e < 2) and g + 8 (e >= 2)); then D = dO . O' / l, which is
+    // sum_j A dA
     float mx[2] = {-INFINITY, -INFINITY}, sm[2] = {0.f, 0.f};
+    float oa[4][4];  // O' rows g / g + 8, channels 8 ct + 2 tq (+1)
+#pragma unroll
+    for (int ct = 0; ct < 4; ++ct)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oa[ct][e] = 0.f;
     for (int kc = 0; kc < nch; ++kc) {
         float s[4][4];
         logits(kc, s);
@@ -216,21 +223,68 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
             cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
             cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
             const float mn = fmaxf(mx[h], cm);
-            if (mn == -INFINITY) continue;  // every key so far masked
-            float acc = mx[h] == -INFINITY ? 0.f : sm[h] * exp2f(mx[h] - mn);
+            // the rescale of what was summed relative to the old max (0 before any valid key)
+            const float f = mn == -INFINITY || mx[h] == -INFINITY ? 0.f : fast_exp2(mx[h] - mn);
+            float acc = sm[h] * f;
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) acc += exp2f(s[nt][2 * h] - mn) + exp2f(s[nt][2 * h + 1] - mn);
+            for (int ct = 0; ct < 4; ++ct) {
+                oa[ct][2 * h] *= f;
+                oa[ct][2 * h + 1] *= f;
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                // 2^(s - m); a masked key (-inf) or a row without a valid key yet gives 0
+                const float p0 = mn == -INFINITY ? 0.f : fast_exp2(s[nt][2 * h] - mn);
+                const float p1 = mn == -INFINITY ? 0.f : fast_exp2(s[nt][2 * h + 1] - mn);
+                s[nt][2 * h] = p0;
+                s[nt][2 * h + 1] = p1;
+                acc += p0 + p1;
+            }
             sm[h] = acc;
             mx[h] = mn;
         }
+        // O' += P V over this chunk's 32 keys (P as bf16 high + low parts)
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int nt = 2 * ks + u;
+                tc_split(s[nt][0], s[nt][1], hi[2 * u], lo[2 * u]);
+                tc_split(s[nt][2], s[nt][3], hi[2 * u + 1], lo[2 * u + 1]);
+            }
+#pragma unroll
+            for (int cp2 = 0; cp2 < 2; ++cp2) {
+                const int key = kc * 32 + 16 * ks + (lane & 7) + 8 * (mat & 1), chunk = 2 * cp2 + (mat >> 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(b0, b1, b2, b3, sV + tc_sw64(key, chunk));
+                mma_bf16_16816(oa[2 * cp2], hi, b0, b1);
+                mma_bf16_16816(oa[2 * cp2], lo, b0, b1);
+                mma_bf16_16816(oa[2 * cp2 + 1], hi, b2, b3);
+                mma_bf16_16816(oa[2 * cp2 + 1], lo, b2, b3);
+            }
+        }
     }
-    float lse[2];
+    float lse[2], D[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         float t = sm[h];
         t += __shfl_xor_sync(0xffffffffu, t, 1);
         t += __shfl_xor_sync(0xffffffffu, t, 2);
         lse[h] = t > 0.f ? mx[h] + log2f(t) : INFINITY;  // no valid key: probabilities 0
+        // dO . O' of row g + 8 h, this thread's 8 channels, then the quad
+        const int row = r0 + g + 8 * h;
+        float dd = 0.f;
+#pragma unroll
+        for (int ct = 0; ct < 4; ++ct) {
+            // channels 8 ct + 2 tq, + 1: 16-byte chunk ct of the row, bytes 4 tq .. 4 tq + 3
+            const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162 *>(sO + tc_sw64(row, ct) + 4 * tq);
+            const float2 df = __bfloat1622float2(d2);
+            dd = fmaf(df.x, oa[ct][2 * h], fmaf(df.y, oa[ct][2 * h + 1], dd));
+        }
+        dd += __shfl_xor_sync(0xffffffffu, dd, 1);
+        dd += __shfl_xor_sync(0xffffffffu, dd, 2);
+        D[h] = t > 0.f ? dd / t : 0.f;
     }
     // probabilities and dA of chunk kc
     auto probs = [&](int kc, float (&a)[4][4], float (&da)[4][4]) {
@@ -238,28 +292,10 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) a[nt][e] = exp2f(a[nt][e] - lse[e >> 1]);
+            for (int e = 0; e < 4; ++e) a[nt][e] = fast_exp2(a[nt][e] - lse[e >> 1]);
         chunk_mma(ado, sV, kc, da);
     };
-    // pass 2: D = sum_j A dA
-    float dsum[2] = {0.f, 0.f};
-    for (int kc = 0; kc < nch; ++kc) {
-        float a[4][4], da[4][4];
-        probs(kc, a, da);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dsum[e >> 1] = fmaf(a[nt][e], da[nt][e], dsum[e >> 1]);
-    }
-    float D[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        float t = dsum[h];
-        t += __shfl_xor_sync(0xffffffffu, t, 1);
-        t += __shfl_xor_sync(0xffffffffu, t, 2);
-        D[h] = t;
-    }
-    // pass 3: dS and dQ += dS K (keys as the contraction index)
+    // pass 2: dS and dQ += dS K (keys as the contraction index)
     float dqa[4][4];
 #pragma unroll
     for (int ct = 0; ct < 4; ++ct)
@@ -404,7 +440,7 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 st = (e & 1) ? st1 : st0;
-                    a[e] = exp2f(sT[nt][e] * p.sl2 - st.x);
+                    a[e] = fast_exp2(sT[nt][e] * p.sl2 - st.x);
                     ds[e] = a[e] * (dT[nt][e] - st.y);
                 }
                 // A fragments (keys x queries, k = queries): this tile's columns are k 8 nt + 2 tq
@@ -463,22 +499,27 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
 // fixed order (lane stride, then a shuffle tree): no atomics, the same bits every call.
 constexpr int kLceTH = 4, kLceTW = 16, kLceGroup = 64, kLceThreads = 256;
 
-// The staged tile, and after the last tile the per-thread partial sums (the same memory).
+// The staged tile (float32 pairs), and after the last tile the per-thread partial sums
+// (the same memory).
 __host__ __device__ inline int bwd_tc_lce_smem(int pairs_g) {
-    const int stage = 2 * (kLceTH + 4) * (kLceTW + 4) * pairs_g * 4, red = kLceThreads * 52 * 4;
+    const int stage = 2 * (kLceTH + 4) * (kLceTW + 4) * pairs_g * 8, red = kLceThreads * 52 * 4;
     return stage > red ? stage : red;
 }
 
+// PG: channel pairs of the group (16, 32, 48 or 64), a constant so that every tap's shared
+// address is the thread's base plus an immediate offset.
+template <int PG>
 __global__ void __launch_bounds__(kLceThreads) bwd_tc_lce_kernel(const BwdTcParams p, const __nv_bfloat16 *lce_w,
                                                                  float *part, int G) {
-    extern __shared__ __align__(16) uint32_t lce_s[];
+    extern __shared__ __align__(16) float2 lce_s[];
     const int pairs = p.C >> 1;
     const int g = blockIdx.x / G, j0 = blockIdx.x - g * G;
-    const int cp0 = g * kLceGroup, pg = min(kLceGroup, pairs - cp0);  // channel pairs of this group
+    const int cp0 = g * kLceGroup;
+    constexpr int pg = PG;
     const int HW = (kLceTH + 4) * (kLceTW + 4);
-    uint32_t *sD = lce_s, *sV = lce_s + HW * pg;
+    float2 *sD = lce_s, *sV = lce_s + HW * pg;
     float *red = reinterpret_cast<float *>(lce_s);  // [threads][52], over the staging after the tiles
-    const int slots = kLceThreads / pg;
+    constexpr int slots = kLceThreads / pg;
     const int cpl = threadIdx.x % pg, slot = threadIdx.x / pg;
     const bool active = slot < slots;
     const int cp = cp0 + cpl, c = 2 * cp;
@@ -492,25 +533,33 @@ __global__ void __launch_bounds__(kLceThreads) bwd_tc_lce_kernel(const BwdTcPara
     for (int t = 0; t < 25; ++t) dw[t] = make_float2(0.f, 0.f);
     const int nrb = (p.H + kLceTH - 1) / kLceTH, ncb = (p.W + kLceTW - 1) / kLceTW;
     const int tiles = p.N * nrb * ncb;
-    const uint32_t *dout32 = reinterpret_cast<const uint32_t *>(p.dout);
-    const uint32_t *v32 = reinterpret_cast<const uint32_t *>(p.v);
-    auto bf2 = [](uint32_t u) { return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)); };
+    const uint4 *dout16 = reinterpret_cast<const uint4 *>(p.dout);  // 4 channel pairs per 16 bytes
+    const uint4 *v16 = reinterpret_cast<const uint4 *>(p.v);
+    constexpr int pg4 = pg >> 2;
+    const int pairs4 = pairs >> 2;
     for (int tile = j0; tile < tiles; tile += G) {
         const int n = tile / (nrb * ncb), rc = tile - n * nrb * ncb, rb = rc / ncb, cb = rc - rb * ncb;
         const int y0 = rb * kLceTH, x0 = cb * kLceTW;
         __syncthreads();  // the previous tile's staging is read
-        for (int i = threadIdx.x; i < HW * pg; i += kLceThreads) {
-            const int px = i / pg, q = i - px * pg;
+        // staging: 16-byte loads (coalesced across the channel group), widened to float32
+        // pairs once here rather than at each of the 25 taps that read them
+        for (int i = threadIdx.x; i < HW * pg4; i += kLceThreads) {
+            const int px = i / pg4, q4 = i - px * pg4;
             const int hy = px / (kLceTW + 4), hx = px - hy * (kLceTW + 4);
             const int y = y0 + hy - 2, x = x0 + hx - 2;
-            uint32_t d = 0u, vv = 0u;
+            uint4 d = make_uint4(0u, 0u, 0u, 0u), vv = d;
             if (y >= 0 && y < p.H && x >= 0 && x < p.W) {
-                const size_t o = (((size_t)n * p.H + y) * p.W + x) * pairs + cp0 + q;
-                d = __ldg(dout32 + o);
-                vv = __ldg(v32 + o);
+                const size_t o = (((size_t)n * p.H + y) * p.W + x) * pairs4 + (cp0 >> 2) + q4;
+                d = __ldg(dout16 + o);
+                vv = __ldg(v16 + o);
             }
-            sD[i] = d;
-            sV[i] = vv;
+            float2 *dd = sD + px * pg + 4 * q4, *dv2 = sV + px * pg + 4 * q4;
+            const uint32_t du[4] = {d.x, d.y, d.z, d.w}, vu[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                dd[e] = make_float2(__uint_as_float(du[e] << 16), __uint_as_float(du[e] & 0xFFFF0000u));
+                dv2[e] = make_float2(__uint_as_float(vu[e] << 16), __uint_as_float(vu[e] & 0xFFFF0000u));
+            }
         }
         __syncthreads();
         if (!active) continue;
@@ -518,7 +567,10 @@ __global__ void __launch_bounds__(kLceThreads) bwd_tc_lce_kernel(const BwdTcPara
             const int ly = pix / kLceTW, lx = pix - ly * kLceTW;
             const int y = y0 + ly, x = x0 + lx;
             if (y >= p.H || x >= p.W) continue;
-            const float2 d = bf2(sD[((ly + 2) * (kLceTW + 4) + lx + 2) * pg + cpl]);
+            // the pixel's top-left halo neighbour; every tap is a constant offset from it
+            const float2 *vb = sV + (ly * (kLceTW + 4) + lx) * pg + cpl;
+            const float2 *db0 = sD + (ly * (kLceTW + 4) + lx) * pg + cpl;
+            const float2 d = db0[(2 * (kLceTW + 4) + 2) * pg];
             db.x += d.x;
             db.y += d.y;
             float2 acc = make_float2(0.f, 0.f);
@@ -526,12 +578,8 @@ __global__ void __launch_bounds__(kLceThreads) bwd_tc_lce_kernel(const BwdTcPara
             for (int a = 0; a < 5; ++a)
 #pragma unroll
                 for (int b = 0; b < 5; ++b) {
-                    const float2 vn = bf2(sV[((ly + a) * (kLceTW + 4) + lx + b) * pg + cpl]);
-                    dw[a * 5 + b].x = fmaf(d.x, vn.x, dw[a * 5 + b].x);
-                    dw[a * 5 + b].y = fmaf(d.y, vn.y, dw[a * 5 + b].y);
-                    const float2 dn = bf2(sD[((ly + 4 - a) * (kLceTW + 4) + lx + 4 - b) * pg + cpl]);
-                    acc.x = fmaf(w[a * 5 + b].x, dn.x, acc.x);
-                    acc.y = fmaf(w[a * 5 + b].y, dn.y, acc.y);
+                    dw[a * 5 + b] = ffma2(d, vb[(a * (kLceTW + 4) + b) * pg], dw[a * 5 + b]);
+                    acc = ffma2(w[a * 5 + b], db0[((4 - a) * (kLceTW + 4) + 4 - b) * pg], acc);
                 }
             *reinterpret_cast<float2 *>(p.dv + (((size_t)n * p.H + y) * p.W + x) * p.C + c) = acc;
         }

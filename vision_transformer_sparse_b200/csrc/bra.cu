@@ -1545,12 +1545,15 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
     {
         const int tr_smem = ((s.P * s.topk <= 10000 ? s.P * s.topk : 0) + s.P + 1) * 4;
         const int q_smem = bwd_tc_query_smem(nw, L, s.topk), k_smem = bwd_tc_key_smem(nw, s.w2);
-        const int l_smem = bwd_tc_lce_smem(std::min(pairs, kLceGroup));
+        const int pg = std::min(pairs, kLceGroup);  // C is a multiple of 32: pg in {16, 32, 48, 64}
+        const int l_smem = bwd_tc_lce_smem(pg);
+        auto lce_kern = pg == 16 ? bwd_tc_lce_kernel<16> : pg == 32 ? bwd_tc_lce_kernel<32>
+                        : pg == 48 ? bwd_tc_lce_kernel<48> : bwd_tc_lce_kernel<64>;
         const unsigned units = (unsigned)((size_t)s.N * s.P * s.heads);
         if ((sync && cudaMemsetAsync(p.bad, 0, sizeof(int), st) != cudaSuccess) ||
             allow_smem(bwd_tc_query_kernel, q_smem) != cudaSuccess ||
             allow_smem(bwd_tc_key_kernel, k_smem) != cudaSuccess ||
-            allow_smem(bwd_tc_lce_kernel, l_smem) != cudaSuccess) {
+            allow_smem(lce_kern, l_smem) != cudaSuccess) {
             rc = BRA_ERR_CUDA;
         } else {
             {
@@ -1559,8 +1562,7 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
             }
             {  // the LCE part of dv (the key kernel adds the attention part) and the LCE partials
                 LaunchScope ls(BRA_KERNEL_BACKWARD, st);
-                bwd_tc_lce_kernel<<<ng * G, kLceThreads, l_smem, st>>>(p, static_cast<const __nv_bfloat16 *>(lce_w),
-                                                                      part, G);
+                lce_kern<<<ng * G, kLceThreads, l_smem, st>>>(p, static_cast<const __nv_bfloat16 *>(lce_w), part, G);
             }
             {
                 LaunchScope ls(BRA_KERNEL_BACKWARD, st);
