@@ -328,7 +328,9 @@ const char *bra_kernel_name(int kernel_class);
  * (region means, routing, attention). The bfloat16 attention then runs, in this order of preference:
  *  - on the 5th-generation tensor cores (tcgen05: scores and probabilities in tensor
  *    memory, one CTA per SM) when d = 32, a region holds 128 or 256 tokens (H/S a
- *    multiple of 8, W/S even) and topk * (H/S) * (W/S) <= 256;
+ *    multiple of 8, W/S even) and topk * (H/S) * (W/S) <= 256; under BRA_VARIANT_SPLIT
+ *    also for regions of 64 tokens (8 x 8) with topk 2 or 4, which fill half of each
+ *    128-row tensor-core tile;
  *  - in the persistent pipeline kernel (tile boxes fetched by the tensor memory
  *    accelerator into multi-stage shared memory by a producer warp, consumed by
  *    mma.sync attention warps and LCE warps) where the shape allows it (64 or 128

@@ -104,6 +104,8 @@ SMALL = [
     (6, 16, 16, 64, 2, 16, 2, "bf16"),    # 256 regions, 6 images (8 routing rows per CTA)
     (2, 12, 12, 64, 2, 6, 12, "bf16"),    # 2x2 regions, topk 12: per-image routing, routed fused kernel
     (1, 20, 20, 64, 2, 5, 20, "bf16"),    # 4x4 regions, 25 of them, topk 20: the same, one column warp
+    (1, 32, 32, 64, 2, 4, 4, "bf16"),     # 8x8 regions, topk 4 -> 256 keys: half-filled tcgen05 tile (split)
+    (2, 16, 16, 64, 2, 2, 2, "bf16"),     # 8x8 regions, topk 2 -> 128 keys: the same, one score half
 ]
 
 
@@ -177,10 +179,21 @@ def test_attend_rejects_out_of_range_region_index(any_variant):
     torch.cuda.synchronize()
 
 
-@pytest.mark.parametrize("shape", [(2, 32, 32, 64, 2, 2, 1), (2, 16, 32, 64, 2, 2, 2)], ids=["w256k1", "w128k2"])
+@pytest.mark.parametrize("shape", [(2, 32, 32, 64, 2, 2, 1), (2, 16, 32, 64, 2, 2, 2), (2, 32, 32, 64, 2, 4, 4)],
+                         ids=["w256k1", "w128k2", "w64k4"])
 def test_tcgen05_attend_duplicates_and_bad_index(shape):
-    """128/256-token regions (the tcgen05 kernel): duplicated routed regions count
-    twice; an out-of-range index is reported (status 6) and its keys are masked."""
+    """64/128/256-token regions (the tcgen05 kernel; 64-token regions take it when it is
+    asked for): duplicated routed regions count twice; an out-of-range index is reported
+    (status 6) and its keys are masked."""
+    N, H, W, C, heads, S, topk = shape
+    prev = bra.set_kernel_variant(VARIANTS["split"])
+    try:
+        _tcgen05_attend_duplicates_and_bad_index(shape)
+    finally:
+        bra.set_kernel_variant(prev)
+
+
+def _tcgen05_attend_duplicates_and_bad_index(shape):
     N, H, W, C, heads, S, topk = shape
     w = synth.Workload("small", 77, N, H, W, C, heads, S, topk, "bf16", region_bias=0.5, lce_b_std=0.05,
                        lce_w_std=0.1)

@@ -180,7 +180,7 @@ __device__ __forceinline__ uint4 umma_tile_chunk(const unsigned char *tile, int 
 // CUDA cores with the true row max: the fallback for a row whose single-pass
 // probabilities overflowed. Returns the normalised O row and the row sum l (then 1).
 __device__ __noinline__ void umma_exact_row(const unsigned char *stage, const UmmaSmem &L, int qi, int w2, int topk,
-                                            bool v0, bool v1, float sl2, float (&o)[32], float &l) {
+                                            uint32_t vmask, float sl2, float (&o)[32], float &l) {
     float q[32];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -198,12 +198,12 @@ __device__ __noinline__ void umma_exact_row(const unsigned char *stage, const Um
     };
     float m = -INFINITY;
     for (int key = 0; key < Lk; ++key)
-        if (key < w2 ? v0 : v1) m = fmaxf(m, score(key));
+        if ((vmask >> (key / w2)) & 1u) m = fmaxf(m, score(key));
 #pragma unroll
     for (int c = 0; c < 32; ++c) o[c] = 0.f;
     l = 0.f;
     for (int key = 0; key < Lk; ++key) {
-        if (!(key < w2 ? v0 : v1)) continue;
+        if (!((vmask >> (key / w2)) & 1u)) continue;
         const float p = exp2f((score(key) - m) * sl2);
         l += p;
         float vv[32];
@@ -227,7 +227,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t bars = base + L.bars;
     const int Lk = prm.topk * prm.w2;
-    const int nT = prm.w2 >> 7;   // 128-query tiles per unit
+    // 128-query tiles per unit; a 64-token region fills the first 64 rows of one tile (the
+    // other rows are independent of them in every product and are never stored)
+    const int nT = prm.w2 >= 128 ? prm.w2 >> 7 : 1;
+    const int tile_rows = prm.w2 < 128 ? prm.w2 : 128;
     const int np = Lk >> 6;       // 64-key chunk pairs per row
     const int heads = prm.heads;
     const int h = blockIdx.x % heads;
@@ -405,9 +408,18 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
             for (int ru = ru0; ru < prm.regions; ru += stride_ru, ++k) {
                 const int s = k & 1, use = k >> 1;
                 if (!umma_wait_warp(bars + 8 * (kUbFull + s), use & 1, lim)) break;
-                const bool v0 = sIdx[s * prm.topk] >= 0;
-                const bool v1 = prm.topk > 1 ? sIdx[s * prm.topk + 1] >= 0 : true;
+                uint32_t vmask = 0;  // routed regions present in the stage
+                for (int a = 0; a < prm.topk; ++a) vmask |= (sIdx[s * prm.topk + a] >= 0 ? 1u : 0u) << a;
                 const uint32_t F = trow + 128 * (k & 1), G = trow + 128 * ((k & 1) ^ 1);
+                if (32 * sub >= tile_rows) {
+                    // a warp with no live row: no scores to read or P to store, only the
+                    // arrivals the barriers count; then it waits until the unit's O is complete
+                    // (every P barrier of the unit has finished its phase) before the next unit
+                    for (int j = 0; j < np; ++j) umma_arrive(bars + 8 * (kUbP + 4 * t + j));
+                    if (np == 4) umma_arrive(bars + 8 * (kUbGRead + t));
+                    if (!umma_wait_warp(bars + 8 * (kUbOFull + t), k & 1, lim)) break;
+                    continue;
+                }
                 if (!umma_wait_warp(bars + 8 * (kUbSFullF + t), k & 1, lim)) break;
                 tc_fence_after();
                 bool gready = np < 4, fail = false;
@@ -427,15 +439,17 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
                 // scores load while the current chunk's exponentials are computed.
                 const int nch = 2 * np;
                 auto chunk_col = [&](int c) { return c < 4 ? F + 32 * c : G + 32 * (c - 4); };
-                auto chunk_valid = [&](int c) { return (c << 5) < prm.w2 ? v0 : v1; };
+                auto chunk_valid = [&](int c) { return ((vmask >> ((c << 5) / prm.w2)) & 1u) != 0u; };
                 uint32_t ra[32], rb[32];
                 float m = -INFINITY;
-                if (v0) {
+                int cref = 0;  // the first valid chunk
+                while (cref < nch && !chunk_valid(cref)) ++cref;
+                if (cref == 0) {
                     tmem_ld32(F, ra);  // chunk 0, kept for its exponentials
                     m = max32(ra, -INFINITY);
-                } else if (np == 4 && prm.topk > 1 && v1) {  // keys 128..255: the second region
-                    if (!wait_g()) break;
-                    tmem_ld32(G, rb);
+                } else if (cref < nch) {  // read for its max only; the pass loads it again
+                    if (cref >= 4 && !wait_g()) break;
+                    tmem_ld32(chunk_col(cref), rb);
                     m = max32(rb, -INFINITY);
                 }
                 const float mneg = m == -INFINITY ? 0.f : -m * sl2;
@@ -606,45 +620,55 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
                     break;
                 }
                 tc_fence_after();
-                uint32_t o[32];
-                tmem_ld32(etm + 256 * t + 128 * (k & 1), o);
-                float l = sRsum[t * 128 + erow];
-                tc_fence_before();
-                umma_arrive(bars + 8 * (kUbOEmpty + t));  // the half may take the next scores
-                float ck[4] = {l, 0.f, 0.f, 0.f};  // NaN unless l and every O value are finite
+                const bool live = 32 * (warp & 3) < tile_rows;  // the warp's 32 rows hold queries
+                if (!live) {  // only the arrivals the barriers count (the storing warp still stores)
+                    umma_arrive(bars + 8 * (kUbOEmpty + t));
+                    if (!umma_wait_warp(bars + 8 * (kUbOTFree + t), k & 1, lim)) {
+                        fail = true;
+                        break;
+                    }
+                    umma_arrive(bars + 8 * (kUbOTReady + t));
+                } else {
+                    uint32_t o[32];
+                    tmem_ld32(etm + 256 * t + 128 * (k & 1), o);
+                    float l = sRsum[t * 128 + erow];
+                    tc_fence_before();
+                    umma_arrive(bars + 8 * (kUbOEmpty + t));  // the half may take the next scores
+                    float ck[4] = {l, 0.f, 0.f, 0.f};  // NaN unless l and every O value are finite
 #pragma unroll
-                for (int e = 0; e < 32; ++e) ck[e & 3] = fmaf(__uint_as_float(o[e]), 0.f, ck[e & 3]);
-                if (!(fabsf((ck[0] + ck[1]) + (ck[2] + ck[3])) <= 3.0e38f)) {
-                    const bool v0 = sIdx[s * prm.topk] >= 0;
-                    const bool v1 = prm.topk > 1 ? sIdx[s * prm.topk + 1] >= 0 : true;
-                    float of[32];
-                    umma_exact_row(sm + s * L.stage_bytes, L, qi, prm.w2, prm.topk, v0, v1, prm.scale_log2, of, l);
+                    for (int e = 0; e < 32; ++e) ck[e & 3] = fmaf(__uint_as_float(o[e]), 0.f, ck[e & 3]);
+                    if (!(fabsf((ck[0] + ck[1]) + (ck[2] + ck[3])) <= 3.0e38f)) {
+                        uint32_t vmask = 0;
+                        for (int a = 0; a < prm.topk; ++a) vmask |= (sIdx[s * prm.topk + a] >= 0 ? 1u : 0u) << a;
+                        float of[32];
+                        umma_exact_row(sm + s * L.stage_bytes, L, qi, prm.w2, prm.topk, vmask, prm.scale_log2, of, l);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(of[e]);
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(of[e]);
+                    }
+                    const float inv = l > 0.f ? 1.f / l : 0.f;
+                    const float4 *srow = reinterpret_cast<const float4 *>(sStage + qi * kUmmaStagePitch);
+                    uint4 ov[4];
+                    uint32_t *ow = reinterpret_cast<uint32_t *>(ov);
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 a = srow[q4];
+                        ow[2 * q4] = pack_bf16x2(fmaf(__uint_as_float(o[4 * q4]), inv, a.x),
+                                                 fmaf(__uint_as_float(o[4 * q4 + 1]), inv, a.y));
+                        ow[2 * q4 + 1] = pack_bf16x2(fmaf(__uint_as_float(o[4 * q4 + 2]), inv, a.z),
+                                                     fmaf(__uint_as_float(o[4 * q4 + 3]), inv, a.w));
+                    }
+                    // the row goes to the tile's smem image; one thread stores the whole tile
+                    if (!umma_wait_warp(bars + 8 * (kUbOTFree + t), k & 1, lim)) {
+                        fail = true;
+                        break;
+                    }
+                    unsigned char *otile = sm + L.otile + t * 8192;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<uint4 *>(otile + erow * 64 + ((q4 ^ ((erow >> 1) & 3)) << 4)) = ov[q4];
+                    fence_proxy_async();  // the rows are read by the tensor store
+                    umma_arrive(bars + 8 * (kUbOTReady + t));
                 }
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                const float4 *srow = reinterpret_cast<const float4 *>(sStage + qi * kUmmaStagePitch);
-                uint4 ov[4];
-                uint32_t *ow = reinterpret_cast<uint32_t *>(ov);
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    const float4 a = srow[q4];
-                    ow[2 * q4] = pack_bf16x2(fmaf(__uint_as_float(o[4 * q4]), inv, a.x),
-                                             fmaf(__uint_as_float(o[4 * q4 + 1]), inv, a.y));
-                    ow[2 * q4 + 1] = pack_bf16x2(fmaf(__uint_as_float(o[4 * q4 + 2]), inv, a.z),
-                                                 fmaf(__uint_as_float(o[4 * q4 + 3]), inv, a.w));
-                }
-                // the row goes to the tile's smem image; one thread stores the whole tile
-                if (!umma_wait_warp(bars + 8 * (kUbOTFree + t), k & 1, lim)) {
-                    fail = true;
-                    break;
-                }
-                unsigned char *otile = sm + L.otile + t * 8192;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(otile + erow * 64 + ((q4 ^ ((erow >> 1) & 3)) << 4)) = ov[q4];
-                fence_proxy_async();  // the rows are read by the tensor store
-                umma_arrive(bars + 8 * (kUbOTReady + t));
                 if (warp == kUmmaLceWarp0 + 4 * tw) {  // the storing thread's warp: keep its control flow uniform
                     bool stored = true;
                     if (lane == 0) {

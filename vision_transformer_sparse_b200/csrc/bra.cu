@@ -733,10 +733,13 @@ static int launch_attend_pipe(const Shape &s, const void *q, const void *k, cons
 
 // ----------------------------------------------------------------------------- tcgen05 attention
 
-// The tcgen05 kernel takes bf16 heads of 32 channels, regions of 128 or 256 tokens
-// (hr a multiple of 8, wr even) and at most 256 keys per query.
+// The tcgen05 kernel takes bf16 heads of 32 channels, regions of 64, 128 or 256 tokens
+// (hr a multiple of 8, wr even), whole 128-key score halves and at most 256 keys per
+// query. Regions of 128 or 256 tokens fill whole 128-query tiles; 64-token regions fill
+// the first half of one.
 static bool umma_shape_ok(const Shape &s) {
-    return s.dtype == BRA_BF16 && s.d == 32 && s.w2 % 128 == 0 && s.topk * s.w2 <= 256 &&
+    return s.dtype == BRA_BF16 && s.d == 32 && (s.w2 % 128 == 0 || s.w2 == 64) && (s.topk * s.w2) % 128 == 0 &&
+           s.topk * s.w2 <= 256 &&
            s.hr % kUmmaRows == 0 && s.wr % 2 == 0 && 128 % s.wr == 0 && s.hr + 4 <= 256 && s.wr + 4 <= 256;
 }
 
@@ -747,6 +750,8 @@ static int launch_attend_umma(const Shape &s, const void *q, const void *k, cons
     const int var = g_variant.load();
     if (var != BRA_VARIANT_AUTO && var != BRA_VARIANT_SPLIT) return BRA_OK;
     if (!umma_shape_ok(s) || !aligned(w, 4) || !aligned(b, 4)) return BRA_OK;
+    // 64-token regions: the half-filled tile only when asked for (BRA_VARIANT_SPLIT)
+    if (s.w2 < 128 && var != BRA_VARIANT_SPLIT) return BRA_OK;
     const UmmaSmem L = umma_smem_layout(s.topk, s.w2, s.hr, s.wr);
     if (L.total > kMaxSmem) return BRA_OK;
     UmmaParams p;
@@ -755,7 +760,7 @@ static int launch_attend_umma(const Shape &s, const void *q, const void *k, cons
         !encode_map_box(&p.tmK, k, s, 32, s.wr, s.hr, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !encode_map_box(&p.tmV, v, s, 32, s.wr, s.hr, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !encode_map_box(&p.tmH, v, s, 32, s.wr + 4, s.hr + 4, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_map_box(&p.tmO, out, s, 32, s.wr, 128 / s.wr, CU_TENSOR_MAP_SWIZZLE_64B))
+        !encode_map_box(&p.tmO, out, s, 32, s.wr, std::min(128, s.w2) / s.wr, CU_TENSOR_MAP_SWIZZLE_64B))
         return BRA_OK;
     p.lce_w = static_cast<const __nv_bfloat16 *>(w);
     p.lce_b = static_cast<const __nv_bfloat16 *>(b);
