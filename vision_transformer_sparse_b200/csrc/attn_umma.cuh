@@ -232,6 +232,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
     const int nT = prm.w2 >= 128 ? prm.w2 >> 7 : 1;
     const int tile_rows = prm.w2 < 128 ? prm.w2 : 128;
     const int np = Lk >> 6;       // 64-key chunk pairs per row
+    const int cpr = prm.w2 >> 5;  // 32-key chunks per routed region
     const int heads = prm.heads;
     const int h = blockIdx.x % heads;
     const int stride_ru = gridDim.x / heads;  // gridDim.x is a multiple of heads
@@ -408,8 +409,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
             for (int ru = ru0; ru < prm.regions; ru += stride_ru, ++k) {
                 const int s = k & 1, use = k >> 1;
                 if (!umma_wait_warp(bars + 8 * (kUbFull + s), use & 1, lim)) break;
-                uint32_t vmask = 0;  // routed regions present in the stage
-                for (int a = 0; a < prm.topk; ++a) vmask |= (sIdx[s * prm.topk + a] >= 0 ? 1u : 0u) << a;
+                uint32_t cmask = 0;  // the 32-key chunks of the routed regions present in the stage
+                for (int a = 0; a < prm.topk; ++a)
+                    if (sIdx[s * prm.topk + a] >= 0) cmask |= ((1u << cpr) - 1u) << (a * cpr);
                 const uint32_t F = trow + 128 * (k & 1), G = trow + 128 * ((k & 1) ^ 1);
                 if (32 * sub >= tile_rows) {
                     // a warp with no live row: no scores to read or P to store, only the
@@ -439,7 +441,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
                 // scores load while the current chunk's exponentials are computed.
                 const int nch = 2 * np;
                 auto chunk_col = [&](int c) { return c < 4 ? F + 32 * c : G + 32 * (c - 4); };
-                auto chunk_valid = [&](int c) { return ((vmask >> ((c << 5) / prm.w2)) & 1u) != 0u; };
+                auto chunk_valid = [&](int c) { return ((cmask >> c) & 1u) != 0u; };
                 uint32_t ra[32], rb[32];
                 float m = -INFINITY;
                 int cref = 0;  // the first valid chunk

@@ -8,27 +8,29 @@
 // Linear(3C, C), drop_path = Identity. The MLP line is read as the same pre-norm residual
 // form, x = x + mlp(norm2(x)).
 //
-//   pos_ln_kernel:  x1 = x + b + dwconv3x3(x)  (zero pad 1)   -> stored;  h = LN1(x1) -> stored
-//   add_ln_kernel:  x2 = x1 + a                                -> stored;  h = LN2(x2) -> stored
+//   pos_ln_tile_kernel:  x1 = x + b + dwconv3x3(x)  (zero pad 1)  -> stored;  h = LN1(x1) -> stored
+//   add_ln_kernel:       x2 = x1 + a                               -> stored;  h = LN2(x2) -> stored
 //
 // LayerNorm: (x - mean) / sqrt(var + 1e-6) * gamma + beta over the C channels of a pixel,
 // var the mean squared deviation (two passes over registers). Arithmetic in float32; every
 // stored value is rounded once to the storage type, and each LayerNorm reads the rounded
 // value that was stored (as a bf16 model stores its activations).
 //
-// One warp per pixel (pixels in warp-strided order, so that neighbouring warps read
-// neighbouring pixels and the 3x3 taps hit L1): lane l owns channel pairs l, l + 32, ...
-// (NP of them, C <= 64 * NP), whose weights it keeps in registers; loads and stores are
-// whole pairs (bf16x2 or float2), so a warp moves one pixel's channels contiguously.
+// A warp works on one pixel at a time: lane l owns channel pairs l, l + 32, ... (NP of
+// them, C <= 64 * NP); loads and stores are whole pairs (bf16x2 or float2), so a warp
+// moves one pixel's channels contiguously.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace bra {
 
 constexpr int kBlockThreads = 256;
+constexpr int kAddUnroll = 4;  // add_ln: pixels per warp and iteration
 
 struct BlockParams {
     const void *x;       // pos_ln: the block input; add_ln: x1
@@ -56,6 +58,10 @@ template <> struct PairIO<__nv_bfloat16> {
         const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
         static_cast<__nv_bfloat162 *>(p)[pair] = h;
     }
+    static __device__ __forceinline__ float2 lds(const void *p, size_t pair) {
+        const uint32_t u = static_cast<const uint32_t *>(p)[pair];
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+    }
 };
 template <> struct PairIO<float> {
     static __device__ __forceinline__ float2 ld(const void *p, size_t pair) {
@@ -63,6 +69,7 @@ template <> struct PairIO<float> {
     }
     static __device__ __forceinline__ float2 round(float2 v) { return v; }
     static __device__ __forceinline__ void st(void *p, size_t pair, float2 v) { static_cast<float2 *>(p)[pair] = v; }
+    static __device__ __forceinline__ float2 lds(const void *p, size_t pair) { return static_cast<const float2 *>(p)[pair]; }
 };
 
 // One parameter element (weights and per-channel vectors need only element alignment).
@@ -111,47 +118,75 @@ __device__ __forceinline__ void ln_store(const float2 (&v)[NP], const float2 (&g
     }
 }
 
+// pos_ln_tile_kernel: one CTA per (image, tile of kPosTH x kPosTW output pixels).
+// The tile's pixels with a one-pixel border, (kPosTH + 2) x (kPosTW + 2) pixels of C
+// channels, are copied into shared memory once (16-byte cp.async pieces, zero outside
+// the image), so the nine taps of every pixel read shared memory; then each warp takes
+// the tile's pixels w, w + 8, ...: lane l owns channel pairs l, l + 32, ... (NP of them),
+// whose weights it keeps in registers.
+constexpr int kPosTH = 4, kPosTW = 32;
+
+__host__ __device__ inline int pos_tile_smem_bytes(int C, int es) { return (kPosTH + 2) * (kPosTW + 2) * C * es; }
+
 template <typename T, int NP>
-__global__ void __launch_bounds__(kBlockThreads) pos_ln_kernel(const BlockParams p) {
-    const int lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kBlockThreads) pos_ln_tile_kernel(const BlockParams p, int tiles_x, int tiles_y) {
+    extern __shared__ __align__(16) unsigned char pos_s[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int pairs = p.C >> 1;
-    float2 w[NP][9], bias[NP], g[NP], bb[NP];
+    int b = blockIdx.x;
+    const int tx = b % tiles_x;
+    b /= tiles_x;
+    const int ty = b % tiles_y, n = b / tiles_y;
+    const int y0 = ty * kPosTH, x0 = tx * kPosTW;
+    constexpr int sp = kPosTW + 2;  // staged pixels per row
+    const int pix_bytes = p.C * (int)sizeof(T), chunks = pix_bytes >> 4;
+    const int total = (kPosTH + 2) * sp * chunks;
+    const unsigned char *xb = static_cast<const unsigned char *>(p.x);
+    for (int e = threadIdx.x; e < total; e += kBlockThreads) {
+        const int pix = e / chunks, ch = e - pix * chunks;
+        const int ly = pix / sp, lx = pix - ly * sp;
+        const int gy = y0 - 1 + ly, gx = x0 - 1 + lx;
+        const bool ok = gy >= 0 && gy < p.H && gx >= 0 && gx < p.W;
+        const size_t gpix = ((size_t)n * p.H + (ok ? gy : 0)) * p.W + (ok ? gx : 0);
+        cp_async16(pos_s + (size_t)e * 16, xb + gpix * pix_bytes + ch * 16, ok);
+    }
+    cp_async_commit();
+    float2 w[NP][9], bias[NP], g[NP], bb[NP];  // loaded while the copies are in flight
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
         const int cp = lane + 32 * j;
         const bool ok = cp < pairs;
         const int c = 2 * cp;
 #pragma unroll
-        for (int t = 0; t < 9; ++t)  // weights (C,3,3): channel c's tap t at c * 9 + t
+        for (int t = 0; t < 9; ++t)
             w[j][t] = ok ? make_float2(ld_elem<T>(p.pos_w, c * 9 + t), ld_elem<T>(p.pos_w, (c + 1) * 9 + t))
                          : make_float2(0.f, 0.f);
         bias[j] = ok ? ld_pair_elems<T>(p.pos_b, cp) : make_float2(0.f, 0.f);
         g[j] = ok ? ld_pair_elems<T>(p.ln_g, cp) : make_float2(0.f, 0.f);
         bb[j] = ok ? ld_pair_elems<T>(p.ln_b, cp) : make_float2(0.f, 0.f);
     }
-    const long long warps = (long long)gridDim.x * (kBlockThreads / 32);
-    for (long long pix = (long long)blockIdx.x * (kBlockThreads / 32) + (threadIdx.x >> 5); pix < p.pixels;
-         pix += warps) {
-        const int xx = (int)(pix % p.W);
-        const long long rowi = pix / p.W;
-        const int yy = (int)(rowi % p.H);
+    cp_async_wait<0>();
+    __syncthreads();
+    for (int t = warp; t < kPosTH * kPosTW; t += kBlockThreads / 32) {
+        const int py = t / kPosTW, px = t - py * kPosTW;
+        if (y0 + py >= p.H || x0 + px >= p.W) continue;  // the same for the whole warp
         float2 acc[NP];
 #pragma unroll
         for (int j = 0; j < NP; ++j) acc[j] = bias[j];
 #pragma unroll
         for (int a = 0; a < 3; ++a) {
-            const int y2 = yy + a - 1;
-            if (y2 < 0 || y2 >= p.H) continue;
+            const int y2 = y0 + py + a - 1;
+            if (y2 < 0 || y2 >= p.H) continue;  // out-of-image taps are the convolution's zero padding
 #pragma unroll
             for (int e = 0; e < 3; ++e) {
-                const int x2 = xx + e - 1;
+                const int x2 = x0 + px + e - 1;
                 if (x2 < 0 || x2 >= p.W) continue;
-                const size_t q0 = (size_t)(pix + (long long)(a - 1) * p.W + (e - 1)) * pairs;
+                const size_t q0 = (size_t)((py + a) * sp + (px + e)) * pairs;
 #pragma unroll
                 for (int j = 0; j < NP; ++j) {
                     const int cp = lane + 32 * j;
                     if (cp < pairs) {
-                        const float2 v = PairIO<T>::ld(p.x, q0 + cp);
+                        const float2 v = PairIO<T>::lds(pos_s, q0 + cp);
                         acc[j].x = fmaf(w[j][3 * a + e].x, v.x, acc[j].x);
                         acc[j].y = fmaf(w[j][3 * a + e].y, v.y, acc[j].y);
                         if (a == 1 && e == 1) {  // the residual: x itself
@@ -162,13 +197,13 @@ __global__ void __launch_bounds__(kBlockThreads) pos_ln_kernel(const BlockParams
                 }
             }
         }
-        const size_t q0 = (size_t)pix * pairs;
+        const size_t o0 = (((size_t)n * p.H + y0 + py) * p.W + x0 + px) * pairs;
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
             acc[j] = PairIO<T>::round(acc[j]);
-            if (lane + 32 * j < pairs) PairIO<T>::st(p.xo, q0 + lane + 32 * j, acc[j]);
+            if (lane + 32 * j < pairs) PairIO<T>::st(p.xo, o0 + lane + 32 * j, acc[j]);
         }
-        ln_store<T, NP>(acc, g, bb, lane, pairs, p.C, p.h, q0);
+        ln_store<T, NP>(acc, g, bb, lane, pairs, p.C, p.h, o0);
     }
 }
 
@@ -183,22 +218,39 @@ __global__ void __launch_bounds__(kBlockThreads) add_ln_kernel(const BlockParams
         g[j] = cp < pairs ? ld_pair_elems<T>(p.ln_g, cp) : make_float2(0.f, 0.f);
         bb[j] = cp < pairs ? ld_pair_elems<T>(p.ln_b, cp) : make_float2(0.f, 0.f);
     }
+    // kAddUnroll pixels per warp and iteration: all their loads are in flight together
     const long long warps = (long long)gridDim.x * (kBlockThreads / 32);
-    for (long long pix = (long long)blockIdx.x * (kBlockThreads / 32) + (threadIdx.x >> 5); pix < p.pixels;
-         pix += warps) {
-        const size_t q0 = (size_t)pix * pairs;
-        float2 v[NP];
+    for (long long pix0 = (long long)blockIdx.x * (kBlockThreads / 32) + (threadIdx.x >> 5); pix0 < p.pixels;
+         pix0 += warps * kAddUnroll) {
+        float2 x1[kAddUnroll][NP], a[kAddUnroll][NP];
 #pragma unroll
-        for (int j = 0; j < NP; ++j) {
-            const int cp = lane + 32 * j;
-            v[j] = make_float2(0.f, 0.f);
-            if (cp < pairs) {
-                const float2 x1 = PairIO<T>::ld(p.x, q0 + cp), a = PairIO<T>::ld(p.a, q0 + cp);
-                v[j] = PairIO<T>::round(make_float2(x1.x + a.x, x1.y + a.y));
-                PairIO<T>::st(p.xo, q0 + cp, v[j]);
+        for (int u = 0; u < kAddUnroll; ++u) {
+            const long long pix = pix0 + u * warps;
+            const size_t q0 = (size_t)pix * pairs;
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const int cp = lane + 32 * j;
+                x1[u][j] = a[u][j] = make_float2(0.f, 0.f);
+                if (pix < p.pixels && cp < pairs) {
+                    x1[u][j] = PairIO<T>::ld(p.x, q0 + cp);
+                    a[u][j] = PairIO<T>::ld(p.a, q0 + cp);
+                }
             }
         }
-        ln_store<T, NP>(v, g, bb, lane, pairs, p.C, p.h, q0);
+#pragma unroll
+        for (int u = 0; u < kAddUnroll; ++u) {
+            const long long pix = pix0 + u * warps;
+            if (pix >= p.pixels) break;  // the same for the whole warp
+            const size_t q0 = (size_t)pix * pairs;
+            float2 v[NP];
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const int cp = lane + 32 * j;
+                v[j] = PairIO<T>::round(make_float2(x1[u][j].x + a[u][j].x, x1[u][j].y + a[u][j].y));
+                if (cp < pairs) PairIO<T>::st(p.xo, q0 + cp, v[j]);
+            }
+            ln_store<T, NP>(v, g, bb, lane, pairs, p.C, p.h, q0);
+        }
     }
 }
 

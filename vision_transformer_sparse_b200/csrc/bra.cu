@@ -1082,14 +1082,20 @@ static int launch_block_pixels(bool pos, const BlockParams &p, cudaStream_t st) 
     const long long want = (p.pixels + kBlockThreads / 32 - 1) / (kBlockThreads / 32);
     const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(want, (long long)sms * 8));
     const int np = (p.C + 63) / 64;
+    // the positional embedding: tiles of kPosTH x kPosTW pixels staged in shared memory
+    const int tiles_x = (p.W + kPosTW - 1) / kPosTW, tiles_y = (p.H + kPosTH - 1) / kPosTH;
+    const long long tiles = p.pixels / ((long long)p.H * p.W) * tiles_x * tiles_y;
+    const int tsmem = pos_tile_smem_bytes(p.C, (int)sizeof(T));
+    if (pos && tiles > INT_MAX) return BRA_ERR_SHAPE;
     LaunchScope ls(BRA_KERNEL_BLOCK, st);
     switch (np) {
-#define BRA_BLOCK_CASE(NP)                                                                         \
-    case NP:                                                                                       \
-        if (pos)                                                                                   \
-            pos_ln_kernel<T, NP><<<grid, kBlockThreads, 0, st>>>(p);                               \
-        else                                                                                       \
-            add_ln_kernel<T, NP><<<grid, kBlockThreads, 0, st>>>(p);                               \
+#define BRA_BLOCK_CASE(NP)                                                                                    \
+    case NP:                                                                                                  \
+        if (pos) {                                                                                            \
+            if (allow_smem(pos_ln_tile_kernel<T, NP>, tsmem) != cudaSuccess) return BRA_ERR_CUDA;             \
+            pos_ln_tile_kernel<T, NP><<<(unsigned)tiles, kBlockThreads, tsmem, st>>>(p, tiles_x, tiles_y);    \
+        } else                                                                                                \
+            add_ln_kernel<T, NP><<<grid, kBlockThreads, 0, st>>>(p);                                          \
         break;
         BRA_BLOCK_CASE(1)
         BRA_BLOCK_CASE(2)
