@@ -58,7 +58,7 @@ template <> struct PairIO<__nv_bfloat16> {
         const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
         static_cast<__nv_bfloat162 *>(p)[pair] = h;
     }
-    static __device__ __forceinline__ float2 lds(const void *p, size_t pair) {
+    static __device__ __forceinline__ float2 lds(const void *p, int pair) {
         const uint32_t u = static_cast<const uint32_t *>(p)[pair];
         return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
     }
@@ -69,8 +69,37 @@ template <> struct PairIO<float> {
     }
     static __device__ __forceinline__ float2 round(float2 v) { return v; }
     static __device__ __forceinline__ void st(void *p, size_t pair, float2 v) { static_cast<float2 *>(p)[pair] = v; }
-    static __device__ __forceinline__ float2 lds(const void *p, size_t pair) { return static_cast<const float2 *>(p)[pair]; }
+    static __device__ __forceinline__ float2 lds(const void *p, int pair) { return static_cast<const float2 *>(p)[pair]; }
 };
+
+// 16 bytes as floats and back (rounded to the type).
+template <typename T> __device__ __forceinline__ void vec_unpack(uint4 u, float (&f)[16 / sizeof(T)]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = __uint_as_float(w[i]);
+    }
+}
+template <typename T> __device__ __forceinline__ uint4 vec_pack(const float (&f)[16 / sizeof(T)]) {
+    uint32_t w[4];
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = __float_as_uint(f[i]);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 // One parameter element (weights and per-channel vectors need only element alignment).
 template <typename T> __device__ __forceinline__ float ld_elem(const void *p, int i) {
@@ -167,26 +196,25 @@ __global__ void __launch_bounds__(kBlockThreads) pos_ln_tile_kernel(const BlockP
     }
     cp_async_wait<0>();
     __syncthreads();
+    // the staged border is zero outside the image, so every tap is taken: a tap on the
+    // border adds w * 0 (the convolution's zero padding)
+    const int rowstep = sp * pairs;
     for (int t = warp; t < kPosTH * kPosTW; t += kBlockThreads / 32) {
         const int py = t / kPosTW, px = t - py * kPosTW;
         if (y0 + py >= p.H || x0 + px >= p.W) continue;  // the same for the whole warp
+        const int c0 = (py * sp + px) * pairs + lane;     // pair `lane` of the tap at (-1, -1)
         float2 acc[NP];
 #pragma unroll
         for (int j = 0; j < NP; ++j) acc[j] = bias[j];
 #pragma unroll
-        for (int a = 0; a < 3; ++a) {
-            const int y2 = y0 + py + a - 1;
-            if (y2 < 0 || y2 >= p.H) continue;  // out-of-image taps are the convolution's zero padding
+        for (int a = 0; a < 3; ++a)
 #pragma unroll
             for (int e = 0; e < 3; ++e) {
-                const int x2 = x0 + px + e - 1;
-                if (x2 < 0 || x2 >= p.W) continue;
-                const size_t q0 = (size_t)((py + a) * sp + (px + e)) * pairs;
+                const int q0 = c0 + a * rowstep + e * pairs;
 #pragma unroll
-                for (int j = 0; j < NP; ++j) {
-                    const int cp = lane + 32 * j;
-                    if (cp < pairs) {
-                        const float2 v = PairIO<T>::lds(pos_s, q0 + cp);
+                for (int j = 0; j < NP; ++j)
+                    if (lane + 32 * j < pairs) {
+                        const float2 v = PairIO<T>::lds(pos_s, q0 + 32 * j);
                         acc[j].x = fmaf(w[j][3 * a + e].x, v.x, acc[j].x);
                         acc[j].y = fmaf(w[j][3 * a + e].y, v.y, acc[j].y);
                         if (a == 1 && e == 1) {  // the residual: x itself
@@ -194,9 +222,7 @@ __global__ void __launch_bounds__(kBlockThreads) pos_ln_tile_kernel(const BlockP
                             acc[j].y += v.y;
                         }
                     }
-                }
             }
-        }
         const size_t o0 = (((size_t)n * p.H + y0 + py) * p.W + x0 + px) * pairs;
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
@@ -250,6 +276,77 @@ __global__ void __launch_bounds__(kBlockThreads) add_ln_kernel(const BlockParams
                 if (cp < pairs) PairIO<T>::st(p.xo, q0 + cp, v[j]);
             }
             ln_store<T, NP>(v, g, bb, lane, pairs, p.C, p.h, q0);
+        }
+    }
+}
+
+// add_ln with 16-byte accesses, for a pixel of C channels that is a power-of-two number
+// LPP <= 32 of 16-byte chunks: lane l holds chunk l mod LPP of pixel l / LPP of the
+// warp's current group of 32 / LPP pixels, and the group's LayerNorm sums run over the
+// LPP lanes of each pixel (xor shuffles that stay inside the pixel's lanes). kAddUnroll
+// groups per warp and iteration have their loads in flight together. Same arithmetic as
+// add_ln_kernel; the sums meet in another order.
+template <typename T, int LPP>
+__global__ void __launch_bounds__(kBlockThreads) add_ln_vec_kernel(const BlockParams p) {
+    constexpr int VE = 16 / (int)sizeof(T);  // elements per chunk
+    constexpr int PPW = 32 / LPP;            // pixels per warp and group
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / LPP, ch = lane % LPP;
+    float g[VE], bb[VE];
+#pragma unroll
+    for (int e = 0; e < VE; ++e) {
+        g[e] = ld_elem<T>(p.ln_g, ch * VE + e);
+        bb[e] = ld_elem<T>(p.ln_b, ch * VE + e);
+    }
+    const uint4 *x1p = static_cast<const uint4 *>(p.x);
+    const uint4 *ap = static_cast<const uint4 *>(p.a);
+    uint4 *x2p = static_cast<uint4 *>(p.xo);
+    uint4 *hp = static_cast<uint4 *>(p.h);
+    const long long warps = (long long)gridDim.x * (kBlockThreads / 32);
+    const long long step = warps * PPW * kAddUnroll;
+    for (long long pix0 = ((long long)blockIdx.x * (kBlockThreads / 32) + (threadIdx.x >> 5)) * PPW * kAddUnroll;
+         pix0 < p.pixels; pix0 += step) {
+        uint4 xv[kAddUnroll], av[kAddUnroll];
+#pragma unroll
+        for (int u = 0; u < kAddUnroll; ++u) {
+            const long long pix = pix0 + u * PPW + sub;
+            xv[u] = av[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (pix < p.pixels) {
+                xv[u] = __ldg(x1p + pix * LPP + ch);
+                av[u] = __ldg(ap + pix * LPP + ch);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kAddUnroll; ++u) {
+            const long long pix = pix0 + u * PPW + sub;
+            float v[VE], xa[VE], aa[VE];
+            vec_unpack<T>(xv[u], xa);
+            vec_unpack<T>(av[u], aa);
+            float s1 = 0.f;
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+                v[e] = PairIO<T>::round(make_float2(xa[e] + aa[e], 0.f)).x;
+                s1 += v[e];
+            }
+#pragma unroll
+            for (int o = LPP / 2; o > 0; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+            const float mean = s1 / (float)p.C;
+            float s2 = 0.f;
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+                const float d = v[e] - mean;
+                s2 = fmaf(d, d, s2);
+            }
+#pragma unroll
+            for (int o = LPP / 2; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+            const float rstd = rsqrtf(s2 / (float)p.C + 1e-6f);
+            float hv[VE];
+#pragma unroll
+            for (int e = 0; e < VE; ++e) hv[e] = fmaf((v[e] - mean) * rstd, g[e], bb[e]);
+            if (pix < p.pixels) {
+                x2p[pix * LPP + ch] = vec_pack<T>(v);
+                hp[pix * LPP + ch] = vec_pack<T>(hv);
+            }
         }
     }
 }

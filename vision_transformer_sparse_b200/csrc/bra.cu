@@ -1087,6 +1087,23 @@ static int launch_block_pixels(bool pos, const BlockParams &p, cudaStream_t st) 
     const long long tiles = p.pixels / ((long long)p.H * p.W) * tiles_x * tiles_y;
     const int tsmem = pos_tile_smem_bytes(p.C, (int)sizeof(T));
     if (pos && tiles > INT_MAX) return BRA_ERR_SHAPE;
+    // add_ln with 16-byte accesses when a pixel is a power-of-two number (<= 32) of 16-byte chunks
+    const int lpp = p.C * (int)sizeof(T) / 16;
+    if (!pos && p.C * (int)sizeof(T) % 16 == 0 && lpp >= 1 && lpp <= 32 && (lpp & (lpp - 1)) == 0) {
+        const long long groups = (p.pixels + 32 / lpp * kAddUnroll - 1) / (32 / lpp * kAddUnroll);
+        const unsigned g2 = (unsigned)std::max<long long>(
+            1, std::min<long long>((groups + kBlockThreads / 32 - 1) / (kBlockThreads / 32), (long long)sms * 8));
+        LaunchScope ls(BRA_KERNEL_BLOCK, st);
+        switch (lpp) {
+            case 1: add_ln_vec_kernel<T, 1><<<g2, kBlockThreads, 0, st>>>(p); break;
+            case 2: add_ln_vec_kernel<T, 2><<<g2, kBlockThreads, 0, st>>>(p); break;
+            case 4: add_ln_vec_kernel<T, 4><<<g2, kBlockThreads, 0, st>>>(p); break;
+            case 8: add_ln_vec_kernel<T, 8><<<g2, kBlockThreads, 0, st>>>(p); break;
+            case 16: add_ln_vec_kernel<T, 16><<<g2, kBlockThreads, 0, st>>>(p); break;
+            default: add_ln_vec_kernel<T, 32><<<g2, kBlockThreads, 0, st>>>(p); break;
+        }
+        return cudaGetLastError() == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+    }
     LaunchScope ls(BRA_KERNEL_BLOCK, st);
     switch (np) {
 #define BRA_BLOCK_CASE(NP)                                                                                    \
