@@ -150,9 +150,10 @@ __device__ __forceinline__ void ln_store(const float2 (&v)[NP], const float2 (&g
 // pos_ln_tile_kernel: one CTA per (image, tile of kPosTH x kPosTW output pixels).
 // The tile's pixels with a one-pixel border, (kPosTH + 2) x (kPosTW + 2) pixels of C
 // channels, are copied into shared memory once (16-byte cp.async pieces, zero outside
-// the image), so the nine taps of every pixel read shared memory; then each warp takes
-// the tile's pixels w, w + 8, ...: lane l owns channel pairs l, l + 32, ... (NP of them),
-// whose weights it keeps in registers.
+// the image), so the nine taps of every pixel read shared memory (a tap on the border
+// adds w * 0: the convolution's zero padding); then each warp takes the tile's pixels
+// w, w + 8, ...: lane l owns channel pairs l, l + 32, ... (NP of them), whose weights it
+// keeps in registers.
 constexpr int kPosTH = 4, kPosTW = 32;
 
 __host__ __device__ inline int pos_tile_smem_bytes(int C, int es) { return (kPosTH + 2) * (kPosTW + 2) * C * es; }
