@@ -106,6 +106,8 @@ SMALL = [
     (1, 20, 20, 64, 2, 5, 20, "bf16"),    # 4x4 regions, 25 of them, topk 20: the same, one column warp
     (1, 32, 32, 64, 2, 4, 4, "bf16"),     # 8x8 regions, topk 4 -> 256 keys: half-filled tcgen05 tile (split)
     (2, 16, 16, 64, 2, 2, 2, "bf16"),     # 8x8 regions, topk 2 -> 128 keys: the same, one score half
+    (1, 28, 28, 192, 6, 7, 4, "bf16"),    # 6 heads (C = 192): a cluster of 6 CTAs per image
+    (2, 32, 32, 160, 5, 4, 2, "bf16"),    # 5 heads (C = 160), 8x8 regions: split path
 ]
 
 

@@ -71,6 +71,9 @@ TC_CASES = [
     (1, 12, 24, 64, 2, 3, 2),     # non-square 4x8-token regions
     (1, 32, 32, 128, 4, 4, 4),    # 64-token regions, 256 keys (the segmentation shape)
     (1, 32, 32, 64, 2, 2, 1),     # 256-token regions, 16 warps (the detection shape)
+    (1, 14, 14, 96, 3, 7, 4),     # 48 channel pairs: five LCE slots per CTA, one idle
+    (1, 20, 20, 32, 1, 5, 3),     # 16 channel pairs: four 4-pixel segments per tile row
+    (1, 14, 14, 192, 6, 7, 4),    # 96 channel pairs: two LCE groups of 48
 ]
 
 
@@ -133,4 +136,26 @@ def test_async_backward_equals_backward_and_reports_index_errors(dtype):
     bad[1, 3, 2] = -1
     bra.backward(d[0], d[1], d[2], d[3], torch.from_numpy(bad).cuda(), do, heads, S, sync=False)
     assert bra.device_status() == 6  # BRA_ERR_INDEX, then cleared
+    assert bra.device_status() == 0
+
+
+def test_backward_with_element_aligned_buffers():
+    """bf16 with 32 channels per head but q, k, v, dout one element past a 16-byte
+    boundary: the tensor-core kernels need 16-byte pieces, so the SIMT kernels run, and
+    the gradients still match the oracle."""
+    N, H, W, C, heads, S, topk = 1, 14, 14, 64, 2, 7, 3
+    q, k, v, dout, w = inputs(N, H, W, C, 777, "bf16")
+    r_idx, _ = oracle.route(q, k, heads, S, topk)
+
+    def shifted(a):  # the same bf16 values at an address 2 bytes past a 16-byte boundary
+        buf = torch.empty(a.size + 8, dtype=torch.bfloat16, device="cuda")
+        t = buf[1:1 + a.size]
+        t.copy_(dev(a, "bf16").reshape(-1))
+        return t.view(a.shape)
+
+    g = bra.backward(shifted(q), shifted(k), shifted(v), dev(w, "bf16"),
+                     torch.from_numpy(np.ascontiguousarray(r_idx, np.int32)).cuda(), shifted(dout), heads, S)
+    torch.cuda.synchronize()
+    got = {name: t.cpu().numpy() for name, t in g.items()}
+    check(got, ob.backward(q, k, v, w, np.zeros(C), heads, S, r_idx, dout))
     assert bra.device_status() == 0

@@ -13,7 +13,8 @@
 //
 // Kernels (bf16 maps, 32 channels per head):
 //   bwd_tc_transpose_kernel: per image, the transposed routing: for every key region the
-//       list of (query region, slot) entries e = p * topk + a that route to it, ascending;
+//       list of (query region, slot) entries e = p * topk + a that route to it, ascending
+//       (one warp ranks the entries 32 at a time);
 //   bwd_tc_query_kernel: one CTA per (image, query region, head), a warp per 16 queries.
 //       Two passes over the keys in chunks of 32, recomputing S = Q K^T: the row statistics
 //       and O' = sum 2^(s - m) V (online), hence D = dO . O' / l = sum A dA; then dA = dO V^T,
@@ -76,40 +77,61 @@ __device__ __forceinline__ void tc_split(float x0, float x1, uint32_t &hi, uint3
 // with r_idx[n][p][a] == pk, in ascending e. Thread pk scans the image's entries in order
 // (from shared memory when they fit), so the order does not depend on scheduling.
 __global__ void __launch_bounds__(256) bwd_tc_transpose_kernel(const BwdTcParams p) {
-    extern __shared__ int tr_s[];  // [P * topk] entries when they fit, then [P + 1] counts
+    extern __shared__ int tr_s[];  // [P] counts, then running list positions
     const int n = blockIdx.x, E = p.P * p.topk;
     const int32_t *ri = p.r_idx + (size_t)n * E;
-    const bool staged = E <= 10000;  // staged entries + counts stay within 48 KB
-    int *cnt = tr_s + (staged ? E : 0);
-    if (staged)
-        for (int e = threadIdx.x; e < E; e += blockDim.x) tr_s[e] = ri[e];
+    int *cnt = tr_s;
+    for (int k = threadIdx.x; k < p.P; k += blockDim.x) cnt[k] = 0;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         const int r = ri[e];
         if (r < 0 || r >= p.P) atomicExch(p.bad, 1);
     }
     __syncthreads();
-    for (int pk = threadIdx.x; pk < p.P; pk += blockDim.x) {
-        int c = 0;
-        for (int e = 0; e < E; ++e) c += (staged ? tr_s[e] : ri[e]) == pk;
-        cnt[pk] = c;
+    if (threadIdx.x >= 32) return;
+    // one warp, entries in order, 32 at a time: the lanes holding the same key region find
+    // each other (match_any); the group's leader adds its size to the region's count, and a
+    // lane's rank in its group is its order among the chunk's entries of that region, so
+    // every list comes out ascending in e, as a serial walk would write it
+    const int lane = threadIdx.x;
+    const unsigned below = (1u << lane) - 1u;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const int r = e < E ? ri[e] : -1;
+        const bool ok = r >= 0 && r < p.P;
+        const unsigned grp = __match_any_sync(0xffffffffu, ok ? r : -1);
+        if (ok && (grp & below) == 0u) cnt[r] += __popc(grp);
+        __syncwarp();
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        int *off = p.kv_off + (size_t)n * (p.P + 1);
-        for (int pk = 0; pk < p.P; ++pk) {
-            off[pk] = acc;
-            acc += cnt[pk];
-            cnt[pk] = off[pk];
-        }
-        off[p.P] = acc;
+    // exclusive prefix sum of the counts: lane l takes regions [l * per, (l + 1) * per)
+    const int per = (p.P + 31) / 32;
+    int local = 0;
+    for (int k = lane * per; k < p.P && k < (lane + 1) * per; ++k) local += cnt[k];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
     }
-    __syncthreads();
+    int run = incl - local;  // entries of the regions before this lane's first one
+    int *off = p.kv_off + (size_t)n * (p.P + 1);
+    for (int k = lane * per; k < p.P && k < (lane + 1) * per; ++k) {
+        const int c = cnt[k];
+        off[k] = run;
+        cnt[k] = run;
+        run += c;
+    }
+    if (lane == 31) off[p.P] = incl;
+    __syncwarp();
     int *list = p.kv_list + (size_t)n * E;
-    for (int pk = threadIdx.x; pk < p.P; pk += blockDim.x) {
-        int w = cnt[pk];
-        for (int e = 0; e < E; ++e)
-            if ((staged ? tr_s[e] : ri[e]) == pk) list[w++] = e;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const int r = e < E ? ri[e] : -1;
+        const bool ok = r >= 0 && r < p.P;
+        const unsigned grp = __match_any_sync(0xffffffffu, ok ? r : -1);
+        if (ok) list[cnt[r] + __popc(grp & below)] = e;
+        __syncwarp();
+        if (ok && (grp & below) == 0u) cnt[r] += __popc(grp);
+        __syncwarp();
     }
 }
 
@@ -489,9 +511,12 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
 // The LCE term out[y,x,c] += b[c] + sum_{a,b} w[c][a][b] V[y+a-2, x+b-2, c] (zero outside) gives
 //   dv[y,x,c]   = sum_{a,b} w[c][a][b] dout[y-a+2, x-b+2, c]      (the LCE part of dv)
 //   dw[c][a][b] = sum_{n,y,x} dout[n,y,x,c] V[n, y+a-2, x+b-2, c],  db[c] = sum dout[..., c].
-// bwd_tc_lce_kernel: tiles of kLceTH x kLceTW pixels and up to kLceGroup channel pairs; the
-// CTA stages the tile's dout and V with a 2-pixel zero border (bf16 pairs, coalesced
-// across channels), thread = (channel pair, pixel slot). Each thread writes the dv of its
+// bwd_tc_lce_kernel: tiles of kLceTH x kLceTW pixels and a group of PG <= kLceGroup channel
+// pairs (PG divides the pairs); the CTA stages the tile's dout and V with a 2-pixel zero
+// border (bf16 pairs, 16-byte cp.async pieces coalesced across channels, the next tile's in
+// flight while this one is summed), thread = (channel pair, slot), slot = a row segment of
+// the tile that the thread walks left to right with a 5 x 5 window of the staging in
+// registers (one new column of five values per pixel). Each thread writes the dv of its
 // pixels and keeps the 25 dw taps and db of its channel pair in registers over every tile
 // of its CTA; CTA (g, j) takes the tiles j, j + G, ... of channel group g, in that order.
 // The slots then meet in shared memory and the CTA writes its partial sums;
@@ -499,10 +524,10 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
 // fixed order (lane stride, then a shuffle tree): no atomics, the same bits every call.
 constexpr int kLceTH = 4, kLceTW = 16, kLceGroup = 64, kLceThreads = 256;
 
-// The staged tile (float32 pairs), and after the last tile the per-thread partial sums
-// (the same memory).
+// Two stages of the staged tile (bf16 pairs of dout and of V), and after the last tile the
+// per-thread partial sums (the same memory).
 __host__ __device__ inline int bwd_tc_lce_smem(int pairs_g) {
-    const int stage = 2 * (kLceTH + 4) * (kLceTW + 4) * pairs_g * 8, red = kLceThreads * 52 * 4;
+    const int stage = 2 * 2 * (kLceTH + 4) * (kLceTW + 4) * pairs_g * 4, red = kLceThreads * 52 * 4;
     return stage > red ? stage : red;
 }
 
@@ -511,17 +536,19 @@ __host__ __device__ inline int bwd_tc_lce_smem(int pairs_g) {
 template <int PG>
 __global__ void __launch_bounds__(kLceThreads) bwd_tc_lce_kernel(const BwdTcParams p, const __nv_bfloat16 *lce_w,
                                                                  float *part, int G) {
-    extern __shared__ __align__(16) float2 lce_s[];
+    extern __shared__ __align__(16) uint32_t lce_s[];
     const int pairs = p.C >> 1;
     const int g = blockIdx.x / G, j0 = blockIdx.x - g * G;
-    const int cp0 = g * kLceGroup;
     constexpr int pg = PG;
-    const int HW = (kLceTH + 4) * (kLceTW + 4);
-    float2 *sD = lce_s, *sV = lce_s + HW * pg;
+    const int cp0 = g * pg;  // the group's first channel pair
+    constexpr int HW = (kLceTH + 4) * (kLceTW + 4);
     float *red = reinterpret_cast<float *>(lce_s);  // [threads][52], over the staging after the tiles
     constexpr int slots = kLceThreads / pg;
+    // slot = (row of the tile, segment of that row): kParts segments of kSeg pixels per row
+    constexpr int SW = kLceTW + 4, kParts = slots / kLceTH, kSeg = kLceTW / kParts;
+    static_assert(kParts >= 1 && kLceTW % kParts == 0, "tile rows and segments must cover the slots");
     const int cpl = threadIdx.x % pg, slot = threadIdx.x / pg;
-    const bool active = slot < slots;
+    const bool active = slot < kLceTH * kParts;
     const int cp = cp0 + cpl, c = 2 * cp;
     float2 w[25];
 #pragma unroll
@@ -537,52 +564,90 @@ __global__ void __launch_bounds__(kLceThreads) bwd_tc_lce_kernel(const BwdTcPara
     const uint4 *v16 = reinterpret_cast<const uint4 *>(p.v);
     constexpr int pg4 = pg >> 2;
     const int pairs4 = pairs >> 2;
-    for (int tile = j0; tile < tiles; tile += G) {
+    // stage st: dout pairs [HW][pg] at lce_s + st * 2 * HW * pg, then V's
+    auto issue = [&](int tile, int st) {
         const int n = tile / (nrb * ncb), rc = tile - n * nrb * ncb, rb = rc / ncb, cb = rc - rb * ncb;
         const int y0 = rb * kLceTH, x0 = cb * kLceTW;
-        __syncthreads();  // the previous tile's staging is read
-        // staging: 16-byte loads (coalesced across the channel group), widened to float32
-        // pairs once here rather than at each of the 25 taps that read them
+        uint32_t *sD = lce_s + st * 2 * HW * pg, *sV = sD + HW * pg;
         for (int i = threadIdx.x; i < HW * pg4; i += kLceThreads) {
             const int px = i / pg4, q4 = i - px * pg4;
-            const int hy = px / (kLceTW + 4), hx = px - hy * (kLceTW + 4);
+            const int hy = px / SW, hx = px - hy * SW;
             const int y = y0 + hy - 2, x = x0 + hx - 2;
-            uint4 d = make_uint4(0u, 0u, 0u, 0u), vv = d;
-            if (y >= 0 && y < p.H && x >= 0 && x < p.W) {
-                const size_t o = (((size_t)n * p.H + y) * p.W + x) * pairs4 + (cp0 >> 2) + q4;
-                d = __ldg(dout16 + o);
-                vv = __ldg(v16 + o);
-            }
-            float2 *dd = sD + px * pg + 4 * q4, *dv2 = sV + px * pg + 4 * q4;
-            const uint32_t du[4] = {d.x, d.y, d.z, d.w}, vu[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                dd[e] = make_float2(__uint_as_float(du[e] << 16), __uint_as_float(du[e] & 0xFFFF0000u));
-                dv2[e] = make_float2(__uint_as_float(vu[e] << 16), __uint_as_float(vu[e] & 0xFFFF0000u));
-            }
+            const bool ok = y >= 0 && y < p.H && x >= 0 && x < p.W;  // outside: zero fill
+            const size_t o = ok ? (((size_t)n * p.H + y) * p.W + x) * pairs4 + (cp0 >> 2) + q4 : 0;
+            cp_async16(sD + px * pg + 4 * q4, dout16 + o, ok);
+            cp_async16(sV + px * pg + 4 * q4, v16 + o, ok);
         }
-        __syncthreads();
-        if (!active) continue;
-        for (int pix = slot; pix < kLceTH * kLceTW; pix += slots) {
-            const int ly = pix / kLceTW, lx = pix - ly * kLceTW;
-            const int y = y0 + ly, x = x0 + lx;
-            if (y >= p.H || x >= p.W) continue;
-            // the pixel's top-left halo neighbour; every tap is a constant offset from it
-            const float2 *vb = sV + (ly * (kLceTW + 4) + lx) * pg + cpl;
-            const float2 *db0 = sD + (ly * (kLceTW + 4) + lx) * pg + cpl;
-            const float2 d = db0[(2 * (kLceTW + 4) + 2) * pg];
-            db.x += d.x;
-            db.y += d.y;
-            float2 acc = make_float2(0.f, 0.f);
+        cp_async_commit();
+    };
+    // tiles j0, j0 + G, ...: the next tile's copies are in flight while this one is summed
+    if (j0 < tiles) issue(j0, 0);
+    int k = 0;
+    for (int tile = j0; tile < tiles; tile += G, ++k) {
+        const int st = k & 1;
+        if (tile + G < tiles) {
+            issue(tile + G, st ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();  // every thread's copies of this tile have landed
+        const int n = tile / (nrb * ncb), rc = tile - n * nrb * ncb, rb = rc / ncb, cb = rc - rb * ncb;
+        const int y0 = rb * kLceTH, x0 = cb * kLceTW;
+        // slot = (row of the tile, segment of that row); the slot walks its segment left to
+        // right with a 5 x 5 window in registers, first of V (for dw and db), then of dout
+        // (for dv): each step loads one new column of five values instead of all 25 taps.
+        // Staged (hy, hx) is pixel (y0 + hy - 2, x0 + hx - 2), so the window of pixel
+        // (ly, lx) is rows ly .. ly + 4, columns lx .. lx + 4 of the staging.
+        const int ly = slot % kLceTH, xs = (slot / kLceTH) * kSeg;
+        if (active && y0 + ly < p.H) {
+            const uint32_t *sD = lce_s + st * 2 * HW * pg, *sV = sD + HW * pg;
+            const uint32_t *vw = sV + (ly * SW + xs) * pg + cpl;             // V window origin
+            const uint32_t *dw0 = sD + (ly * SW + xs) * pg + cpl;            // dout window origin
+            const uint32_t *dc = sD + ((ly + 2) * SW + xs + 2) * pg + cpl;   // dout at the pixel
+            float2 win[5][5];
 #pragma unroll
             for (int a = 0; a < 5; ++a)
 #pragma unroll
-                for (int b = 0; b < 5; ++b) {
-                    dw[a * 5 + b] = ffma2(d, vb[(a * (kLceTW + 4) + b) * pg], dw[a * 5 + b]);
-                    acc = ffma2(w[a * 5 + b], db0[((4 - a) * (kLceTW + 4) + 4 - b) * pg], acc);
+                for (int b = 0; b < 4; ++b) win[a][b] = bf16x2_to_float2(vw[(a * SW + b) * pg]);
+#pragma unroll
+            for (int i = 0; i < kSeg; ++i) {
+#pragma unroll
+                for (int a = 0; a < 5; ++a) win[a][(i + 4) % 5] = bf16x2_to_float2(vw[(a * SW + i + 4) * pg]);
+                if (x0 + xs + i < p.W) {
+                    const float2 d = bf16x2_to_float2(dc[i * pg]);
+                    db.x += d.x;
+                    db.y += d.y;
+#pragma unroll
+                    for (int a = 0; a < 5; ++a)
+#pragma unroll
+                        for (int b = 0; b < 5; ++b) dw[a * 5 + b] = ffma2(d, win[a][(i + b) % 5], dw[a * 5 + b]);
                 }
-            *reinterpret_cast<float2 *>(p.dv + (((size_t)n * p.H + y) * p.W + x) * p.C + c) = acc;
+            }
+            // dv(y, x) = sum_{a,b} w[a][b] dout(y - a + 2, x - b + 2): dout at window (4 - a, 4 - b)
+#pragma unroll
+            for (int a = 0; a < 5; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) win[a][b] = bf16x2_to_float2(dw0[(a * SW + b) * pg]);
+            float2 *dvp = reinterpret_cast<float2 *>(p.dv + (((size_t)n * p.H + y0 + ly) * p.W + x0 + xs) * p.C + c);
+#pragma unroll
+            for (int i = 0; i < kSeg; ++i) {
+#pragma unroll
+                for (int a = 0; a < 5; ++a) win[a][(i + 4) % 5] = bf16x2_to_float2(dw0[(a * SW + i + 4) * pg]);
+                if (x0 + xs + i < p.W) {
+                    float2 acc[5];  // one chain per window row, summed at the end
+#pragma unroll
+                    for (int a = 0; a < 5; ++a) {
+                        acc[a] = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int b = 0; b < 5; ++b) acc[a] = ffma2(w[a * 5 + b], win[4 - a][(i + 4 - b) % 5], acc[a]);
+                    }
+                    dvp[(size_t)i * pairs] = make_float2(((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) + acc[4].x,
+                                                         ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y)) + acc[4].y);
+                }
+            }
         }
+        __syncthreads();  // this stage is read: the copies of tile k + 2 may overwrite it
     }
     // the slots of a channel pair meet in shared memory, then the CTA writes its partial
     __syncthreads();  // every thread is done with the staged tile
@@ -605,13 +670,14 @@ __global__ void __launch_bounds__(kLceThreads) bwd_tc_lce_kernel(const BwdTcPara
     }
 }
 
-// dw[c][t] (t < 25) and db[c] (t = 25): one warp per (c, t) adds the G partials of c's group.
-__global__ void __launch_bounds__(256) bwd_tc_lce_final_kernel(const float *part, int G, int C, float *dw,
+// dw[c][t] (t < 25) and db[c] (t = 25): one warp per (c, t) adds the G partials of c's group
+// (groups of pg channel pairs; each CTA's partials sit in a block of kLceGroup pairs).
+__global__ void __launch_bounds__(256) bwd_tc_lce_final_kernel(const float *part, int G, int C, int pg, float *dw,
                                                                 float *db) {
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (gw >= C * 26) return;
     const int c = gw / 26, t = gw - c * 26;
-    const int cp = c >> 1, g = cp / kLceGroup, ql = (cp - g * kLceGroup) * 2 + (c & 1);
+    const int cp = c >> 1, g = cp / pg, ql = (cp - g * pg) * 2 + (c & 1);
     float s = 0.f;
     for (int j = lane; j < G; j += 32) s += part[((size_t)(g * G + j) * kLceGroup * 2 + ql) * 26 + t];
 #pragma unroll

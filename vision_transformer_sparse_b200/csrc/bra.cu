@@ -1526,8 +1526,12 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
     int sms = 0;
     int rc = sm_count(&sms);
     if (rc) return rc;
-    // LCE gradients: ng channel groups of up to kLceGroup pairs, G CTAs per group
-    const int pairs = s.C / 2, ng = (pairs + kLceGroup - 1) / kLceGroup;
+    // LCE gradients: ng channel groups of pg pairs, G CTAs per group
+    // groups of pg channel pairs, pg the largest of 64, 48, 32, 16 that divides the pairs
+    // (C is a multiple of 32, so 16 always does)
+    const int pairs = s.C / 2;
+    const int pg = pairs % 64 == 0 ? 64 : pairs % 48 == 0 ? 48 : pairs % 32 == 0 ? 32 : 16;
+    const int ng = pairs / pg;
     const int lce_tiles = s.N * ((s.H + kLceTH - 1) / kLceTH) * ((s.W + kLceTW - 1) / kLceTW);
     const int G = std::max(1, std::min(lce_tiles, sms / ng));  // one wave (one CTA per SM)
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -1571,9 +1575,8 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
     p.scale = 1.0f / sqrtf((float)s.d);
     p.sl2 = p.scale * 1.4426950408889634f;
     {
-        const int tr_smem = ((s.P * s.topk <= 10000 ? s.P * s.topk : 0) + s.P + 1) * 4;
+        const int tr_smem = s.P * 4;
         const int q_smem = bwd_tc_query_smem(nw, L, s.topk), k_smem = bwd_tc_key_smem(nw, s.w2);
-        const int pg = std::min(pairs, kLceGroup);  // C is a multiple of 32: pg in {16, 32, 48, 64}
         const int l_smem = bwd_tc_lce_smem(pg);
         auto lce_kern = pg == 16 ? bwd_tc_lce_kernel<16> : pg == 32 ? bwd_tc_lce_kernel<32>
                         : pg == 48 ? bwd_tc_lce_kernel<48> : bwd_tc_lce_kernel<64>;
@@ -1602,7 +1605,7 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
             }
             {
                 LaunchScope ls(BRA_KERNEL_BACKWARD, st);
-                bwd_tc_lce_final_kernel<<<(s.C * 26 * 32 + 255) / 256, 256, 0, st>>>(part, G, s.C, dlce_w, dlce_b);
+                bwd_tc_lce_final_kernel<<<(s.C * 26 * 32 + 255) / 256, 256, 0, st>>>(part, G, s.C, pg, dlce_w, dlce_b);
             }
             if (cudaGetLastError() != cudaSuccess) rc = BRA_ERR_CUDA;
         }
@@ -1641,7 +1644,10 @@ static int backward_impl(const void *q, const void *k, const void *v, const void
         return BRA_ERR_ALIGN;
     int sms = 0;
     if ((rc = sm_count(&sms))) return rc;
-    if (dtype == BRA_BF16 && s.d == 32) return backward_tc(s, q, k, v, lce_w, r_idx, dout, dq, dk, dv, dlce_w, dlce_b, st, sync);
+    // the tensor-core kernels move 16-byte pieces of q, k, v and dout and store float2 gradients
+    const bool tc = dtype == BRA_BF16 && s.d == 32 && aligned(q, 16) && aligned(k, 16) && aligned(v, 16) &&
+                    aligned(dout, 16) && aligned(dq, 8) && aligned(dk, 8) && aligned(dv, 8);
+    if (tc) return backward_tc(s, q, k, v, lce_w, r_idx, dout, dq, dk, dv, dlce_w, dlce_b, st, sync);
     int *flag = nullptr;  // per call (read back here), or the library's device flag
     if (sync ? cudaMallocAsync(reinterpret_cast<void **>(&flag), sizeof(int), st) != cudaSuccess
              : index_flag(&flag) != BRA_OK)
