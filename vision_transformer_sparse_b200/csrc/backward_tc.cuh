@@ -63,6 +63,11 @@ __device__ __forceinline__ size_t tc_pix(const BwdTcParams &p, int n, int r, int
     return (((size_t)n * p.H + y) * p.W + x) * p.C;
 }
 
+// 8-byte global -> shared copy (asynchronous; completes with the thread's cp.async group).
+__device__ __forceinline__ void tc_cp_async8(uint32_t smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_dst), "l"(gmem_src) : "memory");
+}
+
 __device__ __forceinline__ void tc_split(float x0, float x1, uint32_t &hi, uint32_t &lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
     hi = *reinterpret_cast<const uint32_t *>(&h);
@@ -391,12 +396,12 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
         cp_async16_s(k_s + tc_sw64(row, ch), p.k + g, ok);
         cp_async16_s(v_s + tc_sw64(row, ch), p.v + g, ok);
     }
-    // the entry's queries: Q and dO rows, (lse, D) per row (padding: lse = +inf, D = 0)
-    auto load_entry = [&](int idx, int s) {
+    // the entry's queries (query region pr): Q and dO rows, (lse, D) per row, all as
+    // asynchronous copies (padding rows: lse = +inf, D = 0, written directly)
+    auto load_entry = [&](int pr, int s) {
         unsigned char *st = stage0 + s * stage_bytes;
         const uint32_t sq = smem_u32(st), so = sq + Rp * 64;
         float2 *sst = reinterpret_cast<float2 *>(st + 2 * Rp * 64);
-        const int pr = list[idx] / p.topk;
         for (int i = tid; i < Rp * 4; i += nthr) {
             const int row = i >> 2, ch = i & 3;
             const bool ok = row < p.w2;
@@ -404,12 +409,18 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
             cp_async16_s(sq + tc_sw64(row, ch), p.q + g, ok);
             cp_async16_s(so + tc_sw64(row, ch), p.dout + g, ok);
         }
-        for (int row = tid; row < Rp; row += nthr)
-            sst[row] = row < p.w2 ? *reinterpret_cast<const float2 *>(
-                                        p.stats + ((((size_t)n * p.P + pr) * p.heads + m) * p.w2 + row) * 2)
-                                  : make_float2(INFINITY, 0.f);
+        for (int row = tid; row < Rp; row += nthr) {
+            if (row < p.w2)
+                tc_cp_async8(smem_u32(sst + row), p.stats + ((((size_t)n * p.P + pr) * p.heads + m) * p.w2 + row) * 2);
+            else
+                sst[row] = make_float2(INFINITY, 0.f);
+        }
     };
-    if (cnt > 0) load_entry(0, 0);
+    // the query region of entry idx + 1 is read one entry ahead, so that its load overlaps
+    // the current entry's work instead of stalling the next copies
+    int pr_next = cnt > 0 ? list[0] / p.topk : 0;
+    if (cnt > 0) load_entry(pr_next, 0);
+    pr_next = cnt > 1 ? list[1] / p.topk : 0;
     cp_async_commit();
 
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3, mat = lane >> 3;
@@ -421,7 +432,8 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
         for (int e = 0; e < 4; ++e) dka[ct][e] = dva[ct][e] = 0.f;
     uint32_t ak[2][4], av[2][4];
     for (int idx = 0; idx < cnt; ++idx) {
-        if (idx + 1 < cnt) load_entry(idx + 1, (idx + 1) & 1);  // the other stage is free
+        if (idx + 1 < cnt) load_entry(pr_next, (idx + 1) & 1);  // the other stage is free
+        const int pr_after = idx + 2 < cnt ? list[idx + 2] / p.topk : 0;
         cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();
@@ -433,6 +445,7 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
                 ldsm_x4(av[kk][0], av[kk][1], av[kk][2], av[kk][3], sV + tc_sw64(row, chunk));
             }
         }
+        pr_next = pr_after;
         const unsigned char *sQ = stage0 + (idx & 1) * stage_bytes, *sO = sQ + Rp * 64;
         const float2 *sst = reinterpret_cast<const float2 *>(sQ + 2 * Rp * 64);
         for (int qc = 0; qc < Rp / 16; ++qc) {
