@@ -51,6 +51,7 @@ struct BwdTcParams {
     int *bad;                               // set to 1 when an r_idx entry is out of range
     int N, H, W, C, heads, S, topk, P, hr, wr, w2, L, nw;
     float scale, sl2;                       // scale and scale * log2(e)
+    FastDiv div_S, div_wr, div_w2, div_topk, div_heads, div_P;  // the index arithmetic's divisors
 };
 
 __device__ __forceinline__ uint32_t tc_sw64(int row, int chunk) {
@@ -59,7 +60,9 @@ __device__ __forceinline__ uint32_t tc_sw64(int row, int chunk) {
 
 // Element offset of channel 0 of token t of region r of image n.
 __device__ __forceinline__ size_t tc_pix(const BwdTcParams &p, int n, int r, int t) {
-    const int y = (r / p.S) * p.hr + t / p.wr, x = (r % p.S) * p.wr + t % p.wr;
+    uint32_t ri, ti;
+    const int ry = (int)p.div_S.divmod((uint32_t)r, ri), ty = (int)p.div_wr.divmod((uint32_t)t, ti);
+    const int y = ry * p.hr + ty, x = (int)ri * p.wr + (int)ti;
     return (((size_t)n * p.H + y) * p.W + x) * p.C;
 }
 
@@ -152,7 +155,9 @@ __host__ __device__ inline int bwd_tc_query_smem(int nw, int L, int topk) {
 __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const BwdTcParams p) {
     extern __shared__ __align__(128) unsigned char tc_q_s[];
     const int unit = blockIdx.x;
-    const int m = unit % p.heads, npr = unit / p.heads, pr = npr % p.P, n = npr / p.P;
+    uint32_t m_, pr_;
+    const int npr = (int)p.div_heads.divmod((uint32_t)unit, m_), n = (int)p.div_P.divmod((uint32_t)npr, pr_);
+    const int m = (int)m_, pr = (int)pr_;
     const int Rp = p.nw * 16, Lp = (p.L + 31) & ~31, nch = Lp / 32;
     unsigned char *sQ = tc_q_s, *sO = sQ + Rp * 64, *sK = sO + Rp * 64, *sV = sK + Lp * 64;
     int *sRoute = reinterpret_cast<int *>(sV + Lp * 64);
@@ -169,7 +174,7 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
         uint32_t mk = 0;
         for (int b = 0; b < 32; ++b) {
             const int j = w * 32 + b;
-            if (j < p.L && sRoute[j / p.w2] >= 0) mk |= 1u << b;
+            if (j < p.L && sRoute[p.div_w2.div((uint32_t)j)] >= 0) mk |= 1u << b;
         }
         sMask[w] = mk;
     }
@@ -183,7 +188,7 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
     }
     for (int i = tid; i < Lp * 4; i += nthr) {
         const int j = i >> 2, ch = i & 3;
-        const int a = j / p.w2, t = j - a * p.w2;
+        const int a = (int)p.div_w2.div((uint32_t)j), t = j - a * p.w2;
         const int r = j < p.L ? sRoute[a] : -1;
         const bool ok = r >= 0;
         const size_t g = ok ? tc_pix(p, n, r, t) + c0 + 8 * ch : 0;
@@ -379,7 +384,9 @@ __host__ __device__ inline int bwd_tc_key_smem(int nw, int w2) {
 __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const BwdTcParams p) {
     extern __shared__ __align__(128) unsigned char tc_k_s[];
     const int unit = blockIdx.x;
-    const int m = unit % p.heads, npk = unit / p.heads, pk = npk % p.P, n = npk / p.P;
+    uint32_t m_, pk_;
+    const int npk = (int)p.div_heads.divmod((uint32_t)unit, m_), n = (int)p.div_P.divmod((uint32_t)npk, pk_);
+    const int m = (int)m_, pk = (int)pk_;
     const int Kp = p.nw * 16, Rp = (p.w2 + 15) & ~15;
     unsigned char *sK = tc_k_s, *sV = sK + Kp * 64, *stage0 = sV + Kp * 64;
     const int stage_bytes = 2 * Rp * 64 + Rp * 8;
@@ -418,9 +425,9 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
     };
     // the query region of entry idx + 1 is read one entry ahead, so that its load overlaps
     // the current entry's work instead of stalling the next copies
-    int pr_next = cnt > 0 ? list[0] / p.topk : 0;
+    int pr_next = cnt > 0 ? (int)p.div_topk.div((uint32_t)list[0]) : 0;
     if (cnt > 0) load_entry(pr_next, 0);
-    pr_next = cnt > 1 ? list[1] / p.topk : 0;
+    pr_next = cnt > 1 ? (int)p.div_topk.div((uint32_t)list[1]) : 0;
     cp_async_commit();
 
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3, mat = lane >> 3;
@@ -433,7 +440,7 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
     uint32_t ak[2][4], av[2][4];
     for (int idx = 0; idx < cnt; ++idx) {
         if (idx + 1 < cnt) load_entry(pr_next, (idx + 1) & 1);  // the other stage is free
-        const int pr_after = idx + 2 < cnt ? list[idx + 2] / p.topk : 0;
+        const int pr_after = idx + 2 < cnt ? (int)p.div_topk.div((uint32_t)list[idx + 2]) : 0;
         cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();

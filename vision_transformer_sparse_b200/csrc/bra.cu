@@ -1574,6 +1574,12 @@ static int backward_tc(const Shape &s, const void *q, const void *k, const void 
     p.nw = nw;
     p.scale = 1.0f / sqrtf((float)s.d);
     p.sl2 = p.scale * 1.4426950408889634f;
+    p.div_S = FastDiv((uint32_t)s.S);
+    p.div_wr = FastDiv((uint32_t)s.wr);
+    p.div_w2 = FastDiv((uint32_t)s.w2);
+    p.div_topk = FastDiv((uint32_t)s.topk);
+    p.div_heads = FastDiv((uint32_t)s.heads);
+    p.div_P = FastDiv((uint32_t)s.P);
     {
         const int tr_smem = s.P * 4;
         const int q_smem = bwd_tc_query_smem(nw, L, s.topk), k_smem = bwd_tc_key_smem(nw, s.w2);
