@@ -318,7 +318,7 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
             if (big)
                 region_mean_big_kernel<__nv_bfloat16><<<s.N * s.P, kPoolThreads, 0, st>>>(
                     static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled,
-                    s.H, s.W, s.C, s.S);
+                    s.H, s.W, s.C, s.S, FastDiv((uint32_t)s.wr));
             else
                 region_mean_kernel<__nv_bfloat16><<<blocks, kPoolThreads, 0, st>>>(
                     static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), ws, ws + pooled,
@@ -326,7 +326,8 @@ static int launch_route_into(const Shape &s, const void *q, const void *k, int32
         } else {
             if (big)
                 region_mean_big_kernel<float><<<s.N * s.P, kPoolThreads, 0, st>>>(
-                    static_cast<const float *>(q), static_cast<const float *>(k), ws, ws + pooled, s.H, s.W, s.C, s.S);
+                    static_cast<const float *>(q), static_cast<const float *>(k), ws, ws + pooled, s.H, s.W, s.C, s.S,
+                    FastDiv((uint32_t)s.wr));
             else
                 region_mean_kernel<float><<<blocks, kPoolThreads, 0, st>>>(static_cast<const float *>(q),
                                                                           static_cast<const float *>(k), ws,

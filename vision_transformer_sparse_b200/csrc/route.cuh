@@ -92,7 +92,7 @@ region_mean_kernel(const T *__restrict__ q, const T *__restrict__ k, float *__re
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads, 4)
 region_mean_big_kernel(const T *__restrict__ q, const T *__restrict__ k, float *__restrict__ q_r,
-                       float *__restrict__ k_r, int H, int W, int C, int S) {
+                       float *__restrict__ k_r, int H, int W, int C, int S, FastDiv div_wr) {
     constexpr int V = Elem<T>::kVec;
     __shared__ float red[2][kPoolThreads * V];  // [tensor][slots][C]
     const int P = S * S, np = blockIdx.x;
@@ -113,7 +113,8 @@ region_mean_big_kernel(const T *__restrict__ q, const T *__restrict__ k, float *
                 const int t = t0 + b * slots;
                 bq[b] = bk[b] = make_uint4(0u, 0u, 0u, 0u);
                 if (t < w2) {
-                    const int th = t / wr, tw = t - th * wr;
+                    uint32_t twu;
+                    const int th = (int)div_wr.divmod((uint32_t)t, twu), tw = (int)twu;
                     const size_t off = org + ((size_t)th * W + tw) * C;
                     bq[b] = __ldg(reinterpret_cast<const uint4 *>(q + off));
                     bk[b] = __ldg(reinterpret_cast<const uint4 *>(k + off));
