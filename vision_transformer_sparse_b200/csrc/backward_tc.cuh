@@ -235,126 +235,197 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
             for (int e = 0; e < 4; ++e)
                 s[nt][e] = ((mk >> (8 * nt + 2 * tq + (e & 1))) & 1u) ? s[nt][e] * p.sl2 : -INFINITY;
     };
-    // pass 1 (online over the chunks): row max m, row sum l and O' = sum_j 2^(s_j - m) v_j
-    // (this thread holds rows g (e < 2) and g + 8 (e >= 2)); then D = dO . O' / l, which is
-    // sum_j A dA
-    float mx[2] = {-INFINITY, -INFINITY}, sm[2] = {0.f, 0.f};
-    float oa[4][4];  // O' rows g / g + 8, channels 8 ct + 2 tq (+1)
-#pragma unroll
-    for (int ct = 0; ct < 4; ++ct)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) oa[ct][e] = 0.f;
-    for (int kc = 0; kc < nch; ++kc) {
-        float s[4][4];
-        logits(kc, s);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float cm = -INFINITY;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) cm = fmaxf(cm, fmaxf(s[nt][2 * h], s[nt][2 * h + 1]));
-            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
-            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
-            const float mn = fmaxf(mx[h], cm);
-            // the rescale of what was summed relative to the old max (0 before any valid key)
-            const float f = mn == -INFINITY || mx[h] == -INFINITY ? 0.f : fast_exp2(mx[h] - mn);
-            float acc = sm[h] * f;
-#pragma unroll
-            for (int ct = 0; ct < 4; ++ct) {
-                oa[ct][2 * h] *= f;
-                oa[ct][2 * h + 1] *= f;
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                // 2^(s - m); a masked key (-inf) or a row without a valid key yet gives 0
-                const float p0 = mn == -INFINITY ? 0.f : fast_exp2(s[nt][2 * h] - mn);
-                const float p1 = mn == -INFINITY ? 0.f : fast_exp2(s[nt][2 * h + 1] - mn);
-                s[nt][2 * h] = p0;
-                s[nt][2 * h + 1] = p1;
-                acc += p0 + p1;
-            }
-            sm[h] = acc;
-            mx[h] = mn;
-        }
-        // O' += P V over this chunk's 32 keys (P as bf16 high + low parts)
+    // dQ += dS K over chunk kc (keys as the contraction index), dS = A (dA - D)
+    auto dq_chunk = [&](int kc, const float (&a)[4][4], const float (&da)[4][4], const float (&Dr)[2],
+                        float (&dq)[4][4]) {
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int nt = 2 * ks + u;
-                tc_split(s[nt][0], s[nt][1], hi[2 * u], lo[2 * u]);
-                tc_split(s[nt][2], s[nt][3], hi[2 * u + 1], lo[2 * u + 1]);
-            }
-#pragma unroll
-            for (int cp2 = 0; cp2 < 2; ++cp2) {
-                const int key = kc * 32 + 16 * ks + (lane & 7) + 8 * (mat & 1), chunk = 2 * cp2 + (mat >> 1);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(b0, b1, b2, b3, sV + tc_sw64(key, chunk));
-                mma_bf16_16816(oa[2 * cp2], hi, b0, b1);
-                mma_bf16_16816(oa[2 * cp2], lo, b0, b1);
-                mma_bf16_16816(oa[2 * cp2 + 1], hi, b2, b3);
-                mma_bf16_16816(oa[2 * cp2 + 1], lo, b2, b3);
-            }
-        }
-    }
-    float lse[2], D[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        float t = sm[h];
-        t += __shfl_xor_sync(0xffffffffu, t, 1);
-        t += __shfl_xor_sync(0xffffffffu, t, 2);
-        lse[h] = t > 0.f ? mx[h] + log2f(t) : INFINITY;  // no valid key: probabilities 0
-        // dO . O' of row g + 8 h, this thread's 8 channels, then the quad
-        const int row = r0 + g + 8 * h;
-        float dd = 0.f;
-#pragma unroll
-        for (int ct = 0; ct < 4; ++ct) {
-            // channels 8 ct + 2 tq, + 1: 16-byte chunk ct of the row, bytes 4 tq .. 4 tq + 3
-            const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162 *>(sO + tc_sw64(row, ct) + 4 * tq);
-            const float2 df = __bfloat1622float2(d2);
-            dd = fmaf(df.x, oa[ct][2 * h], fmaf(df.y, oa[ct][2 * h + 1], dd));
-        }
-        dd += __shfl_xor_sync(0xffffffffu, dd, 1);
-        dd += __shfl_xor_sync(0xffffffffu, dd, 2);
-        D[h] = t > 0.f ? dd / t : 0.f;
-    }
-    // probabilities and dA of chunk kc
-    auto probs = [&](int kc, float (&a)[4][4], float (&da)[4][4]) {
-        logits(kc, a);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) a[nt][e] = fast_exp2(a[nt][e] - lse[e >> 1]);
-        chunk_mma(ado, sV, kc, da);
-    };
-    // pass 2: dS and dQ += dS K (keys as the contraction index)
-    float dqa[4][4];
-#pragma unroll
-    for (int ct = 0; ct < 4; ++ct)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dqa[ct][e] = 0.f;
-    for (int kc = 0; kc < nch; ++kc) {
-        float a[4][4], da[4][4];
-        probs(kc, a, da);
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int nt = 2 * ks + u;
-                tc_split(a[nt][0] * (da[nt][0] - D[0]), a[nt][1] * (da[nt][1] - D[0]), hi[2 * u], lo[2 * u]);
-                tc_split(a[nt][2] * (da[nt][2] - D[1]), a[nt][3] * (da[nt][3] - D[1]), hi[2 * u + 1], lo[2 * u + 1]);
+                tc_split(a[nt][0] * (da[nt][0] - Dr[0]), a[nt][1] * (da[nt][1] - Dr[0]), hi[2 * u], lo[2 * u]);
+                tc_split(a[nt][2] * (da[nt][2] - Dr[1]), a[nt][3] * (da[nt][3] - Dr[1]), hi[2 * u + 1], lo[2 * u + 1]);
             }
 #pragma unroll
             for (int cp2 = 0; cp2 < 2; ++cp2) {
                 const int key = kc * 32 + 16 * ks + (lane & 7) + 8 * (mat & 1), chunk = 2 * cp2 + (mat >> 1);
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_t(b0, b1, b2, b3, sK + tc_sw64(key, chunk));
-                mma_bf16_16816(dqa[2 * cp2], hi, b0, b1);
-                mma_bf16_16816(dqa[2 * cp2], lo, b0, b1);
-                mma_bf16_16816(dqa[2 * cp2 + 1], hi, b2, b3);
-                mma_bf16_16816(dqa[2 * cp2 + 1], lo, b2, b3);
+                mma_bf16_16816(dq[2 * cp2], hi, b0, b1);
+                mma_bf16_16816(dq[2 * cp2], lo, b0, b1);
+                mma_bf16_16816(dq[2 * cp2 + 1], hi, b2, b3);
+                mma_bf16_16816(dq[2 * cp2 + 1], lo, b2, b3);
             }
+        }
+    };
+    float lse[2], D[2], dqa[4][4];
+#pragma unroll
+    for (int ct = 0; ct < 4; ++ct)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dqa[ct][e] = 0.f;
+    if (nch <= 2) {
+        // at most 64 keys per query: the logits and dA of both chunks stay in registers, the
+        // exponentials are taken once relative to the exact row maximum, and D = sum_j A dA
+        // is summed from them directly (no O' product)
+        float sc[2][4][4], da[2][4][4];
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc) {
+            if (kc >= nch) break;
+            logits(kc, sc[kc]);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) mx[h] = fmaxf(mx[h], fmaxf(sc[kc][nt][2 * h], sc[kc][nt][2 * h + 1]));
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+        }
+        float sm[2] = {0.f, 0.f};
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc) {
+            if (kc >= nch) break;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float mr = mx[e >> 1];
+                    const float pe = mr == -INFINITY ? 0.f : fast_exp2(sc[kc][nt][e] - mr);
+                    sc[kc][nt][e] = pe;
+                    sm[e >> 1] += pe;
+                }
+        }
+        float inv[2], dd[2] = {0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            sm[h] += __shfl_xor_sync(0xffffffffu, sm[h], 1);
+            sm[h] += __shfl_xor_sync(0xffffffffu, sm[h], 2);
+            lse[h] = sm[h] > 0.f ? mx[h] + log2f(sm[h]) : INFINITY;  // no valid key: probabilities 0
+            inv[h] = sm[h] > 0.f ? 1.0f / sm[h] : 0.f;
+        }
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc) {
+            if (kc >= nch) break;
+            chunk_mma(ado, sV, kc, da[kc]);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    sc[kc][nt][e] *= inv[e >> 1];  // A
+                    dd[e >> 1] = fmaf(sc[kc][nt][e], da[kc][nt][e], dd[e >> 1]);
+                }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            dd[h] += __shfl_xor_sync(0xffffffffu, dd[h], 1);
+            dd[h] += __shfl_xor_sync(0xffffffffu, dd[h], 2);
+            D[h] = dd[h];
+        }
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc) {
+            if (kc >= nch) break;
+            dq_chunk(kc, sc[kc], da[kc], D, dqa);
+        }
+    } else {
+        // pass 1 (online over the chunks): row max m, row sum l and O' = sum_j 2^(s_j - m) v_j
+        // (this thread holds rows g (e < 2) and g + 8 (e >= 2)); then D = dO . O' / l, which is
+        // sum_j A dA
+        float mx[2] = {-INFINITY, -INFINITY}, sm[2] = {0.f, 0.f};
+        float oa[4][4];  // O' rows g / g + 8, channels 8 ct + 2 tq (+1)
+#pragma unroll
+        for (int ct = 0; ct < 4; ++ct)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) oa[ct][e] = 0.f;
+        for (int kc = 0; kc < nch; ++kc) {
+            float s[4][4];
+            logits(kc, s);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float cm = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) cm = fmaxf(cm, fmaxf(s[nt][2 * h], s[nt][2 * h + 1]));
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+                const float mn = fmaxf(mx[h], cm);
+                // the rescale of what was summed relative to the old max (0 before any valid key)
+                const float f = mn == -INFINITY || mx[h] == -INFINITY ? 0.f : fast_exp2(mx[h] - mn);
+                float acc = sm[h] * f;
+#pragma unroll
+                for (int ct = 0; ct < 4; ++ct) {
+                    oa[ct][2 * h] *= f;
+                    oa[ct][2 * h + 1] *= f;
+                }
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    // 2^(s - m); a masked key (-inf) or a row without a valid key yet gives 0
+                    const float p0 = mn == -INFINITY ? 0.f : fast_exp2(s[nt][2 * h] - mn);
+                    const float p1 = mn == -INFINITY ? 0.f : fast_exp2(s[nt][2 * h + 1] - mn);
+                    s[nt][2 * h] = p0;
+                    s[nt][2 * h + 1] = p1;
+                    acc += p0 + p1;
+                }
+                sm[h] = acc;
+                mx[h] = mn;
+            }
+            // O' += P V over this chunk's 32 keys (P as bf16 high + low parts)
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int nt = 2 * ks + u;
+                    tc_split(s[nt][0], s[nt][1], hi[2 * u], lo[2 * u]);
+                    tc_split(s[nt][2], s[nt][3], hi[2 * u + 1], lo[2 * u + 1]);
+                }
+#pragma unroll
+                for (int cp2 = 0; cp2 < 2; ++cp2) {
+                    const int key = kc * 32 + 16 * ks + (lane & 7) + 8 * (mat & 1), chunk = 2 * cp2 + (mat >> 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(b0, b1, b2, b3, sV + tc_sw64(key, chunk));
+                    mma_bf16_16816(oa[2 * cp2], hi, b0, b1);
+                    mma_bf16_16816(oa[2 * cp2], lo, b0, b1);
+                    mma_bf16_16816(oa[2 * cp2 + 1], hi, b2, b3);
+                    mma_bf16_16816(oa[2 * cp2 + 1], lo, b2, b3);
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float t = sm[h];
+            t += __shfl_xor_sync(0xffffffffu, t, 1);
+            t += __shfl_xor_sync(0xffffffffu, t, 2);
+            lse[h] = t > 0.f ? mx[h] + log2f(t) : INFINITY;  // no valid key: probabilities 0
+            // dO . O' of row g + 8 h, this thread's 8 channels, then the quad
+            const int row = r0 + g + 8 * h;
+            float dd = 0.f;
+#pragma unroll
+            for (int ct = 0; ct < 4; ++ct) {
+                // channels 8 ct + 2 tq, + 1: 16-byte chunk ct of the row, bytes 4 tq .. 4 tq + 3
+                const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162 *>(sO + tc_sw64(row, ct) + 4 * tq);
+                const float2 df = __bfloat1622float2(d2);
+                dd = fmaf(df.x, oa[ct][2 * h], fmaf(df.y, oa[ct][2 * h + 1], dd));
+            }
+            dd += __shfl_xor_sync(0xffffffffu, dd, 1);
+            dd += __shfl_xor_sync(0xffffffffu, dd, 2);
+            D[h] = t > 0.f ? dd / t : 0.f;
+        }
+        // probabilities and dA of chunk kc
+        auto probs = [&](int kc, float (&a)[4][4], float (&da)[4][4]) {
+            logits(kc, a);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) a[nt][e] = fast_exp2(a[nt][e] - lse[e >> 1]);
+            chunk_mma(ado, sV, kc, da);
+        };
+        // pass 2: dS and dQ += dS K (keys as the contraction index)
+        for (int kc = 0; kc < nch; ++kc) {
+            float a[4][4], da[4][4];
+            probs(kc, a, da);
+            dq_chunk(kc, a, da, D, dqa);
         }
     }
 #pragma unroll
