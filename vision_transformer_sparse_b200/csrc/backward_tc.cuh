@@ -16,9 +16,11 @@
 //       list of (query region, slot) entries e = p * topk + a that route to it, ascending
 //       (one warp ranks the entries 32 at a time);
 //   bwd_tc_query_kernel: one CTA per (image, query region, head), a warp per 16 queries.
-//       Two passes over the keys in chunks of 32, recomputing S = Q K^T: the row statistics
-//       and O' = sum 2^(s - m) V (online), hence D = dO . O' / l = sum A dA; then dA = dO V^T,
-//       dS and dQ = scale dS K. Stores dq and, per query, (lse, D) for the key side;
+//       Up to 64 keys: S = Q K^T and dA = dO V^T of both 32-key chunks in registers, the
+//       row statistics and A from one set of exponentials, D = sum A dA, then dS and
+//       dQ = scale dS K. More keys: two passes over the chunks, recomputing S: the row
+//       statistics and O' = sum 2^(s - m) V (online), hence D = dO . O' / l = sum A dA;
+//       then dA, dS and dQ. Stores dq and, per query, (lse, D) for the key side;
 //   bwd_tc_key_kernel: one CTA per (image, key region, head), a warp per 16 keys. For each
 //       entry of the key region's list (in list order) it recomputes S^T = K Q^T and
 //       dA^T = V dO^T for the entry's queries, then dK += dS^T Q and dV += A^T dO in
@@ -82,8 +84,8 @@ __device__ __forceinline__ void tc_split(float x0, float x1, uint32_t &hi, uint3
 // ----------------------------------------------------------------------------- routing
 
 // One CTA per image: kv_off[n][pk] .. kv_off[n][pk+1] index the entries e = p * topk + a
-// with r_idx[n][p][a] == pk, in ascending e. Thread pk scans the image's entries in order
-// (from shared memory when they fit), so the order does not depend on scheduling.
+// with r_idx[n][p][a] == pk, in ascending e. One warp walks the image's entries in order,
+// 32 at a time, so the order does not depend on scheduling.
 __global__ void __launch_bounds__(256) bwd_tc_transpose_kernel(const BwdTcParams p) {
     extern __shared__ int tr_s[];  // [P] counts, then running list positions
     const int n = blockIdx.x, E = p.P * p.topk;
