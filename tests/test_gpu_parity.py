@@ -108,6 +108,9 @@ SMALL = [
     (2, 16, 16, 64, 2, 2, 2, "bf16"),     # 8x8 regions, topk 2 -> 128 keys: the same, one score half
     (1, 28, 28, 192, 6, 7, 4, "bf16"),    # 6 heads (C = 192): a cluster of 6 CTAs per image
     (2, 32, 32, 160, 5, 4, 2, "bf16"),    # 5 heads (C = 160), 8x8 regions: split path
+    (2, 8, 8, 64, 2, 1, 1, "bf16"),       # S = 1: one region, every query over its whole image
+    (1, 16, 16, 64, 2, 16, 256, "bf16"),  # S = 16, topk = 256: one-token regions, dense limit
+    (1, 16, 16, 64, 2, 16, 256, "f32"),   # the same in float32
 ]
 
 
