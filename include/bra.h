@@ -245,8 +245,8 @@ int bra_block(const void *x, const void *pos_w, const void *pos_b, const void *l
  * LCE only. Given dout = dL/dout (N,H,W,C) in `dtype` and the forward's r_idx, writes
  *   dq, dk, dv: (N,H,W,C) float32;  dlce_w: (C,5,5) float32;  dlce_b: (C) float32.
  * The attention softmax is recomputed from q and k.
- *   - BRA_BF16 with 32 channels per head, q, k, v and dout 16-byte aligned and dq, dk,
- *     dv 8-byte aligned: tensor-core kernels (bf16 products, float32 accumulation; the
+ *   - BRA_BF16 with 32 channels per head, q, k, v, dout and dv 16-byte aligned and dq,
+ *     dk 8-byte aligned: tensor-core kernels (bf16 products, float32 accumulation; the
  *     probabilities and dS enter their products as bf16 high + low parts).
  *     Deterministic: every output element has one writer and every sum a fixed order,
  *     so repeated calls give identical bits. Scratch (the transposed routing, per-query

@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
 // entry's Q and dO tiles (Rp = w2 rounded up to 16 rows) and its per-query (lse, D).
 __host__ __device__ inline int bwd_tc_key_smem(int nw, int w2) {
     const int Rp = (w2 + 15) & ~15;
-    return 2 * nw * 16 * 64 + 2 * (2 * Rp * 64 + Rp * 8) + 128;
+    return 2 * nw * 16 * 64 + 2 * (2 * Rp * 64 + Rp * 8) + nw * 16 * 128 + 128;
 }
 
 __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const BwdTcParams p) {
@@ -475,6 +475,15 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
         const size_t g = ok ? tc_pix(p, n, pk, row) + c0 + 8 * ch : 0;
         cp_async16_s(k_s + tc_sw64(row, ch), p.k + g, ok);
         cp_async16_s(v_s + tc_sw64(row, ch), p.v + g, ok);
+    }
+    // the LCE part of dv already stored for these keys (nw * 16 rows of 32 floats after the
+    // two entry stages), copied now and added to the attention part at the end
+    const uint32_t l_s = smem_u32(stage0 + 2 * stage_bytes);
+    for (int i = tid; i < Kp * 8; i += nthr) {
+        const int row = i >> 3, ch = i & 7;
+        const bool ok = row < p.w2;
+        const size_t g = ok ? tc_pix(p, n, pk, row) + c0 + 4 * ch : 0;
+        cp_async16_s(l_s + row * 128 + ch * 16, p.dv + g, ok);
     }
     // the entry's queries (query region pr): Q and dO rows, (lse, D) per row, all as
     // asynchronous copies (padding rows: lse = +inf, D = 0, written directly)
@@ -583,6 +592,8 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
         __syncthreads();  // the stage is read: the next prefetch may overwrite it
     }
     cp_async_wait<0>();
+    __syncthreads();  // every thread's copy of the LCE part has landed
+    const float *sL = reinterpret_cast<const float *>(stage0 + 2 * stage_bytes);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int row = k0 + g + 8 * h;
@@ -592,9 +603,8 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
         for (int ct = 0; ct < 4; ++ct) {
             const int c = 8 * ct + 2 * tq;
             *reinterpret_cast<float2 *>(p.dk + o + c) = make_float2(p.scale * dka[ct][2 * h], p.scale * dka[ct][2 * h + 1]);
-            float2 *dv = reinterpret_cast<float2 *>(p.dv + o + c);
-            const float2 lce = *dv;
-            *dv = make_float2(lce.x + dva[ct][2 * h], lce.y + dva[ct][2 * h + 1]);
+            const float2 lce = *reinterpret_cast<const float2 *>(sL + row * 32 + c);
+            *reinterpret_cast<float2 *>(p.dv + o + c) = make_float2(lce.x + dva[ct][2 * h], lce.y + dva[ct][2 * h + 1]);
         }
     }
 }

@@ -1651,9 +1651,9 @@ static int backward_impl(const void *q, const void *k, const void *v, const void
         return BRA_ERR_ALIGN;
     int sms = 0;
     if ((rc = sm_count(&sms))) return rc;
-    // the tensor-core kernels move 16-byte pieces of q, k, v and dout and store float2 gradients
+    // the tensor-core kernels move 16-byte pieces of q, k, v, dout and dv and store float2 gradients
     const bool tc = dtype == BRA_BF16 && s.d == 32 && aligned(q, 16) && aligned(k, 16) && aligned(v, 16) &&
-                    aligned(dout, 16) && aligned(dq, 8) && aligned(dk, 8) && aligned(dv, 8);
+                    aligned(dout, 16) && aligned(dq, 8) && aligned(dk, 8) && aligned(dv, 16);
     if (tc) return backward_tc(s, q, k, v, lce_w, r_idx, dout, dq, dk, dv, dlce_w, dlce_b, st, sync);
     int *flag = nullptr;  // per call (read back here), or the library's device flag
     if (sync ? cudaMallocAsync(reinterpret_cast<void **>(&flag), sizeof(int), st) != cudaSuccess
