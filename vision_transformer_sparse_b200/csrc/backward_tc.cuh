@@ -172,14 +172,13 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
         sRoute[a] = r;
     }
     __syncthreads();
-    for (int w = tid; w < nch; w += nthr) {
-        uint32_t mk = 0;
-        for (int b = 0; b < 32; ++b) {
-            const int j = w * 32 + b;
-            if (j < p.L && sRoute[p.div_w2.div((uint32_t)j)] >= 0) mk |= 1u << b;
+    if (tid < 32)  // warp 0: one key per lane, one ballot per 32-key chunk
+        for (int w = 0; w < nch; ++w) {
+            const int j = w * 32 + tid;
+            const bool live = j < p.L && sRoute[p.div_w2.div((uint32_t)j)] >= 0;
+            const uint32_t mk = __ballot_sync(0xffffffffu, live);
+            if (tid == 0) sMask[w] = mk;
         }
-        sMask[w] = mk;
-    }
     const uint32_t q_s = smem_u32(sQ), o_s = smem_u32(sO), k_s = smem_u32(sK), v_s = smem_u32(sV);
     for (int i = tid; i < Rp * 4; i += nthr) {
         const int row = i >> 2, ch = i & 3;
@@ -188,14 +187,17 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
         cp_async16_s(q_s + tc_sw64(row, ch), p.q + g, ok);
         cp_async16_s(o_s + tc_sw64(row, ch), p.dout + g, ok);
     }
-    for (int i = tid; i < Lp * 4; i += nthr) {
-        const int j = i >> 2, ch = i & 3;
+    // two 16-byte pieces of a key row per step: one address for four copies
+    for (int i = tid; i < Lp * 2; i += nthr) {
+        const int j = i >> 1, ch = 2 * (i & 1);
         const int a = (int)p.div_w2.div((uint32_t)j), t = j - a * p.w2;
         const int r = j < p.L ? sRoute[a] : -1;
         const bool ok = r >= 0;
         const size_t g = ok ? tc_pix(p, n, r, t) + c0 + 8 * ch : 0;
         cp_async16_s(k_s + tc_sw64(j, ch), p.k + g, ok);
+        cp_async16_s(k_s + tc_sw64(j, ch + 1), p.k + g + 8, ok);
         cp_async16_s(v_s + tc_sw64(j, ch), p.v + g, ok);
+        cp_async16_s(v_s + tc_sw64(j, ch + 1), p.v + g + 8, ok);
     }
     cp_async_commit();
     cp_async_wait<0>();
@@ -491,12 +493,14 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
         unsigned char *st = stage0 + s * stage_bytes;
         const uint32_t sq = smem_u32(st), so = sq + Rp * 64;
         float2 *sst = reinterpret_cast<float2 *>(st + 2 * Rp * 64);
-        for (int i = tid; i < Rp * 4; i += nthr) {
-            const int row = i >> 2, ch = i & 3;
+        for (int i = tid; i < Rp * 2; i += nthr) {  // two 16-byte pieces of a row per step
+            const int row = i >> 1, ch = 2 * (i & 1);
             const bool ok = row < p.w2;
             const size_t g = ok ? tc_pix(p, n, pr, row) + c0 + 8 * ch : 0;
             cp_async16_s(sq + tc_sw64(row, ch), p.q + g, ok);
+            cp_async16_s(sq + tc_sw64(row, ch + 1), p.q + g + 8, ok);
             cp_async16_s(so + tc_sw64(row, ch), p.dout + g, ok);
+            cp_async16_s(so + tc_sw64(row, ch + 1), p.dout + g + 8, ok);
         }
         for (int row = tid; row < Rp; row += nthr) {
             if (row < p.w2)
