@@ -180,12 +180,14 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_query_kernel(const
             if (tid == 0) sMask[w] = mk;
         }
     const uint32_t q_s = smem_u32(sQ), o_s = smem_u32(sO), k_s = smem_u32(sK), v_s = smem_u32(sV);
-    for (int i = tid; i < Rp * 4; i += nthr) {
-        const int row = i >> 2, ch = i & 3;
+    for (int i = tid; i < Rp * 2; i += nthr) {  // two 16-byte pieces of a row per step
+        const int row = i >> 1, ch = 2 * (i & 1);
         const bool ok = row < p.w2;
         const size_t g = ok ? tc_pix(p, n, pr, row) + c0 + 8 * ch : 0;
         cp_async16_s(q_s + tc_sw64(row, ch), p.q + g, ok);
+        cp_async16_s(q_s + tc_sw64(row, ch + 1), p.q + g + 8, ok);
         cp_async16_s(o_s + tc_sw64(row, ch), p.dout + g, ok);
+        cp_async16_s(o_s + tc_sw64(row, ch + 1), p.dout + g + 8, ok);
     }
     // two 16-byte pieces of a key row per step: one address for four copies
     for (int i = tid; i < Lp * 2; i += nthr) {
@@ -471,21 +473,24 @@ __global__ void __launch_bounds__(32 * kBwdTcMaxWarps) bwd_tc_key_kernel(const B
     const int e0 = off[pk], cnt = off[pk + 1] - e0;
     const int *list = p.kv_list + (size_t)n * p.P * p.topk + e0;
     const uint32_t k_s = smem_u32(sK), v_s = smem_u32(sV);
-    for (int i = tid; i < Kp * 4; i += nthr) {
-        const int row = i >> 2, ch = i & 3;
+    for (int i = tid; i < Kp * 2; i += nthr) {  // two 16-byte pieces of a row per step
+        const int row = i >> 1, ch = 2 * (i & 1);
         const bool ok = row < p.w2;
         const size_t g = ok ? tc_pix(p, n, pk, row) + c0 + 8 * ch : 0;
         cp_async16_s(k_s + tc_sw64(row, ch), p.k + g, ok);
+        cp_async16_s(k_s + tc_sw64(row, ch + 1), p.k + g + 8, ok);
         cp_async16_s(v_s + tc_sw64(row, ch), p.v + g, ok);
+        cp_async16_s(v_s + tc_sw64(row, ch + 1), p.v + g + 8, ok);
     }
     // the LCE part of dv already stored for these keys (nw * 16 rows of 32 floats after the
     // two entry stages), copied now and added to the attention part at the end
     const uint32_t l_s = smem_u32(stage0 + 2 * stage_bytes);
-    for (int i = tid; i < Kp * 8; i += nthr) {
-        const int row = i >> 3, ch = i & 7;
+    for (int i = tid; i < Kp * 2; i += nthr) {  // four 16-byte pieces of a row per step
+        const int row = i >> 1, ch = 4 * (i & 1);
         const bool ok = row < p.w2;
         const size_t g = ok ? tc_pix(p, n, pk, row) + c0 + 4 * ch : 0;
-        cp_async16_s(l_s + row * 128 + ch * 16, p.dv + g, ok);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) cp_async16_s(l_s + row * 128 + (ch + u) * 16, p.dv + g + 4 * u, ok);
     }
     // the entry's queries (query region pr): Q and dO rows, (lse, D) per row, all as
     // asynchronous copies (padding rows: lse = +inf, D = 0, written directly)
